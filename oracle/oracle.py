@@ -1,0 +1,176 @@
+"""ctypes front end of the BitLinear oracle (``bitlinear_oracle.cpp``).
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the benchmark's
+CPU-baseline leg may import this module; the library never does.
+
+Each function mirrors one step of the BitLinear forward of BitNet b1.58 ("The Era of
+1-bit LLMs", dmarx anthology record LIT-380, Key takeaways bullets 1 and 4): absmean
+ternary weights, per-token absmax int8 activations, the integer contraction and the
+rescale. Inputs are numpy arrays (fp32, or bf16 carried as uint16 bit patterns); the
+work happens in the single-threaded C++ code.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "bitlinear_oracle.cpp")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+F32 = 0
+BF16 = 1
+
+GXX_FLAGS = ["-O2", "-std=c++17", "-ffp-contract=off", "-fno-fast-math", "-shared", "-fPIC"]
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle into ``oracle/liboracle.so`` (plain g++, no GPU)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        subprocess.check_call(["g++", *GXX_FLAGS, _SRC, "-o", _LIB])
+    return _LIB
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        _lib = ctypes.CDLL(build())
+        p, i64, f32, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_int
+        _lib.oracle_absmean.argtypes = [p, i32, i64, p]
+        _lib.oracle_absmean.restype = i32
+        _lib.oracle_ternarize.argtypes = [p, i32, i64, f32, f32, p]
+        _lib.oracle_ternarize.restype = i32
+        _lib.oracle_pack.argtypes = [p, i64, i64, p]
+        _lib.oracle_pack.restype = None
+        _lib.oracle_unpack.argtypes = [p, i64, i64, p]
+        _lib.oracle_unpack.restype = i32
+        _lib.oracle_quantize_acts.argtypes = [p, i32, i64, i64, p, p]
+        _lib.oracle_quantize_acts.restype = i32
+        _lib.oracle_contract_i32.argtypes = [p, p, i64, i64, i64, p]
+        _lib.oracle_contract_i32.restype = None
+        _lib.oracle_rescale.argtypes = [p, p, f32, i64, i64, p]
+        _lib.oracle_rescale.restype = None
+        _lib.oracle_to_bf16.argtypes = [p, i64, p]
+        _lib.oracle_to_bf16.restype = None
+    return _lib
+
+
+def _ptr(a: np.ndarray) -> int:
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data
+
+
+def _as_input(a: np.ndarray) -> tuple[np.ndarray, int]:
+    """fp32 arrays pass as fp32; uint16 arrays are bf16 bit patterns."""
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.float32:
+        return a, F32
+    if a.dtype == np.uint16:
+        return a, BF16
+    raise TypeError(f"oracle inputs are float32 or bf16-as-uint16, got {a.dtype}")
+
+
+def absmean(W: np.ndarray) -> np.float32:
+    """gamma = mean|W|: exact sum of |w|, rounded once to double, / n, rounded to fp32."""
+    W, dt = _as_input(W)
+    out = np.zeros(1, np.float32)
+    rc = lib().oracle_absmean(_ptr(W), dt, W.size, _ptr(out))
+    if rc != 0:
+        raise ValueError("non-finite weight")
+    return out[0]
+
+
+def ternarize(W: np.ndarray, gamma: float, eps: float) -> np.ndarray:
+    """c = RoundClip(w / (gamma + eps), -1, 1), fp32 quotient, ties to even."""
+    W, dt = _as_input(W)
+    codes = np.zeros(W.shape, np.int8)
+    rc = lib().oracle_ternarize(_ptr(W), dt, W.size, float(gamma), float(eps), _ptr(codes))
+    if rc != 0:
+        raise RuntimeError("FPU rounding mode is not round-to-nearest")
+    return codes
+
+
+def pack(codes: np.ndarray) -> np.ndarray:
+    """2-bit packing of an int8 [N][K] code array (K % 16 == 0) -> uint8 [N][K/4]."""
+    codes = np.ascontiguousarray(codes, dtype=np.int8)
+    N, K = codes.shape
+    assert K % 16 == 0
+    out = np.zeros((N, K // 4), np.uint8)
+    lib().oracle_pack(_ptr(codes), N, K, _ptr(out))
+    return out
+
+
+def unpack(packed: np.ndarray, K: int) -> np.ndarray:
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    N = packed.shape[0]
+    assert packed.shape[1] * 4 == K
+    codes = np.zeros((N, K), np.int8)
+    if lib().oracle_unpack(_ptr(packed), N, K, _ptr(codes)) != 0:
+        raise ValueError("packed buffer holds the unused 2-bit code 3")
+    return codes
+
+
+def quantize_weights(W: np.ndarray, eps: float = 1e-5) -> tuple[np.ndarray, np.float32]:
+    """absmean -> ternarize -> pack. Returns (packed uint8 [N][K/4], gamma)."""
+    gamma = absmean(W)
+    return pack(ternarize(W, gamma, eps)), gamma
+
+
+def quantize_acts(x: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """Per-token absmax int8: returns (q int8 [M][K], scale fp32 [M] = absmax/127)."""
+    x, dt = _as_input(x)
+    M, K = x.shape
+    q = np.zeros((M, K), np.int8)
+    s = np.zeros(M, np.float32)
+    rc = lib().oracle_quantize_acts(_ptr(x), dt, M, K, _ptr(q), _ptr(s))
+    if rc == 1:
+        raise ValueError("non-finite activation")
+    if rc != 0:
+        raise RuntimeError("FPU rounding mode is not round-to-nearest")
+    return q, s
+
+
+def contract_i32(q: np.ndarray, codes: np.ndarray) -> np.ndarray:
+    """acc[t,n] = sum_{c=+1} q[t,k] - sum_{c=-1} q[t,k] (int32)."""
+    q = np.ascontiguousarray(q, dtype=np.int8)
+    codes = np.ascontiguousarray(codes, dtype=np.int8)
+    M, K = q.shape
+    N = codes.shape[0]
+    assert codes.shape[1] == K
+    acc = np.zeros((M, N), np.int32)
+    lib().oracle_contract_i32(_ptr(q), _ptr(codes), M, N, K, _ptr(acc))
+    return acc
+
+
+def rescale(acc: np.ndarray, scale: np.ndarray, gamma: float) -> np.ndarray:
+    """y = float(acc) * (scale_t * gamma), fp32."""
+    acc = np.ascontiguousarray(acc, dtype=np.int32)
+    scale = np.ascontiguousarray(scale, dtype=np.float32)
+    M, N = acc.shape
+    y = np.zeros((M, N), np.float32)
+    lib().oracle_rescale(_ptr(acc), _ptr(scale), float(gamma), M, N, _ptr(y))
+    return y
+
+
+def to_bf16(y: np.ndarray) -> np.ndarray:
+    """fp32 -> bf16 bit patterns (uint16), round half to even."""
+    y = np.ascontiguousarray(y, dtype=np.float32)
+    out = np.zeros(y.shape, np.uint16)
+    lib().oracle_to_bf16(_ptr(y), y.size, _ptr(out))
+    return out
+
+
+def forward(x: np.ndarray, packed: np.ndarray, gamma: float, out: str = "f32") -> np.ndarray:
+    """Whole BitLinear forward from packed weights: y [M][N] fp32 (or bf16 bits)."""
+    K = x.shape[1]
+    q, s = quantize_acts(x)
+    acc = contract_i32(q, unpack(packed, K))
+    y = rescale(acc, s, gamma)
+    return to_bf16(y) if out == "bf16" else y
