@@ -1,0 +1,138 @@
+/*
+ * bitlinear.h - C ABI of the B200 (sm_100a) BitLinear forward library.
+ *
+ * What it computes: the BitLinear layer of BitNet b1.58 ("The Era of 1-bit LLMs: All
+ * Large Language Models are in 1.58 Bits"). In the words of the dmarx anthology record
+ * LIT-380 (Key takeaways, bullet 1), nn.Linear is replaced by BitLinear, the weights are
+ * constrained to {-1, 0, +1} by an absmean quantization function and the activations are
+ * 8-bit; bullet 4 says the matrix product becomes integer addition. The searcharxiv.com
+ * abstract page (Abstract) states that every weight is ternary. The pages give no formula;
+ * the library implements the plainest reading:
+ *
+ *   gamma    = mean |W|                                    (fp32; exact sum, rounded once)
+ *   c[n,k]   = RoundClip(W[n,k] / (gamma + eps), -1, 1)     (fp32 quotient, ties to even)
+ *   a_t      = max_k |x[t,k]|,  r_t = 127 / a_t,  s_t = a_t / 127           (fp32)
+ *   q[t,k]   = clip(rne(x[t,k] * r_t), -127, 127)           (0 if a_t == 0 or x == 0)
+ *   acc[t,n] = sum_k c[n,k] * q[t,k]                         (exact int32)
+ *   y[t,n]   = float(acc[t,n]) * (s_t * gamma)               (fp32, or its bf16 RNE)
+ *
+ * Shapes follow nn.Linear: W [N][K] (out x in), x [M][K], y [M][N], all row-major.
+ *
+ * Packed weight format ("1.58 bit ... 2 bits in practice", hackerpaper HN page,
+ * thread 17): trit c is stored as the 2-bit code u = c + 1 (0, 1, 2; 3 is never
+ * written). Row n occupies K/4 bytes at byte offset n*K/4. The little-endian 32-bit word
+ * g of a row holds trits k = 16g .. 16g+15; trit k = 16g + 4j + i (i, j in 0..3) is in
+ * bits 8i+2j .. 8i+2j+1 of that word. (Shifting the word right by 2j and masking with
+ * 0x03030303 yields trits 16g+4j .. 16g+4j+3 as four consecutive bytes.)
+ *
+ * Conventions for every entry point:
+ *  - Ownership: the caller allocates and frees every buffer. Device pointers must stay
+ *    valid until the work queued on `stream` has finished. The library keeps no pointer
+ *    after a call returns and never allocates or frees device memory in these calls.
+ *  - Execution: work is queued asynchronously on `stream` (a cudaStream_t; NULL is the
+ *    legacy default stream) on the current CUDA device. Argument errors are reported
+ *    synchronously, before anything is queued. A failed launch returns BL_ERR_CUDA.
+ *    Faults found on the device (non-finite input, a wait that timed out) are recorded
+ *    in a per-device status word read by bitlinear_get_device_status().
+ *  - Shapes: M, N >= 1; K >= 64 and K % 64 == 0; M*K, N*K and M*N below 2^31.
+ *    Otherwise BL_ERR_UNSUPPORTED_SHAPE.
+ *  - Alignment: every device pointer 16-byte aligned, else BL_ERR_MISALIGNED.
+ *  - Thread safety: calls on different streams may run concurrently; they share only the
+ *    device status word.
+ */
+#ifndef BITLINEAR_H_
+#define BITLINEAR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BL_OK = 0,
+  BL_ERR_INVALID_ARG = 1,       /* null pointer, bad dtype, eps < 0 or not finite */
+  BL_ERR_UNSUPPORTED_SHAPE = 2, /* shape outside the limits above */
+  BL_ERR_MISALIGNED = 3,        /* a pointer is not 16-byte aligned */
+  BL_ERR_CUDA = 4,              /* a CUDA runtime call or kernel launch failed */
+  BL_ERR_TIMEOUT = 5,           /* a device-side wait exceeded its limit (status word) */
+  BL_ERR_NONFINITE = 6,         /* Inf or NaN in W or x (status word) */
+  BL_ERR_WORKSPACE = 7          /* workspace missing or smaller than required */
+} bl_status;
+
+typedef enum { BL_F32 = 0, BL_BF16 = 1, BL_I32 = 2 } bl_dtype;
+
+/* Device bytes of workspace that bitlinear_quantize_weights (for N x K) and
+ * bitlinear_forward / bitlinear_contract_i32 (for M x N x K) need; the largest of the
+ * three. Pure host function. Returns 0 for shapes the library rejects. */
+size_t bitlinear_workspace_size(int M, int N, int K);
+
+/* Absmean ternary weight quantization (LIT-380 bullet 1; Abstract of the searcharxiv.com
+ * page): gamma = mean|W| over all N*K weights, then every weight becomes the code
+ * RoundClip(w / (gamma + eps), -1, 1), packed 2 bits per trit.
+ *   W       device, [N][K] row-major, fp32 (w_dtype BL_F32) or bf16 (BL_BF16); read only.
+ *   eps     >= 0, finite (1e-5 is the usual choice); added to gamma in fp32.
+ *   packed  device, N*K/4 bytes, written in the packed format above.
+ *   gamma   device, one float, written.
+ *   ws      device workspace of at least bitlinear_workspace_size(1, N, K) bytes; its
+ *           contents on entry do not matter and are clobbered.
+ * gamma is the exact sum of |w| rounded once to double, divided by N*K in double and
+ * rounded to float, so it does not depend on launch shape or summation order.
+ * Inf/NaN in W sets BL_ERR_NONFINITE in the device status word (outputs undefined). */
+bl_status bitlinear_quantize_weights(const void* W, int w_dtype, int N, int K, float eps,
+                                     uint8_t* packed, float* gamma, void* ws,
+                                     size_t ws_bytes, void* stream);
+
+/* Per-token absmax int8 activation quantization ("activations are 8-bit", LIT-380
+ * bullet 1): q = clip(rne(x * (127 / a_t)), -127, 127), scale_t = a_t / 127.
+ *   x      device, [M][K], fp32 or bf16 (x_dtype); read only.
+ *   xq     device, [M][K] int8, written.
+ *   scale  device, [M] fp32, written (0 for an all-zero row).
+ * Inf/NaN in x sets BL_ERR_NONFINITE in the device status word. */
+bl_status bitlinear_quantize_acts(const void* x, int x_dtype, int M, int K, int8_t* xq,
+                                  float* scale, void* stream);
+
+/* The BitLinear forward: quantize x per token, contract with the packed ternary weights
+ * in exact int32 ("integer addition", LIT-380 bullet 4) and rescale by s_t * gamma.
+ *   x       device, [M][K], fp32 or bf16 (x_dtype).
+ *   packed  device, [N][K/4] packed codes from bitlinear_quantize_weights.
+ *   gamma   device, one float.
+ *   y       device, [M][N], y_dtype BL_F32 or BL_BF16 (RNE of the fp32 value).
+ *   ws      device workspace of at least bitlinear_workspace_size(M, N, K) bytes.
+ * Small M runs one CUDA-core kernel that quantizes x in its prologue; larger M quantizes
+ * x into the workspace and runs the tcgen05 int8 tensor-core GEMM. Both give the same
+ * bits. */
+bl_status bitlinear_forward(const void* x, int x_dtype, const uint8_t* packed,
+                            const float* gamma, void* y, int y_dtype, int M, int N, int K,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/* The integer stage alone (test hook, same kernels as bitlinear_forward):
+ * acc[t,n] = sum_k c[n,k] * xq[t,k].
+ *   xq      device, [M][K] int8 (values in [-127, 127]).
+ *   packed  device, [N][K/4].
+ *   acc     device, [M][N] int32, written.
+ *   ws      device workspace of at least bitlinear_workspace_size(M, N, K) bytes. */
+bl_status bitlinear_contract_i32(const int8_t* xq, const uint8_t* packed, int32_t* acc,
+                                 int M, int N, int K, void* ws, size_t ws_bytes,
+                                 void* stream);
+
+/* Waits for `stream`, then reads and clears the current device's status word:
+ * BL_OK, BL_ERR_NONFINITE or BL_ERR_TIMEOUT (the first recorded wins in that order of
+ * severity: TIMEOUT over NONFINITE). BL_ERR_CUDA if the wait or the read fails. */
+bl_status bitlinear_get_device_status(void* stream);
+
+/* Test hook for the bounded-wait machinery: runs one block that waits on an mbarrier no
+ * thread ever arrives on, giving up after `timeout_ns` nanoseconds (1e3 .. 5e9). The
+ * kernel then records BL_ERR_TIMEOUT in the status word and exits normally, so the
+ * context stays usable. */
+bl_status bitlinear_debug_timeout_probe(uint64_t timeout_ns, void* stream);
+
+/* Human-readable name of a status code (static string). */
+const char* bitlinear_status_string(bl_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BITLINEAR_H_ */

@@ -1,0 +1,188 @@
+"""Thin Python binding of libbitlinear.so (C ABI in include/bitlinear.h).
+
+Argument marshalling only: every step of the BitLinear forward runs in the library's
+sm_100a kernels. PyTorch supplies device memory and the current stream. There is no
+fallback: if the shared library is missing or no CUDA device is present, the calls raise.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libbitlinear.so")
+
+BL_F32, BL_BF16, BL_I32 = 0, 1, 2
+STATUS = {
+    0: "BL_OK", 1: "BL_ERR_INVALID_ARG", 2: "BL_ERR_UNSUPPORTED_SHAPE", 3: "BL_ERR_MISALIGNED",
+    4: "BL_ERR_CUDA", 5: "BL_ERR_TIMEOUT", 6: "BL_ERR_NONFINITE", 7: "BL_ERR_WORKSPACE",
+}
+
+# Every symbol declared in include/bitlinear.h.
+EXPORTS = (
+    "bitlinear_workspace_size", "bitlinear_quantize_weights", "bitlinear_quantize_acts",
+    "bitlinear_forward", "bitlinear_contract_i32", "bitlinear_get_device_status",
+    "bitlinear_debug_timeout_probe", "bitlinear_status_string",
+)
+
+
+class BitLinearError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {STATUS.get(status, status)}")
+        self.status = status
+
+
+_lib = None
+
+
+def load_library() -> ctypes.CDLL:
+    """Loads the in-tree libbitlinear.so (built by ternary_weight_linear_03_b200.build)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m ternary_weight_linear_03_b200.build`"
+            " (or __graft_entry__.build()); there is no fallback implementation")
+    lib = ctypes.CDLL(LIB_PATH)
+    p, i, f, sz, u64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_uint64
+    lib.bitlinear_workspace_size.argtypes = [i, i, i]
+    lib.bitlinear_workspace_size.restype = sz
+    lib.bitlinear_quantize_weights.argtypes = [p, i, i, i, f, p, p, p, sz, p]
+    lib.bitlinear_quantize_weights.restype = i
+    lib.bitlinear_quantize_acts.argtypes = [p, i, i, i, p, p, p]
+    lib.bitlinear_quantize_acts.restype = i
+    lib.bitlinear_forward.argtypes = [p, i, p, p, p, i, i, i, i, p, sz, p]
+    lib.bitlinear_forward.restype = i
+    lib.bitlinear_contract_i32.argtypes = [p, p, p, i, i, i, p, sz, p]
+    lib.bitlinear_contract_i32.restype = i
+    lib.bitlinear_get_device_status.argtypes = [p]
+    lib.bitlinear_get_device_status.restype = i
+    lib.bitlinear_debug_timeout_probe.argtypes = [u64, p]
+    lib.bitlinear_debug_timeout_probe.restype = i
+    lib.bitlinear_status_string.argtypes = [i]
+    lib.bitlinear_status_string.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def _check(status: int, what: str) -> None:
+    if status != 0:
+        raise BitLinearError(status, what)
+
+
+def _dev(t: torch.Tensor, name: str) -> int:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return BL_F32
+    if t.dtype == torch.bfloat16:
+        return BL_BF16
+    raise TypeError(f"unsupported dtype {t.dtype} (fp32 or bf16)")
+
+
+def _stream(stream) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def workspace_size(M: int, N: int, K: int) -> int:
+    return int(load_library().bitlinear_workspace_size(M, N, K))
+
+
+def workspace(M: int, N: int, K: int, device="cuda") -> torch.Tensor:
+    """A caller-owned device workspace large enough for (M, N, K)."""
+    n = workspace_size(M, N, K)
+    if n == 0:
+        raise BitLinearError(2, "workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def quantize_weights(W: torch.Tensor, eps: float = 1e-5, packed: torch.Tensor | None = None,
+                     gamma: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+                     stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """Absmean ternary quantization of W [N][K] -> (packed uint8 [N][K/4], gamma fp32 [1])."""
+    lib = load_library()
+    N, K = W.shape
+    if packed is None:
+        packed = torch.empty((N, K // 4), dtype=torch.uint8, device=W.device)
+    if gamma is None:
+        gamma = torch.empty(1, dtype=torch.float32, device=W.device)
+    if ws is None:
+        ws = workspace(1, N, K, W.device)
+    _check(lib.bitlinear_quantize_weights(
+        _dev(W, "W"), _dtype_code(W), N, K, float(eps), _dev(packed, "packed"),
+        _dev(gamma, "gamma"), _dev(ws, "ws"), ws.numel(), _stream(stream)),
+        "bitlinear_quantize_weights")
+    return packed, gamma
+
+
+def quantize_acts(x: torch.Tensor, stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """Per-token absmax int8: x [M][K] -> (xq int8 [M][K], scale fp32 [M])."""
+    lib = load_library()
+    M, K = x.shape
+    xq = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    scale = torch.empty(M, dtype=torch.float32, device=x.device)
+    _check(lib.bitlinear_quantize_acts(_dev(x, "x"), _dtype_code(x), M, K, _dev(xq, "xq"),
+                                       _dev(scale, "scale"), _stream(stream)),
+           "bitlinear_quantize_acts")
+    return xq, scale
+
+
+def forward(x: torch.Tensor, packed: torch.Tensor, gamma: torch.Tensor,
+            out_dtype: torch.dtype = torch.bfloat16, y: torch.Tensor | None = None,
+            ws: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """BitLinear forward: y [M][N] = rescale(int32 contraction of quantized x with W)."""
+    lib = load_library()
+    M, K = x.shape
+    N = packed.shape[0]
+    if packed.shape[1] * 4 != K:
+        raise ValueError("packed must be [N][K/4]")
+    if y is None:
+        y = torch.empty((M, N), dtype=out_dtype, device=x.device)
+    if ws is None:
+        ws = workspace(M, N, K, x.device)
+    _check(lib.bitlinear_forward(
+        _dev(x, "x"), _dtype_code(x), _dev(packed, "packed"), _dev(gamma, "gamma"), _dev(y, "y"),
+        _dtype_code(y), M, N, K, _dev(ws, "ws"), ws.numel(), _stream(stream)),
+        "bitlinear_forward")
+    return y
+
+
+def contract_i32(xq: torch.Tensor, packed: torch.Tensor, acc: torch.Tensor | None = None,
+                 ws: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Integer stage only: acc [M][N] int32 = sum_k c[n,k] * xq[t,k]."""
+    lib = load_library()
+    M, K = xq.shape
+    N = packed.shape[0]
+    if acc is None:
+        acc = torch.empty((M, N), dtype=torch.int32, device=xq.device)
+    if ws is None:
+        ws = workspace(M, N, K, xq.device)
+    _check(lib.bitlinear_contract_i32(_dev(xq, "xq"), _dev(packed, "packed"), _dev(acc, "acc"),
+                                      M, N, K, _dev(ws, "ws"), ws.numel(), _stream(stream)),
+           "bitlinear_contract_i32")
+    return acc
+
+
+def get_device_status(stream=None) -> int:
+    """Synchronizes the stream, returns and clears the device status word (0 = BL_OK)."""
+    return int(load_library().bitlinear_get_device_status(_stream(stream)))
+
+
+def debug_timeout_probe(timeout_ns: int, stream=None) -> None:
+    _check(load_library().bitlinear_debug_timeout_probe(int(timeout_ns), _stream(stream)),
+           "bitlinear_debug_timeout_probe")
+
+
+def status_string(status: int) -> str:
+    return load_library().bitlinear_status_string(status).decode()

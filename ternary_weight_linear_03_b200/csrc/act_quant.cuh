@@ -1,0 +1,131 @@
+// Per-token absmax int8 activation quantization ("activations are 8-bit", dmarx anthology
+// record LIT-380, Key takeaways bullet 1):
+//   a_t = max_k |x[t,k]|,  r_t = fl(127 / a_t),  s_t = fl(a_t / 127),
+//   q[t,k] = clip(rne(fl(x[t,k] * r_t)), -127, 127)   (0 when a_t == 0 or x == 0).
+// One block per token row; the row is read once from HBM (the second pass hits L1/L2).
+// Optionally also writes rowsum_t = sum_k q[t,k], which the tensor-core GEMM subtracts
+// from its accumulators (the packed weights are stored as c + 1, see gemm_tc.cuh).
+#pragma once
+
+#include "common.cuh"
+
+namespace bl {
+
+constexpr int kAqThreads = 256;
+
+// Loads 8 consecutive elements (one 16-byte bf16 vector or two fp32 vectors) as floats.
+template <bool kBf16>
+__device__ __forceinline__ void load8(const void* row, int c, float (&v)[8]) {
+  if (kBf16) {
+    const uint4 p = reinterpret_cast<const uint4*>(row)[c];
+    const uint32_t h[4] = {p.x, p.y, p.z, p.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      v[2 * q] = __uint_as_float(h[q] << 16);
+      v[2 * q + 1] = __uint_as_float(h[q] & 0xffff0000u);
+    }
+  } else {
+    const float4 a = reinterpret_cast<const float4*>(row)[2 * c];
+    const float4 b = reinterpret_cast<const float4*>(row)[2 * c + 1];
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+}
+
+__device__ __forceinline__ float block_max(float v, float* red) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  v = (lane < static_cast<int>(blockDim.x >> 5)) ? red[lane] : 0.0f;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+  return v;
+}
+
+__device__ __forceinline__ int block_sum(int v, int* red) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  v = (lane < static_cast<int>(blockDim.x >> 5)) ? red[lane] : 0;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  return v;
+}
+
+// Absolute value as a plain sign-bit clear (exact); NaN stays NaN and is caught by the
+// finiteness test on the row maximum.
+__device__ __forceinline__ float abs_bits(float x) {
+  return __uint_as_float(__float_as_uint(x) & 0x7fffffffu);
+}
+
+// grid = M blocks, K % 8 == 0. rowsum may be null.
+template <bool kBf16>
+__global__ void __launch_bounds__(kAqThreads) act_quant_kernel(
+    const void* __restrict__ x, int K, int8_t* __restrict__ xq, float* __restrict__ scale,
+    int* __restrict__ rowsum) {
+  __shared__ float redf[32];
+  __shared__ int redi[32];
+  const int t = blockIdx.x;
+  const char* row = static_cast<const char*>(x) + static_cast<size_t>(t) * K * (kBf16 ? 2 : 4);
+  const int nc = K / 8;
+  float a = 0.0f;
+  bool bad = false;
+  for (int c = threadIdx.x; c < nc; c += blockDim.x) {
+    float v[8];
+    load8<kBf16>(row, c, v);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float m = abs_bits(v[i]);
+      bad |= !(m <= 3.4028234663852886e38f);
+      a = fmaxf(a, m);
+    }
+  }
+  if (bad) record_status(kStatusNonfinite);
+  a = block_max(a, redf);
+  const float r = (a > 0.0f) ? __fdiv_rn(127.0f, a) : 0.0f;
+  int8_t* qrow = xq + static_cast<size_t>(t) * K;
+  int sum = 0;
+  for (int c = threadIdx.x; c < nc; c += blockDim.x) {
+    float v[8];
+    load8<kBf16>(row, c, v);
+    uint32_t lo = 0u, hi = 0u;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int q = (a > 0.0f) ? quant_i8(v[i], r) : 0;
+      sum += q;
+      const uint32_t b = static_cast<uint32_t>(q) & 0xffu;
+      if (i < 4) lo |= b << (8 * i); else hi |= b << (8 * (i - 4));
+    }
+    reinterpret_cast<uint2*>(qrow)[c] = make_uint2(lo, hi);
+  }
+  if (threadIdx.x == 0) scale[t] = (a > 0.0f) ? __fdiv_rn(a, 127.0f) : 0.0f;
+  if (rowsum != nullptr) {
+    sum = block_sum(sum, redi);
+    if (threadIdx.x == 0) rowsum[t] = sum;
+  }
+}
+
+// rowsum_t = sum_k xq[t,k] for int8 input given directly (the integer test hook).
+__global__ void __launch_bounds__(kAqThreads) rowsum_i8_kernel(const int8_t* __restrict__ xq,
+                                                              int K, int* __restrict__ rowsum) {
+  __shared__ int redi[32];
+  const int t = blockIdx.x;
+  const int4* row = reinterpret_cast<const int4*>(xq + static_cast<size_t>(t) * K);
+  int sum = 0;
+  for (int c = threadIdx.x; c < K / 16; c += blockDim.x) {
+    const int4 p = row[c];
+    const int w[4] = {p.x, p.y, p.z, p.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) sum = __dp4a(w[i], 0x01010101, sum);
+  }
+  sum = block_sum(sum, redi);
+  if (threadIdx.x == 0) rowsum[t] = sum;
+}
+
+}  // namespace bl

@@ -1,0 +1,356 @@
+// C ABI of the BitLinear library (declared in include/bitlinear.h): argument checks,
+// workspace layout, kernel selection and launches. One translation unit holds every
+// kernel so that the device status word is a single object per device.
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/bitlinear.h"
+#include "act_quant.cuh"
+#include "common.cuh"
+#include "gemm_tc.cuh"
+#include "gemv.cuh"
+#include "weight_quant.cuh"
+
+namespace {
+
+using bl::WqWorkspace;
+
+constexpr int kGemvMaxM = 4;            // M above this runs the tensor-core GEMM
+constexpr int kGemvMaxSmem = 200 * 1024;  // xq rows held in shared memory by the GEMV
+constexpr unsigned long long kWaitLimitNs = 4000000000ull;  // 4 s per mbarrier wait
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool shape_ok(long long M, long long N, long long K) {
+  if (M < 1 || N < 1 || K < 64 || (K % 64) != 0) return false;
+  const long long lim = 1ll << 31;
+  return M * K < lim && N * K < lim && M * N < lim;
+}
+
+int num_sms() {
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (sms <= 0) sms = 148;
+  }
+  return sms;
+}
+
+bool use_gemv(int M, int K) { return M <= kGemvMaxM && static_cast<long long>(M) * K <= kGemvMaxSmem; }
+
+// Workspace layout of the forward / contract paths that run the GEMM:
+//   [xq M*K int8][scale M fp32][rowsum M int32], each 256-byte aligned.
+struct FwdWs {
+  int8_t* xq;
+  float* scale;
+  int* rowsum;
+  size_t bytes;
+};
+FwdWs fwd_ws_layout(void* base, int M, int K) {
+  FwdWs w{};
+  const size_t a = align_up(static_cast<size_t>(M) * K, 256);
+  const size_t b = align_up(static_cast<size_t>(M) * 4, 256);
+  char* p = static_cast<char*>(base);
+  w.xq = reinterpret_cast<int8_t*>(p);
+  w.scale = reinterpret_cast<float*>(p + a);
+  w.rowsum = reinterpret_cast<int*>(p + a + b);
+  w.bytes = a + 2 * b;
+  return w;
+}
+
+bl_status launch_status() {
+  return (cudaGetLastError() == cudaSuccess) ? BL_OK : BL_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ TMA descriptors
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D uint8 tensor [rows][cols] with row pitch `pitch` bytes, box [box_rows][box_cols].
+bool make_map_u8(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
+                 uint64_t pitch, uint32_t box_cols, uint32_t box_rows, bool swizzle128) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {pitch};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ GEMV launch
+int choose_lpr_log2(int cpr) {
+  int best = 5;
+  long long best_cost = (cpr + 31) / 32 * 32;
+  for (int l = 4; l >= 2; --l) {
+    const int L = 1 << l;
+    const long long cost = static_cast<long long>(cpr + L - 1) / L * L;
+    if (cost < best_cost) { best = l; best_cost = cost; }
+  }
+  return best;
+}
+
+template <int MT, int XM, int OM>
+bl_status launch_gemv_t(const void* x, const uint8_t* packed, const float* gamma, void* y,
+                        int N, int K, cudaStream_t s) {
+  auto kern = bl::gemv_kernel<MT, XM, OM>;
+  const int smem = MT * K;
+  static int configured_smem = -1;
+  static int blocks_per_sm = 1;
+  if (configured_smem < smem) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemvMaxSmem) !=
+        cudaSuccess)
+      return BL_ERR_CUDA;
+    configured_smem = smem;
+  }
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_per_sm, kern, bl::kGemvThreads,
+                                                    smem) != cudaSuccess ||
+      blocks_per_sm < 1)
+    blocks_per_sm = 1;
+  const int lpr_log2 = choose_lpr_log2(K / 64);
+  const long long rows_per_block = static_cast<long long>(bl::kGemvWarps) * (32 >> lpr_log2);
+  const long long need = (N + rows_per_block - 1) / rows_per_block;
+  const int grid = static_cast<int>(std::min<long long>(need, 1ll * blocks_per_sm * num_sms()));
+  kern<<<grid, bl::kGemvThreads, smem, s>>>(x, packed, gamma, y, N, K, lpr_log2);
+  return launch_status();
+}
+
+template <int XM, int OM>
+bl_status launch_gemv_m(const void* x, const uint8_t* packed, const float* gamma, void* y,
+                        int M, int N, int K, cudaStream_t s) {
+  switch (M) {
+    case 1: return launch_gemv_t<1, XM, OM>(x, packed, gamma, y, N, K, s);
+    case 2: return launch_gemv_t<2, XM, OM>(x, packed, gamma, y, N, K, s);
+    case 3: return launch_gemv_t<3, XM, OM>(x, packed, gamma, y, N, K, s);
+    case 4: return launch_gemv_t<4, XM, OM>(x, packed, gamma, y, N, K, s);
+    default: return BL_ERR_UNSUPPORTED_SHAPE;
+  }
+}
+
+template <int XM>
+bl_status launch_gemv_x(const void* x, const uint8_t* packed, const float* gamma, void* y,
+                        int y_dtype, int M, int N, int K, cudaStream_t s) {
+  switch (y_dtype) {
+    case BL_F32: return launch_gemv_m<XM, bl::kOf32>(x, packed, gamma, y, M, N, K, s);
+    case BL_BF16: return launch_gemv_m<XM, bl::kObf16>(x, packed, gamma, y, M, N, K, s);
+    case BL_I32: return launch_gemv_m<XM, bl::kOi32>(x, packed, gamma, y, M, N, K, s);
+    default: return BL_ERR_INVALID_ARG;
+  }
+}
+
+// ------------------------------------------------------------------ GEMM launch
+template <int OM>
+bl_status launch_gemm_t(const int8_t* xq, const uint8_t* packed, const int* rowsum,
+                        const float* scale, const float* gamma, void* y, int M, int N, int K,
+                        cudaStream_t s) {
+  CUtensorMap map_a, map_b;
+  if (!make_map_u8(&map_a, xq, K, M, K, bl::tc::BK, bl::tc::BM, true)) return BL_ERR_CUDA;
+  if (!make_map_u8(&map_b, packed, K / 4, N, K / 4, bl::tc::BK / 4, bl::tc::BN, false))
+    return BL_ERR_CUDA;
+  auto kern = bl::gemm_tc_kernel<OM>;
+  static bool configured = false;
+  if (!configured) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             bl::tc::SMEM_BYTES) != cudaSuccess)
+      return BL_ERR_CUDA;
+    configured = true;
+  }
+  const long long tiles = static_cast<long long>((M + bl::tc::BM - 1) / bl::tc::BM) *
+                          ((N + bl::tc::BN - 1) / bl::tc::BN);
+  const int grid = static_cast<int>(std::min<long long>(tiles, num_sms()));
+  kern<<<grid, bl::tc::THREADS, bl::tc::SMEM_BYTES, s>>>(map_a, map_b, rowsum, scale, gamma, y,
+                                                         M, N, K, kWaitLimitNs);
+  return launch_status();
+}
+
+bl_status launch_gemm(const int8_t* xq, const uint8_t* packed, const int* rowsum,
+                      const float* scale, const float* gamma, void* y, int y_dtype, int M, int N,
+                      int K, cudaStream_t s) {
+  switch (y_dtype) {
+    case BL_F32: return launch_gemm_t<0>(xq, packed, rowsum, scale, gamma, y, M, N, K, s);
+    case BL_BF16: return launch_gemm_t<1>(xq, packed, rowsum, scale, gamma, y, M, N, K, s);
+    case BL_I32: return launch_gemm_t<2>(xq, packed, rowsum, scale, gamma, y, M, N, K, s);
+    default: return BL_ERR_INVALID_ARG;
+  }
+}
+
+bl_status launch_act_quant(const void* x, int x_dtype, int M, int K, int8_t* xq, float* scale,
+                           int* rowsum, cudaStream_t s) {
+  if (x_dtype == BL_BF16)
+    bl::act_quant_kernel<true><<<M, bl::kAqThreads, 0, s>>>(x, K, xq, scale, rowsum);
+  else
+    bl::act_quant_kernel<false><<<M, bl::kAqThreads, 0, s>>>(x, K, xq, scale, rowsum);
+  return launch_status();
+}
+
+// ------------------------------------------------------------------ debug probe
+__global__ void timeout_probe_kernel(unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    bl::mbar_init(&bar, 1);
+    bl::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) bl::mbar_wait(&bar, 0u, limit_ns);  // nothing ever arrives
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t bitlinear_workspace_size(int M, int N, int K) {
+  if (!shape_ok(M, N, K)) return 0;
+  size_t need = sizeof(WqWorkspace);
+  if (!use_gemv(M, K)) {
+    FwdWs w = fwd_ws_layout(nullptr, M, K);
+    need = std::max(need, w.bytes);
+  }
+  return align_up(need, 256);
+}
+
+bl_status bitlinear_quantize_weights(const void* W, int w_dtype, int N, int K, float eps,
+                                     uint8_t* packed, float* gamma, void* ws, size_t ws_bytes,
+                                     void* stream) {
+  if (!W || !packed || !gamma || !ws) return BL_ERR_INVALID_ARG;
+  if (w_dtype != BL_F32 && w_dtype != BL_BF16) return BL_ERR_INVALID_ARG;
+  if (!(eps >= 0.0f) || !std::isfinite(eps)) return BL_ERR_INVALID_ARG;
+  if (!shape_ok(1, N, K)) return BL_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(W) || !aligned16(packed) || !aligned16(gamma) || !aligned16(ws))
+    return BL_ERR_MISALIGNED;
+  if (ws_bytes < sizeof(WqWorkspace)) return BL_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  WqWorkspace* w = static_cast<WqWorkspace*>(ws);
+  if (cudaMemsetAsync(w, 0, sizeof(WqWorkspace), s) != cudaSuccess) return BL_ERR_CUDA;
+  const long long n = static_cast<long long>(N) * K;
+  const bool bf16 = (w_dtype == BL_BF16);
+  const long long nvec = n / (bf16 ? 8 : 4);
+  const long long want = (nvec + bl::kWqThreads * 4 - 1) / (bl::kWqThreads * 4);
+  const int grid1 = static_cast<int>(std::max<long long>(1, std::min<long long>(want, 4ll * num_sms())));
+  if (bf16)
+    bl::absmean_partial_kernel<true><<<grid1, bl::kWqThreads, 0, s>>>(W, n, eps, w, gamma);
+  else
+    bl::absmean_partial_kernel<false><<<grid1, bl::kWqThreads, 0, s>>>(W, n, eps, w, gamma);
+  if (launch_status() != BL_OK) return BL_ERR_CUDA;
+  const long long nwords = n / 16;
+  const int grid2 = static_cast<int>(std::max<long long>(
+      1, std::min<long long>((nwords + 255) / 256, 8ll * num_sms())));
+  if (bf16)
+    bl::ternarize_pack_kernel<true><<<grid2, 256, 0, s>>>(W, nwords, w,
+                                                          reinterpret_cast<uint32_t*>(packed));
+  else
+    bl::ternarize_pack_kernel<false><<<grid2, 256, 0, s>>>(W, nwords, w,
+                                                           reinterpret_cast<uint32_t*>(packed));
+  return launch_status();
+}
+
+bl_status bitlinear_quantize_acts(const void* x, int x_dtype, int M, int K, int8_t* xq,
+                                  float* scale, void* stream) {
+  if (!x || !xq || !scale) return BL_ERR_INVALID_ARG;
+  if (x_dtype != BL_F32 && x_dtype != BL_BF16) return BL_ERR_INVALID_ARG;
+  if (!shape_ok(M, 1, K)) return BL_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(x) || !aligned16(xq) || !aligned16(scale)) return BL_ERR_MISALIGNED;
+  return launch_act_quant(x, x_dtype, M, K, xq, scale, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+bl_status bitlinear_forward(const void* x, int x_dtype, const uint8_t* packed,
+                            const float* gamma, void* y, int y_dtype, int M, int N, int K,
+                            void* ws, size_t ws_bytes, void* stream) {
+  if (!x || !packed || !gamma || !y) return BL_ERR_INVALID_ARG;
+  if (x_dtype != BL_F32 && x_dtype != BL_BF16) return BL_ERR_INVALID_ARG;
+  if (y_dtype != BL_F32 && y_dtype != BL_BF16) return BL_ERR_INVALID_ARG;
+  if (!shape_ok(M, N, K)) return BL_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(x) || !aligned16(packed) || !aligned16(gamma) || !aligned16(y))
+    return BL_ERR_MISALIGNED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (use_gemv(M, K)) {
+    if (x_dtype == BL_BF16)
+      return launch_gemv_x<bl::kXbf16>(x, packed, gamma, y, y_dtype, M, N, K, s);
+    return launch_gemv_x<bl::kXf32>(x, packed, gamma, y, y_dtype, M, N, K, s);
+  }
+  if (!ws) return BL_ERR_WORKSPACE;
+  if (!aligned16(ws)) return BL_ERR_MISALIGNED;
+  FwdWs w = fwd_ws_layout(ws, M, K);
+  if (ws_bytes < w.bytes) return BL_ERR_WORKSPACE;
+  bl_status st = launch_act_quant(x, x_dtype, M, K, w.xq, w.scale, w.rowsum, s);
+  if (st != BL_OK) return st;
+  return launch_gemm(w.xq, packed, w.rowsum, w.scale, gamma, y, y_dtype, M, N, K, s);
+}
+
+bl_status bitlinear_contract_i32(const int8_t* xq, const uint8_t* packed, int32_t* acc, int M,
+                                 int N, int K, void* ws, size_t ws_bytes, void* stream) {
+  if (!xq || !packed || !acc) return BL_ERR_INVALID_ARG;
+  if (!shape_ok(M, N, K)) return BL_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(xq) || !aligned16(packed) || !aligned16(acc)) return BL_ERR_MISALIGNED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (use_gemv(M, K)) return launch_gemv_x<bl::kXi8>(xq, packed, nullptr, acc, BL_I32, M, N, K, s);
+  if (!ws) return BL_ERR_WORKSPACE;
+  if (!aligned16(ws)) return BL_ERR_MISALIGNED;
+  FwdWs w = fwd_ws_layout(ws, M, K);
+  if (ws_bytes < w.bytes) return BL_ERR_WORKSPACE;
+  bl::rowsum_i8_kernel<<<M, bl::kAqThreads, 0, s>>>(xq, K, w.rowsum);
+  if (launch_status() != BL_OK) return BL_ERR_CUDA;
+  return launch_gemm(xq, packed, w.rowsum, nullptr, nullptr, acc, BL_I32, M, N, K, s);
+}
+
+bl_status bitlinear_get_device_status(void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return BL_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, bl::g_status, sizeof v) != cudaSuccess) return BL_ERR_CUDA;
+  const unsigned int zero = 0;
+  if (cudaMemcpyToSymbol(bl::g_status, &zero, sizeof zero) != cudaSuccess) return BL_ERR_CUDA;
+  if (v & bl::kStatusTimeout) return BL_ERR_TIMEOUT;
+  if (v & bl::kStatusNonfinite) return BL_ERR_NONFINITE;
+  return BL_OK;
+}
+
+bl_status bitlinear_debug_timeout_probe(uint64_t timeout_ns, void* stream) {
+  if (timeout_ns < 1000ull || timeout_ns > 5000000000ull) return BL_ERR_INVALID_ARG;
+  timeout_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(timeout_ns);
+  return launch_status();
+}
+
+const char* bitlinear_status_string(bl_status status) {
+  switch (status) {
+    case BL_OK: return "BL_OK";
+    case BL_ERR_INVALID_ARG: return "BL_ERR_INVALID_ARG";
+    case BL_ERR_UNSUPPORTED_SHAPE: return "BL_ERR_UNSUPPORTED_SHAPE";
+    case BL_ERR_MISALIGNED: return "BL_ERR_MISALIGNED";
+    case BL_ERR_CUDA: return "BL_ERR_CUDA";
+    case BL_ERR_TIMEOUT: return "BL_ERR_TIMEOUT";
+    case BL_ERR_NONFINITE: return "BL_ERR_NONFINITE";
+    case BL_ERR_WORKSPACE: return "BL_ERR_WORKSPACE";
+  }
+  return "BL_ERR_UNKNOWN";
+}
+
+}  // extern "C"

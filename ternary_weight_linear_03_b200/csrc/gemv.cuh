@@ -1,0 +1,246 @@
+// Decode BitLinear (small M): one CUDA-core kernel that quantizes the M tokens in its
+// prologue and then streams the packed ternary weights once from HBM.
+//
+// The contraction is the "integer addition" of BitNet b1.58 (dmarx anthology record
+// LIT-380, Key takeaways bullet 4). Weights are stored as u = c + 1 in {0, 1, 2}, so
+//   acc[t,n] = sum_k c[n,k] q[t,k] = sum_k u[n,k] q[t,k] - rowsum_t,
+// and one packed 32-bit word (16 trits) unpacks to four int8x4 registers with one shift
+// and one mask each (the packed layout puts trits 16g+4j .. 16g+4j+3 in bits 2j of the
+// four bytes). The byte products run on dp4a; rowsum_t = sum_k q[t,k] comes from the
+// prologue.
+//
+// Layout. Each lane owns 16-byte chunks (64 trits) of a weight row; LPR lanes share a row
+// and reduce with warp shuffles. The quantized activations live in shared memory with
+// chunk-major order inside each 16-trit group (unit g * CPR + c holds k = 64c + 16g ..
+// 64c + 16g + 15), so the lanes of a row read consecutive 16-byte units (no bank
+// conflicts) and lanes of different rows read the same unit (broadcast).
+#pragma once
+
+#include "act_quant.cuh"
+#include "common.cuh"
+
+namespace bl {
+
+constexpr int kGemvThreads = 512;
+constexpr int kGemvWarps = kGemvThreads / 32;
+constexpr int kGemvUnroll = 4;
+
+enum XMode { kXf32 = 0, kXbf16 = 1, kXi8 = 2 };
+enum OMode { kOf32 = 0, kObf16 = 1, kOi32 = 2 };
+
+template <int MT>
+struct GemvShared {
+  float red_f[MT][32];
+  int red_i[MT][32];
+  float f[MT];      // s_t * gamma
+  int rowsum[MT];
+};
+
+// Loads 16 consecutive x values of row t starting at element k (k % 16 == 0).
+template <int XM>
+__device__ __forceinline__ void load16(const void* x, long long off, float (&v)[16]) {
+  if (XM == kXbf16) {
+    const uint4* p = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(x) + off);
+    const uint4 a = p[0], b = p[1];
+    const uint32_t h[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      v[2 * q] = __uint_as_float(h[q] << 16);
+      v[2 * q + 1] = __uint_as_float(h[q] & 0xffff0000u);
+    }
+  } else {
+    const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(x) + off);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 a = p[q];
+      v[4 * q] = a.x; v[4 * q + 1] = a.y; v[4 * q + 2] = a.z; v[4 * q + 3] = a.w;
+    }
+  }
+}
+
+template <int MT, int XM, int OM>
+__global__ void __launch_bounds__(kGemvThreads) gemv_kernel(
+    const void* __restrict__ x, const uint8_t* __restrict__ packed,
+    const float* __restrict__ gamma_ptr, void* __restrict__ y, int N, int K, int lpr_log2) {
+  extern __shared__ __align__(16) unsigned char xs_raw[];  // [MT][K] int8, permuted
+  __shared__ GemvShared<MT> sh;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int CPR = K >> 6;   // 16-byte packed chunks per weight row
+  const int KB = K >> 4;    // 16-element groups per token row
+
+  // ---------------------------------------------------------------- prologue: x -> int8
+  if (XM == kXi8) {
+    int sum[MT];
+#pragma unroll
+    for (int t = 0; t < MT; ++t) sum[t] = 0;
+    for (int kb = tid; kb < KB; kb += kGemvThreads) {
+      const int unit = (kb & 3) * CPR + (kb >> 2);
+#pragma unroll
+      for (int t = 0; t < MT; ++t) {
+        const int4 q = reinterpret_cast<const int4*>(
+            static_cast<const int8_t*>(x) + static_cast<long long>(t) * K)[kb];
+        reinterpret_cast<int4*>(xs_raw + t * K)[unit] = q;
+        sum[t] = __dp4a(q.x, 0x01010101, sum[t]);
+        sum[t] = __dp4a(q.y, 0x01010101, sum[t]);
+        sum[t] = __dp4a(q.z, 0x01010101, sum[t]);
+        sum[t] = __dp4a(q.w, 0x01010101, sum[t]);
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < MT; ++t) {
+      int v = sum[t];
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+      if (lane == 0) sh.red_i[t][warp] = v;
+    }
+    __syncthreads();
+    if (tid < MT) {
+      int v = 0;
+      for (int w = 0; w < kGemvWarps; ++w) v += sh.red_i[tid][w];
+      sh.rowsum[tid] = v;
+      sh.f[tid] = 0.0f;
+    }
+  } else {
+    float amax[MT];
+    bool bad = false;
+#pragma unroll
+    for (int t = 0; t < MT; ++t) amax[t] = 0.0f;
+    for (int kb = tid; kb < KB; kb += kGemvThreads) {
+#pragma unroll
+      for (int t = 0; t < MT; ++t) {
+        float v[16];
+        load16<XM>(x, static_cast<long long>(t) * K + 16 * kb, v);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float m = abs_bits(v[i]);
+          bad |= !(m <= 3.4028234663852886e38f);
+          amax[t] = fmaxf(amax[t], m);
+        }
+      }
+    }
+    if (bad) record_status(kStatusNonfinite);
+#pragma unroll
+    for (int t = 0; t < MT; ++t) {
+      float v = amax[t];
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+      if (lane == 0) sh.red_f[t][warp] = v;
+    }
+    __syncthreads();
+    float r[MT];
+#pragma unroll
+    for (int t = 0; t < MT; ++t) {
+      float a = 0.0f;
+      for (int w = 0; w < kGemvWarps; ++w) a = fmaxf(a, sh.red_f[t][w]);
+      amax[t] = a;
+      r[t] = (a > 0.0f) ? __fdiv_rn(127.0f, a) : 0.0f;
+    }
+    int sum[MT];
+#pragma unroll
+    for (int t = 0; t < MT; ++t) sum[t] = 0;
+    for (int kb = tid; kb < KB; kb += kGemvThreads) {
+      const int unit = (kb & 3) * CPR + (kb >> 2);
+#pragma unroll
+      for (int t = 0; t < MT; ++t) {
+        float v[16];
+        load16<XM>(x, static_cast<long long>(t) * K + 16 * kb, v);
+        uint32_t w4[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int q = (amax[t] > 0.0f) ? quant_i8(v[i], r[t]) : 0;
+          sum[t] += q;
+          w4[i >> 2] |= (static_cast<uint32_t>(q) & 0xffu) << (8 * (i & 3));
+        }
+        reinterpret_cast<uint4*>(xs_raw + t * K)[unit] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < MT; ++t) {
+      int v = sum[t];
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+      if (lane == 0) sh.red_i[t][warp] = v;
+    }
+    __syncthreads();
+    if (tid < MT) {
+      int v = 0;
+      for (int w = 0; w < kGemvWarps; ++w) v += sh.red_i[tid][w];
+      sh.rowsum[tid] = v;
+      const float s = (amax[tid] > 0.0f) ? __fdiv_rn(amax[tid], 127.0f) : 0.0f;
+      sh.f[tid] = __fmul_rn(s, *gamma_ptr);
+    }
+  }
+  __syncthreads();
+
+  // ---------------------------------------------------------------- stream the weights
+  const int LPR = 1 << lpr_log2;
+  const int RPW = 32 >> lpr_log2;
+  const int sub = lane & (LPR - 1);
+  const int rsel = lane >> lpr_log2;
+  const long long warps_total = static_cast<long long>(gridDim.x) * kGemvWarps;
+  const uint4* xs4 = reinterpret_cast<const uint4*>(xs_raw);
+  const int xs_row_units = K >> 4;
+
+  for (long long rg = static_cast<long long>(blockIdx.x) * kGemvWarps + warp;
+       rg * RPW < N; rg += warps_total) {
+    const long long n = rg * RPW + rsel;
+    const bool valid = n < N;
+    int acc[MT];
+#pragma unroll
+    for (int t = 0; t < MT; ++t) acc[t] = 0;
+    if (valid) {
+      const uint4* prow = reinterpret_cast<const uint4*>(packed + n * (K >> 2));
+      for (int c0 = sub; c0 < CPR; c0 += LPR * kGemvUnroll) {
+        uint4 wv[kGemvUnroll];
+#pragma unroll
+        for (int u = 0; u < kGemvUnroll; ++u) {
+          const int c = c0 + u * LPR;
+          wv[u] = (c < CPR) ? ld_stream_v4(prow + c) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < kGemvUnroll; ++u) {
+          const int c = c0 + u * LPR;
+          if (c < CPR) {
+            const uint32_t words[4] = {wv[u].x, wv[u].y, wv[u].z, wv[u].w};
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              const uint32_t wd = words[g];
+              const int r0 = static_cast<int>(wd & 0x03030303u);
+              const int r1 = static_cast<int>((wd >> 2) & 0x03030303u);
+              const int r2 = static_cast<int>((wd >> 4) & 0x03030303u);
+              const int r3 = static_cast<int>((wd >> 6) & 0x03030303u);
+#pragma unroll
+              for (int t = 0; t < MT; ++t) {
+                const uint4 xv = xs4[t * xs_row_units + g * CPR + c];
+                acc[t] = __dp4a(r0, static_cast<int>(xv.x), acc[t]);
+                acc[t] = __dp4a(r1, static_cast<int>(xv.y), acc[t]);
+                acc[t] = __dp4a(r2, static_cast<int>(xv.z), acc[t]);
+                acc[t] = __dp4a(r3, static_cast<int>(xv.w), acc[t]);
+              }
+            }
+          }
+        }
+      }
+    }
+    for (int off = LPR >> 1; off > 0; off >>= 1) {
+#pragma unroll
+      for (int t = 0; t < MT; ++t) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], off);
+    }
+    if (valid && sub == 0) {
+#pragma unroll
+      for (int t = 0; t < MT; ++t) {
+        const int a = acc[t] - sh.rowsum[t];
+        const long long o = static_cast<long long>(t) * N + n;
+        if (OM == kOi32) {
+          static_cast<int*>(y)[o] = a;
+        } else {
+          const float v = __fmul_rn(__int2float_rn(a), sh.f[t]);
+          if (OM == kOf32) static_cast<float*>(y)[o] = v;
+          else static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(v);
+        }
+      }
+    }
+  }
+}
+
+}  // namespace bl

@@ -1,0 +1,284 @@
+"""CUDA path vs the oracle, element by element, through the C ABI (gpu marker).
+
+Bars: ternary codes, packed bytes, int8 codes, scales and int32 accumulators are compared
+bit-exactly; fp32 outputs within 1e-6 relative error and bf16 outputs within 1 ulp (in
+practice both are bit-identical, because both sides fix the same fp32 operation order).
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import ternary_weight_linear_03_b200 as bl
+from oracle import oracle as orc
+from ternary_weight_linear_03_b200 import synthetic as syn
+
+pytestmark = pytest.mark.gpu
+
+FP32_RTOL = 1e-6
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _device():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    bl.load_library()
+    assert bl.get_device_status() == 0
+    yield
+    assert bl.get_device_status() == 0
+
+
+def _np_in(t: torch.Tensor):
+    return syn.bf16_bits(t) if t.dtype == torch.bfloat16 else t.numpy()
+
+
+def _bf16_to_f32(bits: np.ndarray) -> np.ndarray:
+    return (bits.astype(np.uint32) << 16).view(np.float32)
+
+
+def assert_f32_close(got: np.ndarray, ref: np.ndarray):
+    err = np.abs(got.astype(np.float64) - ref.astype(np.float64))
+    assert np.all(err <= FP32_RTOL * np.abs(ref.astype(np.float64))), float(err.max())
+
+
+def assert_bf16_within_1ulp(got_bits: np.ndarray, ref_bits: np.ndarray):
+    g = got_bits.astype(np.int32)
+    r = ref_bits.astype(np.int32)
+    # same sign and adjacent bit patterns (bf16 ordering is monotone within a sign)
+    same_sign = (g >> 15) == (r >> 15)
+    close = np.abs(g - r) <= 1
+    zeros = ((g & 0x7FFF) == 0) & ((r & 0x7FFF) == 0)
+    assert np.all((same_sign & close) | zeros)
+
+
+# ----------------------------------------------------------------------------- weights
+
+
+@pytest.mark.parametrize("N,K,dtype", [
+    (256, 256, torch.float32), (293, 192, torch.float32), (4096, 1536, torch.float32),
+    (300, 8640, torch.bfloat16), (8, 64, torch.bfloat16), (1, 64, torch.float32),
+])
+def test_quantize_weights_bit_exact(N, K, dtype):
+    W = syn.weights(N, K, 0.02, seed=N * 7 + K, dtype=dtype)
+    packed, gamma = bl.quantize_weights(W.cuda(), eps=1e-5)
+    ref_packed, ref_gamma = orc.quantize_weights(_np_in(W), 1e-5)
+    assert gamma.item() == float(ref_gamma)
+    np.testing.assert_array_equal(packed.cpu().numpy(), ref_packed)
+
+
+@pytest.mark.parametrize("kind", ["wide", "subnormal", "zeros", "constant", "sparse"])
+def test_quantize_weights_exact_sum_edge_cases(kind):
+    rng = np.random.default_rng(17)
+    N, K = 96, 640
+    if kind == "wide":
+        w = rng.choice([-1, 1], N * K) * 10.0 ** rng.uniform(-30, 30, N * K)
+    elif kind == "subnormal":
+        w = rng.standard_normal(N * K) * 1e-40
+        w[::5] = rng.standard_normal(len(w[::5])) * 0.02
+    elif kind == "zeros":
+        w = np.zeros(N * K)
+    elif kind == "constant":
+        w = np.full(N * K, -0.013)
+    else:
+        w = rng.standard_normal(N * K) * 0.02
+        w[rng.random(N * K) < 0.9] = 0.0
+    W = np.ascontiguousarray(w.astype(np.float32).reshape(N, K))
+    for eps in (1e-5, 0.0):
+        packed, gamma = bl.quantize_weights(torch.from_numpy(W).cuda(), eps=eps)
+        ref_packed, ref_gamma = orc.quantize_weights(W, eps)
+        assert gamma.item() == float(ref_gamma), (kind, eps)
+        np.testing.assert_array_equal(packed.cpu().numpy(), ref_packed)
+
+
+def test_ternarize_ties_on_device():
+    """Weights exactly at 0.5 (gamma + eps) and one ulp either side."""
+    d = np.float32(0.71875)
+    half = np.float32(0.5) * d  # exact
+    up = np.nextafter(half, np.float32(1))
+    dn = np.nextafter(half, np.float32(0))
+    row = [half, -half, up, -up, dn, -dn, np.float32(1.5) * d, -np.float32(1.5) * d]
+    W = np.array(row * 8, np.float32)  # 64 values
+    # pad a second row so that mean|W| is exactly d: need sum|W| = 128 d
+    s = float(np.abs(W).astype(np.float64).sum())
+    rest = np.full(64, np.float32((128 * float(d) - s) / 64), np.float32)
+    W = np.stack([W, rest])
+    ref_gamma = orc.absmean(W)
+    packed, gamma = bl.quantize_weights(torch.from_numpy(W).cuda(), eps=0.0)
+    assert gamma.item() == float(ref_gamma)
+    ref_packed, _ = orc.quantize_weights(W, 0.0)
+    np.testing.assert_array_equal(packed.cpu().numpy(), ref_packed)
+    if ref_gamma == d:
+        codes = orc.unpack(ref_packed, 64)[0, :8]
+        np.testing.assert_array_equal(codes, [0, 0, 1, -1, 0, 0, 1, -1])
+
+
+# ----------------------------------------------------------------------------- activations
+
+
+@pytest.mark.parametrize("M,K,dtype,outliers", [
+    (8, 256, torch.float32, 0.0), (16, 1536, torch.bfloat16, 0.01),
+    (5, 8640, torch.bfloat16, 0.0), (64, 3200, torch.float32, 0.01),
+])
+def test_quantize_acts_bit_exact(M, K, dtype, outliers):
+    x = syn.activations(M, K, seed=M + K, dtype=dtype, outlier_frac=outliers)
+    x[0].zero_()                       # all-zero row
+    if M > 2:
+        x[1].zero_()
+        x[1, 7] = -3.25                # one-hot row
+    xq, scale = bl.quantize_acts(x.cuda())
+    ref_q, ref_s = orc.quantize_acts(_np_in(x))
+    np.testing.assert_array_equal(xq.cpu().numpy(), ref_q)
+    np.testing.assert_array_equal(scale.cpu().numpy(), ref_s)
+
+
+# ----------------------------------------------------------------------------- contraction
+
+
+CONTRACT_SHAPES = [
+    (1, 256, 256), (2, 293, 192), (3, 1000, 1536), (4, 777, 64),       # CUDA-core path
+    (5, 300, 640), (16, 4096, 1536), (130, 293, 8640), (300, 520, 1536),  # tensor-core path
+    (129, 257, 128), (64, 64, 64),
+]
+
+
+@pytest.mark.parametrize("M,N,K", CONTRACT_SHAPES)
+def test_contract_i32_bit_exact(M, N, K):
+    rng = np.random.default_rng(M * 1000 + N + K)
+    q = rng.integers(-127, 128, size=(M, K)).astype(np.int8)
+    q[0, :] = 127  # extreme row
+    codes = rng.integers(-1, 2, size=(N, K)).astype(np.int8)
+    codes[0, :] = 1
+    packed = orc.pack(codes)
+    acc = bl.contract_i32(torch.from_numpy(q).cuda(), torch.from_numpy(packed).cuda())
+    np.testing.assert_array_equal(acc.cpu().numpy(), orc.contract_i32(q, codes))
+
+
+# ----------------------------------------------------------------------------- forward
+
+
+@pytest.mark.parametrize("M,N,K,x_dtype", [
+    (8, 256, 256, torch.float32),          # tiny config
+    (1, 4096, 1536, torch.bfloat16), (4, 4096, 1536, torch.bfloat16),
+    (16, 4096, 1536, torch.bfloat16),
+    (3, 1000, 3200, torch.float32), (200, 600, 8640, torch.bfloat16),
+])
+@pytest.mark.parametrize("out", ["f32", "bf16"])
+def test_forward_matches_oracle(M, N, K, x_dtype, out):
+    W = syn.weights(N, K, 0.02, seed=1000 + N)
+    x = syn.activations(M, K, seed=2000 + M, dtype=x_dtype, outlier_frac=0.01)
+    packed, gamma = bl.quantize_weights(W.cuda())
+    y = bl.forward(x.cuda(), packed, gamma,
+                   out_dtype=torch.float32 if out == "f32" else torch.bfloat16)
+    ref = orc.forward(_np_in(x), packed.cpu().numpy(), gamma.item(), out=out)
+    if out == "f32":
+        assert_f32_close(y.cpu().numpy(), ref)
+        np.testing.assert_array_equal(y.cpu().numpy(), ref)  # same op order: identical
+    else:
+        got = y.cpu().view(torch.int16).numpy().view(np.uint16)
+        assert_bf16_within_1ulp(got, ref)
+        np.testing.assert_array_equal(got, ref)
+
+
+def test_forward_tiny_config_end_to_end():
+    """Tiny config: W 256x256 ~N(0,0.02), x 8x256 ~N(0,1) fp32, seed 0, fp32 out."""
+    W = syn.weights(256, 256, 0.02, seed=0)
+    x = syn.activations(8, 256, seed=0, dtype=torch.float32)
+    packed, gamma = bl.quantize_weights(W.cuda())
+    y = bl.forward(x.cuda(), packed, gamma, out_dtype=torch.float32)
+    ref_packed, ref_gamma = orc.quantize_weights(W.numpy(), 1e-5)
+    ref = orc.forward(x.numpy(), ref_packed, ref_gamma)
+    np.testing.assert_array_equal(y.cpu().numpy(), ref)
+
+
+def test_forward_paths_agree_at_the_switch():
+    """M = 4 runs the CUDA-core kernel, M = 5 the tensor-core GEMM: rows must agree."""
+    W = syn.weights(1000, 1536, 0.02, seed=5)
+    x = syn.activations(5, 1536, seed=6)
+    packed, gamma = bl.quantize_weights(W.cuda())
+    y5 = bl.forward(x.cuda(), packed, gamma, out_dtype=torch.float32)
+    y4 = bl.forward(x[:4].contiguous().cuda(), packed, gamma, out_dtype=torch.float32)
+    torch.testing.assert_close(y5[:4], y4, rtol=0, atol=0)
+
+
+# ----------------------------------------------------------------------------- full sizes
+
+
+FULL = [
+    ("700m_up_1536x4096", 16), ("3b_gate_up_3200x8640", 64), ("3b_down_8640x3200", 1),
+    ("70b_up_8192x28672", 176), ("70b_down_28672x8192", 16),
+]
+
+
+@pytest.mark.parametrize("name,M", FULL)
+def test_full_size_sampled_rows(name, M):
+    """Full-size matrices: gamma and every packed byte exactly, outputs on sampled rows."""
+    wl = syn.WORKLOADS[name]
+    N, K = wl["N"], wl["K"]
+    W = syn.weights(N, K, wl["sigma"], seed=syn.w_seed(name))
+    x = syn.activations(M, K, seed=syn.x_seed(name, M), dtype=wl["x_dtype"],
+                        outlier_frac=wl["outlier_frac"])
+    packed, gamma = bl.quantize_weights(W.cuda())
+    assert gamma.item() == float(orc.absmean(W.numpy()))
+    rows = np.random.default_rng(0).choice(N, size=min(N, 96), replace=False)
+    rows.sort()
+    ref_packed_rows, _ = None, None
+    codes = orc.ternarize(np.ascontiguousarray(W.numpy()[rows]), gamma.item(), 1e-5)
+    np.testing.assert_array_equal(packed.cpu().numpy()[rows], orc.pack(codes))
+    y = bl.forward(x.cuda(), packed, gamma, out_dtype=torch.bfloat16)
+    ref = orc.forward(_np_in(x), orc.pack(codes), gamma.item(), out="bf16")
+    got = y.cpu().view(torch.int16).numpy().view(np.uint16)[:, rows]
+    np.testing.assert_array_equal(got, ref)
+
+
+def test_prefill_shape_sampled_rows():
+    """M = 4096, K = 8192, N = 28672 through the tensor-core path, sampled outputs."""
+    name = "70b_prefill_4096x8192x28672"
+    wl = syn.WORKLOADS[name]
+    N, K, M = wl["N"], wl["K"], 4096
+    W = syn.weights(N, K, wl["sigma"], seed=syn.w_seed(name))
+    x = syn.activations(M, K, seed=syn.x_seed(name, M), dtype=torch.bfloat16)
+    packed, gamma = bl.quantize_weights(W.cuda())
+    y = bl.forward(x.cuda(), packed, gamma, out_dtype=torch.bfloat16)
+    rng = np.random.default_rng(1)
+    rows = np.sort(rng.choice(N, 64, replace=False))
+    toks = np.sort(rng.choice(M, 48, replace=False))
+    codes = orc.ternarize(np.ascontiguousarray(W.numpy()[rows]), gamma.item(), 1e-5)
+    xs = x[torch.from_numpy(toks)].contiguous()
+    ref = orc.forward(syn.bf16_bits(xs), orc.pack(codes), gamma.item(), out="bf16")
+    got = y.cpu()[torch.from_numpy(toks)][:, torch.from_numpy(rows)]
+    np.testing.assert_array_equal(got.contiguous().view(torch.int16).numpy().view(np.uint16), ref)
+
+
+# ----------------------------------------------------------------------------- status word
+
+
+def test_nonfinite_inputs_set_status():
+    W = torch.randn(64, 64, device="cuda")
+    W[3, 5] = float("nan")
+    bl.quantize_weights(W)
+    assert bl.get_device_status() == 6
+    x = torch.randn(2, 64, device="cuda")
+    x[1, 1] = float("inf")
+    bl.quantize_acts(x)
+    assert bl.get_device_status() == 6
+    assert bl.get_device_status() == 0  # read clears
+
+
+def test_timeout_probe_reports_and_context_survives():
+    bl.debug_timeout_probe(2_000_000)  # 2 ms wait on a barrier nobody arrives on
+    assert bl.get_device_status() == 5
+    W = syn.weights(256, 256, 0.02, seed=0)
+    packed, gamma = bl.quantize_weights(W.cuda())
+    assert gamma.item() == float(orc.absmean(W.numpy()))
+    assert bl.get_device_status() == 0
+
+
+def test_repeatable():
+    W = syn.weights(2048, 1536, 0.02, seed=3).cuda()
+    x = syn.activations(64, 1536, seed=4).cuda()
+    p1, g1 = bl.quantize_weights(W)
+    p2, g2 = bl.quantize_weights(W)
+    assert torch.equal(p1, p2) and torch.equal(g1, g2)
+    assert torch.equal(bl.forward(x, p1, g1), bl.forward(x, p2, g2))
