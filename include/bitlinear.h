@@ -117,6 +117,24 @@ bl_status bitlinear_contract_i32(const int8_t* xq, const uint8_t* packed, int32_
                                  int M, int N, int K, void* ws, size_t ws_bytes,
                                  void* stream);
 
+/* bitlinear_forward without a workspace argument. The paper has no counterpart: this
+ * entry point exists for callers that cannot allocate device memory at the point of
+ * call, e.g. code running inside another runtime whose memory planner owns the whole
+ * device and forbids further cudaMalloc, or latency-critical paths that avoid cudaMalloc
+ * and cudaFree because those calls can synchronize the device.
+ *   Same arguments, results and errors as bitlinear_forward, minus ws / ws_bytes.
+ *   Scratch: a 16 MiB array compiled into the library (held on every GPU that loads it
+ *   until the process exits). Small M needs none; otherwise M*K + 8*M bytes (each part
+ *   rounded up to 256) must fit in 16 MiB, else BL_ERR_WORKSPACE is returned before
+ *   anything is queued.
+ *   The first call on a device looks up the array's device address (cudaGetSymbolAddress)
+ *   and caches it; make that first call before any stream capture.
+ *   Every call on a device shares the one array: calls whose work overlaps on the GPU
+ *   race and give undefined results. The library allocates and frees nothing here. */
+bl_status bitlinear_forward_noalloc(const void* x, int x_dtype, const uint8_t* packed,
+                                    const float* gamma, void* y, int y_dtype, int M, int N,
+                                    int K, void* stream);
+
 /* Waits for `stream`, then reads and clears the current device's status word:
  * BL_OK, BL_ERR_NONFINITE or BL_ERR_TIMEOUT (the first recorded wins in that order of
  * severity: TIMEOUT over NONFINITE). BL_ERR_CUDA if the wait or the read fails. */

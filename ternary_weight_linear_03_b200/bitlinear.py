@@ -24,7 +24,8 @@ STATUS = {
 # Every symbol declared in include/bitlinear.h.
 EXPORTS = (
     "bitlinear_workspace_size", "bitlinear_quantize_weights", "bitlinear_quantize_acts",
-    "bitlinear_forward", "bitlinear_contract_i32", "bitlinear_get_device_status",
+    "bitlinear_forward", "bitlinear_forward_noalloc", "bitlinear_contract_i32",
+    "bitlinear_get_device_status",
     "bitlinear_debug_timeout_probe", "bitlinear_status_string",
 )
 
@@ -57,6 +58,8 @@ def load_library() -> ctypes.CDLL:
     lib.bitlinear_quantize_acts.restype = i
     lib.bitlinear_forward.argtypes = [p, i, p, p, p, i, i, i, i, p, sz, p]
     lib.bitlinear_forward.restype = i
+    lib.bitlinear_forward_noalloc.argtypes = [p, i, p, p, p, i, i, i, i, p]
+    lib.bitlinear_forward_noalloc.restype = i
     lib.bitlinear_contract_i32.argtypes = [p, p, p, i, i, i, p, sz, p]
     lib.bitlinear_contract_i32.restype = i
     lib.bitlinear_get_device_status.argtypes = [p]
@@ -155,6 +158,25 @@ def forward(x: torch.Tensor, packed: torch.Tensor, gamma: torch.Tensor,
         _dev(x, "x"), _dtype_code(x), _dev(packed, "packed"), _dev(gamma, "gamma"), _dev(y, "y"),
         _dtype_code(y), M, N, K, _dev(ws, "ws"), ws.numel(), _stream(stream)),
         "bitlinear_forward")
+    return y
+
+
+def forward_noalloc(x: torch.Tensor, packed: torch.Tensor, gamma: torch.Tensor,
+                    out_dtype: torch.dtype = torch.bfloat16, y: torch.Tensor | None = None,
+                    stream=None) -> torch.Tensor:
+    """bitlinear_forward without a workspace: the library's built-in 16 MiB device scratch
+    serves the tensor-core path (for callers that cannot allocate; calls must not overlap
+    on the GPU)."""
+    lib = load_library()
+    M, K = x.shape
+    N = packed.shape[0]
+    if packed.shape[1] * 4 != K:
+        raise ValueError("packed must be [N][K/4]")
+    if y is None:
+        y = torch.empty((M, N), dtype=out_dtype, device=x.device)
+    _check(lib.bitlinear_forward_noalloc(
+        _dev(x, "x"), _dtype_code(x), _dev(packed, "packed"), _dev(gamma, "gamma"), _dev(y, "y"),
+        _dtype_code(y), M, N, K, _stream(stream)), "bitlinear_forward_noalloc")
     return y
 
 

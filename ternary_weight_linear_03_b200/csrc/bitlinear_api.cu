@@ -225,6 +225,40 @@ __global__ void timeout_probe_kernel(unsigned long long limit_ns) {
 
 }  // namespace
 
+// ------------------------------------------------------------------ no-allocation forward
+// Scratch for bitlinear_forward_noalloc: the int8 activations, per-token scales and
+// row sums that the tensor-core path stages between its two kernels. It is a file-scope
+// device array, so every GPU that loads this library holds these 16 MiB until the
+// process exits, and every call of bitlinear_forward_noalloc on a device shares it.
+static constexpr size_t kNoAllocScratchBytes = static_cast<size_t>(16) << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device. In host code the array's
+// name is only a host-side stand-in, so the address is looked up once per device with
+// cudaGetSymbolAddress (with that device current) and cached.
+bl_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BL_ERR_CUDA;
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return BL_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return BL_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return BL_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 size_t bitlinear_workspace_size(int M, int N, int K) {
@@ -331,6 +365,37 @@ bl_status bitlinear_get_device_status(void* stream) {
   if (v & bl::kStatusTimeout) return BL_ERR_TIMEOUT;
   if (v & bl::kStatusNonfinite) return BL_ERR_NONFINITE;
   return BL_OK;
+}
+
+// Same computation as bitlinear_forward, for callers that cannot allocate device memory:
+// the staging buffers of the tensor-core path live in g_noalloc_scratch instead of a
+// caller-supplied workspace. Nothing in the scratch has to start at zero (each call
+// writes every byte it later reads). No cudaMalloc, cudaFree or allocating library call
+// is made. Calls that overlap on the GPU (other streams, other host threads) race on the
+// shared scratch; callers serialize them.
+bl_status bitlinear_forward_noalloc(const void* x, int x_dtype, const uint8_t* packed,
+                                    const float* gamma, void* y, int y_dtype, int M, int N,
+                                    int K, void* stream) {
+  if (!x || !packed || !gamma || !y) return BL_ERR_INVALID_ARG;
+  if (x_dtype != BL_F32 && x_dtype != BL_BF16) return BL_ERR_INVALID_ARG;
+  if (y_dtype != BL_F32 && y_dtype != BL_BF16) return BL_ERR_INVALID_ARG;
+  if (!shape_ok(M, N, K)) return BL_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(x) || !aligned16(packed) || !aligned16(gamma) || !aligned16(y))
+    return BL_ERR_MISALIGNED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (use_gemv(M, K)) {
+    if (x_dtype == BL_BF16)
+      return launch_gemv_x<bl::kXbf16>(x, packed, gamma, y, y_dtype, M, N, K, s);
+    return launch_gemv_x<bl::kXf32>(x, packed, gamma, y, y_dtype, M, N, K, s);
+  }
+  if (fwd_ws_layout(nullptr, M, K).bytes > kNoAllocScratchBytes) return BL_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  bl_status st = noalloc_scratch(&scratch);
+  if (st != BL_OK) return st;
+  FwdWs w = fwd_ws_layout(scratch, M, K);
+  st = launch_act_quant(x, x_dtype, M, K, w.xq, w.scale, w.rowsum, s);
+  if (st != BL_OK) return st;
+  return launch_gemm(w.xq, packed, w.rowsum, w.scale, gamma, y, y_dtype, M, N, K, s);
 }
 
 bl_status bitlinear_debug_timeout_probe(uint64_t timeout_ns, void* stream) {
