@@ -5,6 +5,10 @@ A step is one pass of the whole BitLinear hot path over one batch: absmean terna
 quantization of the fp32 weight matrix (gamma, codes, 2-bit packing), per-token int8
 quantization of the activations, the int32 contraction and the rescale to bf16.
 
+The timed loop replays one CUDA graph per step (captured from the same library calls), so
+host launch overhead is not part of the number; `e2e` times the plain library calls with
+host buffers instead.
+
 Default workload: the 700M-class FFN up-projection (K=1536, N=4096, W ~ N(0, 0.02) fp32,
 bf16 activations ~ N(0, 1) with 1% outlier channels x20), M = 16 tokens. Inputs larger
 than L2: the step cycles through enough weight copies (8 x 25 MB) that every step reads
@@ -28,6 +32,7 @@ import sys
 import threading
 import time
 
+import numpy as np
 import torch
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -163,12 +168,15 @@ def run_reference(args):
     x = syn.activations(M, K, seed=syn.x_seed(name, M), dtype=wl["x_dtype"],
                         outlier_frac=wl["outlier_frac"])
     xin = syn.bf16_bits(x) if x.dtype == torch.bfloat16 else x.numpy()
-    # a bounded sample per step: every weight is quantized, outputs for a row subset
-    rows = N if N * K * M <= 16 * 4096 * 1536 else max(64, (16 * 4096 * 1536) // (K * M))
+    # A bounded sample per step: the first R weight rows go through the whole path
+    # (absmean over those rows, ternarize, pack, forward for all M tokens). Every part of
+    # the work is linear in the number of rows, so tokens/s = M * R / (N * step time).
+    R = min(N, 512)
+    Wr = np.ascontiguousarray(W[:R])
 
     def step():
-        packed, gamma = orc.quantize_weights(W, 1e-5)
-        orc.forward(xin, packed[:rows], gamma, out="bf16")
+        packed, gamma = orc.quantize_weights(Wr, 1e-5)
+        orc.forward(xin, packed, gamma, out="bf16")
 
     for _ in range(args.warmup):
         step()
@@ -176,10 +184,9 @@ def run_reference(args):
     for _ in range(args.steps):
         step()
     el = time.perf_counter() - t0
-    frac = rows / N
-    value = M * args.steps / el * frac  # tokens/s scaled from the sampled rows
-    sample = (f"each step: absmean+ternarize+pack of all {N}x{K} weights, forward of M={M} "
-              f"for {rows}/{N} output rows; tokens/s scaled by that row fraction")
+    value = M * args.steps * R / (N * el)
+    sample = (f"each step: rows 0..{R - 1} of the {N}x{K} weights through absmean, ternarize, "
+              f"pack and the forward of M={M} tokens; scaled by {R}/{N} (work is linear in rows)")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -229,20 +236,34 @@ def main():
 
     def step(i, ev=None):
         if ev is not None:
-            ev[0].record(stream)
+            ev[0].record()
         bl.quantize_weights(Ws[i % copies], 1e-5, packed=packed, gamma=gamma, ws=ws)
         if ev is not None:
-            ev[1].record(stream)
+            ev[1].record()
         bl.forward(xs[i % copies], packed, gamma, y=y, ws=ws)
         if ev is not None:
-            ev[2].record(stream)
+            ev[2].record()
 
-    for i in range(args.warmup):
+    for i in range(max(args.warmup, copies)):  # eager warm-up also configures every kernel
         step(i)
     torch.cuda.synchronize()
     assert bl.get_device_status() == 0
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    # One CUDA graph per weight copy (the step's launches with timing-event nodes between
+    # the weight quantization and the forward); the timed loop replays them in turn.
+    graphs, evs = [], []
+    for i in range(copies):
+        ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)]
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step(i, ev)
+        graphs.append(g)
+        evs.append(ev)
+    for i in range(max(3, args.warmup)):
+        graphs[i % copies].replay()
+    torch.cuda.synchronize()
+    assert bl.get_device_status() == 0
+
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     if dist is not None:
@@ -251,7 +272,7 @@ def main():
     with ClockSampler(local) as clk:
         start.record(stream)
         for i in range(args.steps):
-            step(i, evs[i])
+            graphs[i % copies].replay()
         end.record(stream)
         torch.cuda.synchronize()
     if dist is not None:
@@ -265,6 +286,7 @@ def main():
     if status != 0:
         raise SystemExit(f"device status {bl.status_string(status)} after the timed region")
 
+    # per-launch times: the event nodes of each copy's graph as of its last replay
     wq_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     fw_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     hbm_peak, _, peak_kind = peaks()
@@ -324,6 +346,7 @@ def main():
                "h2d_bytes_per_step": W_h.numel() * 4 + x_h.numel() * x_h.element_size(),
                "d2h_bytes_per_step": y_h.numel() * 2, "steps": e2e_steps}
 
+    del graphs
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
@@ -332,7 +355,7 @@ def main():
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(name, M)
-    launches_per_step = 2 + (1 if M <= 4 else 2)
+    launches_per_step = 1 + (1 if M <= 4 else 2)  # weight quant + (GEMV | act quant + GEMM)
     out = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps,

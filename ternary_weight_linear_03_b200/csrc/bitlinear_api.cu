@@ -12,6 +12,7 @@
 #include "../../include/bitlinear.h"
 #include "act_quant.cuh"
 #include "common.cuh"
+#include "gemm_skinny.cuh"
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
 #include "weight_quant.cuh"
@@ -20,7 +21,8 @@ namespace {
 
 using bl::WqWorkspace;
 
-constexpr int kGemvMaxM = 4;            // M above this runs the tensor-core GEMM
+constexpr int kGemvMaxM = 4;            // M above this runs a tensor-core kernel
+constexpr int kSkinnyMaxM = 256;        // M above this runs the prefill GEMM
 constexpr int kGemvMaxSmem = 200 * 1024;  // xq rows held in shared memory by the GEMV
 constexpr unsigned long long kWaitLimitNs = 4000000000ull;  // 4 s per mbarrier wait
 
@@ -64,6 +66,49 @@ FwdWs fwd_ws_layout(void* base, int M, int K) {
   w.scale = reinterpret_cast<float*>(p + a);
   w.rowsum = reinterpret_cast<int*>(p + a + b);
   w.bytes = a + 2 * b;
+  return w;
+}
+
+// Split-K plan of the skinny tensor-core kernel for M tokens (4 < M <= 256).
+struct SkinnyPlan {
+  int bnt;     // token tile: M rounded up to a multiple of 16
+  int tiles;   // 128-row weight tiles
+  int splits;  // K ranges per tile
+  int kbps;    // 128-wide K blocks per split
+};
+SkinnyPlan skinny_plan(int M, int N, int K) {
+  SkinnyPlan p{};
+  p.bnt = (M + 15) / 16 * 16;
+  p.tiles = (N + bl::sk::BW - 1) / bl::sk::BW;
+  const int KB = (K + bl::sk::BK - 1) / bl::sk::BK;
+  // Split K only when the weight tiles alone leave most SMs idle, and keep at least 4
+  // K blocks per split so that each CTA streams long enough to cover its fixed costs.
+  long long splits = 1;
+  if (p.tiles < num_sms()) splits = (num_sms() + p.tiles - 1) / p.tiles;
+  splits = std::max<long long>(1, std::min<long long>(splits, std::max(1, KB / 4)));
+  p.kbps = static_cast<int>((KB + splits - 1) / splits);
+  p.kbps = (p.kbps + bl::sk::KPS - 1) / bl::sk::KPS * bl::sk::KPS;  // whole super-tiles
+  p.splits = (KB + p.kbps - 1) / p.kbps;                          // no empty split
+  return p;
+}
+
+// Workspace of the skinny path: the FwdWs part, then (only when splits > 1) the int32
+// sums [M][N] and one arrival counter per weight tile, contiguous so one memset clears
+// both.
+struct SkinnyWs {
+  int* partial;
+  unsigned int* counters;
+  size_t bytes;  // total, including the FwdWs part
+};
+SkinnyWs skinny_ws_layout(void* base, int M, int N, int K, const SkinnyPlan& p) {
+  SkinnyWs w{};
+  const size_t head = fwd_ws_layout(nullptr, M, K).bytes;
+  const size_t part = (p.splits > 1) ? align_up(static_cast<size_t>(M) * N * 4, 256) : 0;
+  const size_t cnt = align_up(static_cast<size_t>(p.tiles) * 4, 256);
+  char* c = static_cast<char*>(base);
+  w.partial = reinterpret_cast<int*>(c + head);
+  w.counters = reinterpret_cast<unsigned int*>(c + head + part);
+  w.bytes = head + part + cnt;
   return w;
 }
 
@@ -203,6 +248,57 @@ bl_status launch_gemm(const int8_t* xq, const uint8_t* packed, const int* rowsum
   }
 }
 
+template <int OM>
+bl_status launch_skinny_t(const int8_t* xq, const uint8_t* packed, const int* rowsum,
+                          const float* scale, const float* gamma, void* y, int M, int N, int K,
+                          const SkinnyPlan& p, const SkinnyWs& w, cudaStream_t s) {
+  CUtensorMap map_x, map_w;
+  if (!make_map_u8(&map_x, xq, K, M, K, bl::sk::BK, p.bnt, true)) return BL_ERR_CUDA;
+  if (!make_map_u8(&map_w, packed, K / 4, N, K / 4, bl::sk::BK * bl::sk::KPS / 4, bl::sk::BW,
+                   true))
+    return BL_ERR_CUDA;
+  auto kern = bl::gemm_skinny_kernel<OM>;
+  static bool configured = false;
+  if (!configured) {
+    int most = 0;
+    for (int b = 16; b <= bl::sk::BW * 2; b += 16) most = std::max(most, bl::sk::smem_bytes(b));
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, most) !=
+        cudaSuccess)
+      return BL_ERR_CUDA;
+    configured = true;
+  }
+  if (p.splits > 1 &&
+      cudaMemsetAsync(w.partial, 0,
+                      reinterpret_cast<char*>(w.counters + p.tiles) -
+                          reinterpret_cast<char*>(w.partial),
+                      s) != cudaSuccess)
+    return BL_ERR_CUDA;
+  kern<<<p.tiles * p.splits, bl::sk::THREADS, bl::sk::smem_bytes(p.bnt), s>>>(
+      map_x, map_w, rowsum, scale, gamma, y, w.partial, w.counters, M, N, K, p.bnt, p.splits,
+      p.kbps, kWaitLimitNs);
+  return launch_status();
+}
+
+bl_status launch_skinny(const int8_t* xq, const uint8_t* packed, const int* rowsum,
+                        const float* scale, const float* gamma, void* y, int y_dtype, int M,
+                        int N, int K, void* ws, cudaStream_t s) {
+  const SkinnyPlan p = skinny_plan(M, N, K);
+  const SkinnyWs w = skinny_ws_layout(ws, M, N, K, p);
+  switch (y_dtype) {
+    case BL_F32: return launch_skinny_t<0>(xq, packed, rowsum, scale, gamma, y, M, N, K, p, w, s);
+    case BL_BF16: return launch_skinny_t<1>(xq, packed, rowsum, scale, gamma, y, M, N, K, p, w, s);
+    case BL_I32: return launch_skinny_t<2>(xq, packed, rowsum, scale, gamma, y, M, N, K, p, w, s);
+    default: return BL_ERR_INVALID_ARG;
+  }
+}
+
+// Workspace bytes the forward / contract paths need for (M, N, K).
+size_t fwd_ws_bytes(int M, int N, int K) {
+  if (use_gemv(M, K)) return 0;
+  if (M <= kSkinnyMaxM) return skinny_ws_layout(nullptr, M, N, K, skinny_plan(M, N, K)).bytes;
+  return fwd_ws_layout(nullptr, M, K).bytes;
+}
+
 bl_status launch_act_quant(const void* x, int x_dtype, int M, int K, int8_t* xq, float* scale,
                            int* rowsum, cudaStream_t s) {
   if (x_dtype == BL_BF16)
@@ -210,6 +306,51 @@ bl_status launch_act_quant(const void* x, int x_dtype, int M, int K, int8_t* xq,
   else
     bl::act_quant_kernel<false><<<M, bl::kAqThreads, 0, s>>>(x, K, xq, scale, rowsum);
   return launch_status();
+}
+
+// ------------------------------------------------------------------ weight quantization
+// Workspace of bitlinear_quantize_weights: the WqWorkspace header, then the per-block
+// lists of ambiguous weights (8 bytes each; room for n/32 of them in total). A smaller
+// workspace only makes more blocks re-read their range; results do not change.
+size_t wq_ws_bytes(long long n) {
+  return align_up(sizeof(WqWorkspace), 256) + align_up(static_cast<size_t>(n / 32) * 8, 256);
+}
+
+template <bool kBf16>
+bl_status launch_weight_quant_t(const void* W, long long n, float eps, void* ws,
+                                size_t ws_bytes, float* gamma, uint32_t* packed,
+                                cudaStream_t s) {
+  auto kern = bl::weight_quant_kernel<kBf16>;
+  static int blocks_per_sm = 0;
+  if (blocks_per_sm == 0) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_per_sm, kern, bl::kWqThreads, 0) !=
+            cudaSuccess ||
+        blocks_per_sm < 1)
+      return BL_ERR_CUDA;
+  }
+  const long long nwords = n / 16;
+  const long long want = (nwords + bl::kWqThreads * 4 - 1) / (bl::kWqThreads * 4);
+  const int grid = static_cast<int>(
+      std::max<long long>(1, std::min<long long>(want, 1ll * blocks_per_sm * num_sms())));
+  WqWorkspace* hdr = static_cast<WqWorkspace*>(ws);
+  const size_t head = align_up(sizeof(WqWorkspace), 256);
+  unsigned long long* lists =
+      reinterpret_cast<unsigned long long*>(static_cast<char*>(ws) + head);
+  const long long room = (ws_bytes > head) ? static_cast<long long>((ws_bytes - head) / 8) : 0;
+  int cap = static_cast<int>(std::min<long long>(room / grid, 1ll << 30));
+  if (cudaMemsetAsync(hdr, 0, sizeof(WqWorkspace), s) != cudaSuccess) return BL_ERR_CUDA;
+  unsigned long long limit = kWaitLimitNs;
+  void* args[] = {const_cast<void**>(&W), &n, &eps, &hdr, &lists, &cap, &gamma, &packed, &limit};
+  if (cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kern), dim3(grid),
+                                  dim3(bl::kWqThreads), args, 0, s) != cudaSuccess)
+    return BL_ERR_CUDA;
+  return launch_status();
+}
+
+bl_status launch_weight_quant(const void* W, bool bf16, long long n, float eps, void* ws,
+                              size_t ws_bytes, float* gamma, uint32_t* packed, cudaStream_t s) {
+  return bf16 ? launch_weight_quant_t<true>(W, n, eps, ws, ws_bytes, gamma, packed, s)
+              : launch_weight_quant_t<false>(W, n, eps, ws, ws_bytes, gamma, packed, s);
 }
 
 // ------------------------------------------------------------------ debug probe
@@ -263,11 +404,7 @@ extern "C" {
 
 size_t bitlinear_workspace_size(int M, int N, int K) {
   if (!shape_ok(M, N, K)) return 0;
-  size_t need = sizeof(WqWorkspace);
-  if (!use_gemv(M, K)) {
-    FwdWs w = fwd_ws_layout(nullptr, M, K);
-    need = std::max(need, w.bytes);
-  }
+  const size_t need = std::max(wq_ws_bytes(static_cast<long long>(N) * K), fwd_ws_bytes(M, N, K));
   return align_up(need, 256);
 }
 
@@ -282,28 +419,8 @@ bl_status bitlinear_quantize_weights(const void* W, int w_dtype, int N, int K, f
     return BL_ERR_MISALIGNED;
   if (ws_bytes < sizeof(WqWorkspace)) return BL_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  WqWorkspace* w = static_cast<WqWorkspace*>(ws);
-  if (cudaMemsetAsync(w, 0, sizeof(WqWorkspace), s) != cudaSuccess) return BL_ERR_CUDA;
-  const long long n = static_cast<long long>(N) * K;
-  const bool bf16 = (w_dtype == BL_BF16);
-  const long long nvec = n / (bf16 ? 8 : 4);
-  const long long want = (nvec + bl::kWqThreads * 4 - 1) / (bl::kWqThreads * 4);
-  const int grid1 = static_cast<int>(std::max<long long>(1, std::min<long long>(want, 4ll * num_sms())));
-  if (bf16)
-    bl::absmean_partial_kernel<true><<<grid1, bl::kWqThreads, 0, s>>>(W, n, eps, w, gamma);
-  else
-    bl::absmean_partial_kernel<false><<<grid1, bl::kWqThreads, 0, s>>>(W, n, eps, w, gamma);
-  if (launch_status() != BL_OK) return BL_ERR_CUDA;
-  const long long nwords = n / 16;
-  const int grid2 = static_cast<int>(std::max<long long>(
-      1, std::min<long long>((nwords + 255) / 256, 8ll * num_sms())));
-  if (bf16)
-    bl::ternarize_pack_kernel<true><<<grid2, 256, 0, s>>>(W, nwords, w,
-                                                          reinterpret_cast<uint32_t*>(packed));
-  else
-    bl::ternarize_pack_kernel<false><<<grid2, 256, 0, s>>>(W, nwords, w,
-                                                           reinterpret_cast<uint32_t*>(packed));
-  return launch_status();
+  return launch_weight_quant(W, w_dtype == BL_BF16, static_cast<long long>(N) * K, eps, ws,
+                             ws_bytes, gamma, reinterpret_cast<uint32_t*>(packed), s);
 }
 
 bl_status bitlinear_quantize_acts(const void* x, int x_dtype, int M, int K, int8_t* xq,
@@ -332,10 +449,12 @@ bl_status bitlinear_forward(const void* x, int x_dtype, const uint8_t* packed,
   }
   if (!ws) return BL_ERR_WORKSPACE;
   if (!aligned16(ws)) return BL_ERR_MISALIGNED;
+  if (ws_bytes < fwd_ws_bytes(M, N, K)) return BL_ERR_WORKSPACE;
   FwdWs w = fwd_ws_layout(ws, M, K);
-  if (ws_bytes < w.bytes) return BL_ERR_WORKSPACE;
   bl_status st = launch_act_quant(x, x_dtype, M, K, w.xq, w.scale, w.rowsum, s);
   if (st != BL_OK) return st;
+  if (M <= kSkinnyMaxM)
+    return launch_skinny(w.xq, packed, w.rowsum, w.scale, gamma, y, y_dtype, M, N, K, ws, s);
   return launch_gemm(w.xq, packed, w.rowsum, w.scale, gamma, y, y_dtype, M, N, K, s);
 }
 
@@ -348,10 +467,12 @@ bl_status bitlinear_contract_i32(const int8_t* xq, const uint8_t* packed, int32_
   if (use_gemv(M, K)) return launch_gemv_x<bl::kXi8>(xq, packed, nullptr, acc, BL_I32, M, N, K, s);
   if (!ws) return BL_ERR_WORKSPACE;
   if (!aligned16(ws)) return BL_ERR_MISALIGNED;
+  if (ws_bytes < fwd_ws_bytes(M, N, K)) return BL_ERR_WORKSPACE;
   FwdWs w = fwd_ws_layout(ws, M, K);
-  if (ws_bytes < w.bytes) return BL_ERR_WORKSPACE;
   bl::rowsum_i8_kernel<<<M, bl::kAqThreads, 0, s>>>(xq, K, w.rowsum);
   if (launch_status() != BL_OK) return BL_ERR_CUDA;
+  if (M <= kSkinnyMaxM)
+    return launch_skinny(xq, packed, w.rowsum, nullptr, nullptr, acc, BL_I32, M, N, K, ws, s);
   return launch_gemm(xq, packed, w.rowsum, nullptr, nullptr, acc, BL_I32, M, N, K, s);
 }
 

@@ -1,0 +1,346 @@
+// Skinny BitLinear (4 < M <= 256 tokens) on the tcgen05 tensor cores, operands swapped:
+//   D[n][t] = sum_k u[n][k] * xq[t][k]     (A = 128 unpacked weight rows, B = the M tokens)
+// so the weights fill the MMA's 128-row slot and the few tokens its N slot (16..256), and
+// every weight tile is unpacked once no matter how many tokens there are. This is the
+// integer "addition" of BitNet b1.58 (dmarx anthology record LIT-380, Key takeaways
+// bullet 4) in the same u = c + 1 form as the other kernels (acc = D - rowsum_t).
+//
+// Three shared-memory rings:
+//   W  packed weight super-tiles: 128 rows x 128 bytes (512 K, four K blocks), one TMA box
+//      with the 128-byte swizzle, so every row is fetched as one 128-byte burst;
+//   X  int8 token tiles: bnt rows x 128 (one K block), 128-byte swizzle;
+//   U  unpacked weight tiles: 128 rows x 128 int8 in the swizzled K-major layout the MMA
+//      reads (several in flight, so unpacking runs ahead of the MMAs).
+//
+// Work unit = (128-row weight tile, K range of whole super-tiles). When there are too few
+// weight tiles to fill the GPU, K is split across CTAs: each split adds its exact int32
+// partial tile into a zeroed int32 buffer with fire-and-forget atomic adds, and the last
+// split to finish (per-tile arrival counter) rescales the sums and writes y. Integer
+// adds, so the split does not change a single bit.
+//
+// 6 warps: warps 0-3 unpack (thread t owns weight row t) during the main loop and run
+// the epilogue (TMEM lanes 32*w .. 32*w+31) at the end; warp 4 issues the TMA loads;
+// warp 5 allocates TMEM and issues the MMAs.
+#pragma once
+
+#include "common.cuh"
+#include "gemm_tc.cuh"
+
+namespace bl {
+
+namespace sk {
+constexpr int BW = 128;                 // weight rows per tile (MMA M)
+constexpr int BK = 128;                 // K per K block
+constexpr int KPS = 4;                  // K blocks per packed super-tile
+constexpr int MMA_K = 32;
+constexpr int WP_BYTES = BW * BK * KPS / 4;  // 16 KB packed super-tile
+constexpr int WU_BYTES = BW * BK;            // 16 KB unpacked tile
+constexpr int THREADS = 192;
+constexpr int MAX_SW = 4, MAX_SX = 8, MAX_SU = 4;
+
+struct Barriers {
+  uint64_t w_full[MAX_SW], w_empty[MAX_SW];
+  uint64_t x_full[MAX_SX], x_empty[MAX_SX];
+  uint64_t u_full[MAX_SU], u_empty[MAX_SU];
+  uint64_t acc_full;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+  int last;
+};
+
+struct Plan {
+  int sw, sx, su;
+};
+
+__host__ __device__ constexpr int x_tile_bytes(int bnt) { return bnt * BK; }
+// Shared memory per CTA: small token tiles keep two CTAs per SM, large ones use one.
+__host__ __device__ constexpr int smem_budget(int bnt) {
+  return bnt <= 64 ? 110 * 1024 : 200 * 1024;
+}
+__host__ __device__ constexpr Plan plan_for(int bnt) {
+  // 2 packed super-tiles, 4 unpacked tiles if the token tiles still double-buffer
+  int su = MAX_SU, sx = 0;
+  const int sw = 2;
+  const int room = smem_budget(bnt) - 1024 - static_cast<int>(sizeof(Barriers));
+  while (true) {
+    sx = (room - sw * WP_BYTES - su * WU_BYTES) / x_tile_bytes(bnt);
+    if (sx >= 2 || su == 2) break;
+    --su;
+  }
+  if (sx > MAX_SX) sx = MAX_SX;
+  return Plan{sw, sx, su};
+}
+__host__ __device__ constexpr int smem_bytes(int bnt) {
+  return 1024 + plan_for(bnt).sw * WP_BYTES + plan_for(bnt).sx * x_tile_bytes(bnt) +
+         plan_for(bnt).su * WU_BYTES + static_cast<int>(sizeof(Barriers));
+}
+__host__ __device__ constexpr uint32_t tmem_cols(int bnt) {
+  return bnt <= 32 ? 32u : bnt <= 64 ? 64u : bnt <= 128 ? 128u : 256u;
+}
+}  // namespace sk
+
+__device__ __forceinline__ void tmem_ld_x16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+
+// Fire-and-forget atomic add (the result is not returned, so the issuer does not wait).
+__device__ __forceinline__ void red_add_s32(int* p, int v) {
+  asm volatile("red.relaxed.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void epi_bar_sync() {  // the 4 unpack/epilogue warps only
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+
+// Rescales one accumulator and stores it. OM: 0 fp32, 1 bf16, 2 int32 (acc only).
+template <int OM>
+__device__ __forceinline__ void store_out(void* y, long long o, int a, float scale_t,
+                                          float gamma) {
+  if (OM == 2) {
+    static_cast<int*>(y)[o] = a;
+  } else {
+    const float val = __fmul_rn(__int2float_rn(a), __fmul_rn(scale_t, gamma));
+    if (OM == 0) static_cast<float*>(y)[o] = val;
+    else static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(val);
+  }
+}
+
+// bnt = token tile (multiple of 16, >= M). grid = n_tiles * splits; CTA u handles weight
+// tile u / splits and the K blocks [split * kbps, min(KB, (split + 1) * kbps)), kbps a
+// multiple of KPS.
+template <int OM>
+__global__ void __launch_bounds__(sk::THREADS, 1) gemm_skinny_kernel(
+    const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w,
+    const int* __restrict__ rowsum, const float* __restrict__ scale,
+    const float* __restrict__ gamma_ptr, void* __restrict__ y, int* __restrict__ partial,
+    unsigned int* __restrict__ counters, int M, int N, int K, int bnt, int splits,
+    int kb_per_split, unsigned long long limit_ns) {
+  using namespace sk;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const Plan pl = plan_for(bnt);
+  const int XB = x_tile_bytes(bnt);
+  unsigned char* sWp = smem;                    // SW x [128][128 B] swizzled
+  unsigned char* sWu = sWp + pl.sw * WP_BYTES;  // SU x [128][128] swizzled
+  unsigned char* sX = sWu + pl.su * WU_BYTES;   // SX x [bnt][128] swizzled
+  Barriers* bar = reinterpret_cast<Barriers*>(sX + pl.sx * XB);
+  volatile int* abort_flag = &bar->abort;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile = blockIdx.x / splits;
+  const int split = blockIdx.x % splits;
+  const int n0 = tile * BW;
+  const int KB = (K + BK - 1) / BK;
+  const int kb0 = split * kb_per_split;
+  const int kb1 = min(KB, kb0 + kb_per_split);
+  const uint32_t ncols = tmem_cols(bnt);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < pl.sw; ++i) {
+      mbar_init(&bar->w_full[i], 1);
+      mbar_init(&bar->w_empty[i], 4);
+    }
+    for (int i = 0; i < pl.sx; ++i) {
+      mbar_init(&bar->x_full[i], 1);
+      mbar_init(&bar->x_empty[i], 1);
+    }
+    for (int i = 0; i < pl.su; ++i) {
+      mbar_init(&bar->u_full[i], 4);
+      mbar_init(&bar->u_empty[i], 1);
+    }
+    mbar_init(&bar->acc_full, 1);
+    mbar_init(&bar->drain, 1);
+    bar->abort = 0;
+    bar->last = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(&bar->tmem_base, ncols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = bar->tmem_base;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&map_x);
+      prefetch_tmap(&map_w);
+      int sw = 0, sx = 0;
+      uint32_t wph = 0, xph = 0;
+      long long w_issued = 0, x_issued = 0;
+      bool ok = true;
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (((kb - kb0) & (KPS - 1)) == 0) {
+          if (!tc_wait(&bar->w_empty[sw], wph ^ 1u, limit_ns, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(&bar->w_full[sw], WP_BYTES);
+          tma_load_2d(sWp + sw * WP_BYTES, &map_w, kb * (BK / 4), n0, &bar->w_full[sw]);
+          ++w_issued;
+          if (++sw == pl.sw) { sw = 0; wph ^= 1u; }
+        }
+        if (!tc_wait(&bar->x_empty[sx], xph ^ 1u, limit_ns, abort_flag)) { ok = false; break; }
+        mbar_arrive_expect_tx(&bar->x_full[sx], XB);
+        tma_load_2d(sX + sx * XB, &map_x, kb * BK, 0, &bar->x_full[sx]);
+        ++x_issued;
+        if (++sx == pl.sx) { sx = 0; xph ^= 1u; }
+      }
+      if (!ok) {  // wait (bounded) for the copies still in flight
+        for (long long i = w_issued - 1; i >= 0 && i > w_issued - 1 - pl.sw; --i)
+          mbar_wait(&bar->w_full[i % pl.sw], static_cast<uint32_t>((i / pl.sw) & 1),
+                    100000000ull);
+        for (long long i = x_issued - 1; i >= 0 && i > x_issued - 1 - pl.sx; --i)
+          mbar_wait(&bar->x_full[i % pl.sx], static_cast<uint32_t>((i / pl.sx) & 1),
+                    100000000ull);
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_i8(BW, bnt);
+      int su = 0, sx = 0;
+      uint32_t uph = 0, xph = 0;
+      bool ok = true, issued_any = false;
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (!tc_wait(&bar->u_full[su], uph, limit_ns, abort_flag) ||
+            !tc_wait(&bar->x_full[sx], xph, limit_ns, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(sWu + su * WU_BYTES);
+        const uint32_t b_addr = smem_u32(sX + sx * XB);
+#pragma unroll
+        for (int kk = 0; kk < BK / MMA_K; ++kk)
+          mma_i8(tmem_base, smem_desc_k128(a_addr + kk * MMA_K),
+                 smem_desc_k128(b_addr + kk * MMA_K), idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+        issued_any = true;
+        mma_commit(&bar->u_empty[su]);
+        mma_commit(&bar->x_empty[sx]);
+        if (++su == pl.su) { su = 0; uph ^= 1u; }
+        if (++sx == pl.sx) { sx = 0; xph ^= 1u; }
+      }
+      if (ok) {
+        mma_commit(&bar->acc_full);
+      } else if (issued_any) {
+        mma_commit(&bar->drain);
+        mbar_wait(&bar->drain, 0u, 100000000ull);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ warps 0-3
+    const int r = threadIdx.x;  // weight row of the tile owned by this thread (0..127)
+    const int rs = r & 7;       // its 128-byte swizzle phase
+    int sw = 0, su = 0;
+    uint32_t wph = 0, uph = 0;
+    bool ok = true;
+    for (int kb = kb0; kb < kb1; ++kb) {
+      const int q = (kb - kb0) & (KPS - 1);
+      bool got = true;
+      if (q == 0) got = tc_wait(&bar->w_full[sw], wph, limit_ns, abort_flag);
+      got = got && tc_wait(&bar->u_empty[su], uph ^ 1u, limit_ns, abort_flag);
+      if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+      const unsigned char* src = sWp + sw * WP_BYTES + r * 128;
+      unsigned char* dst = sWu + su * WU_BYTES + r * 128;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        // logical 16-byte chunk 2q+h of the packed row = K block q, words 4h .. 4h+3
+        const uint4 p = *reinterpret_cast<const uint4*>(src + (((2 * q + h) ^ rs) << 4));
+        const uint32_t words[4] = {p.x, p.y, p.z, p.w};
+#pragma unroll
+        for (int mq = 0; mq < 4; ++mq) {
+          const uint32_t w = words[mq];
+          const int chunk = 4 * h + mq;  // 16-trit group = 16-byte chunk of the unpacked row
+          const uint4 o = make_uint4(w & 0x03030303u, (w >> 2) & 0x03030303u,
+                                     (w >> 4) & 0x03030303u, (w >> 6) & 0x03030303u);
+          *reinterpret_cast<uint4*>(dst + ((chunk ^ rs) << 4)) = o;
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar->u_full[su]);
+      if (++su == pl.su) { su = 0; uph ^= 1u; }
+      if (q == KPS - 1 || kb == kb1 - 1) {  // done with this packed super-tile
+        if (lane == 0) mbar_arrive(&bar->w_empty[sw]);
+        if (++sw == pl.sw) { sw = 0; wph ^= 1u; }
+      }
+    }
+    // ---------------------------------------------------------------- epilogue
+    const bool got = ok && tc_wait(&bar->acc_full, 0u, limit_ns, abort_flag);
+    if (__all_sync(0xffffffffu, got)) {
+      tc_fence_after();
+      const int n = n0 + warp * 32 + lane;  // this thread's TMEM lane = weight row
+      const bool nvalid = n < N;
+      const float gamma = (OM == 2) ? 0.0f : *gamma_ptr;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
+      if (splits == 1) {
+        for (int c0 = 0; c0 < bnt; c0 += 16) {
+          uint32_t v[16];
+          tmem_ld_x16(taddr + c0, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int t = c0 + j;
+            if (t < M && nvalid)
+              store_out<OM>(y, static_cast<long long>(t) * N + n,
+                            static_cast<int>(v[j]) - rowsum[t], OM == 2 ? 0.0f : scale[t],
+                            gamma);
+          }
+        }
+      } else {
+        // exact int32 partial of this split, added into acc32[t][n] (zeroed by the host)
+        for (int c0 = 0; c0 < bnt; c0 += 16) {
+          uint32_t v[16];
+          tmem_ld_x16(taddr + c0, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int t = c0 + j;
+            if (t < M && nvalid)
+              red_add_s32(partial + static_cast<long long>(t) * N + n, static_cast<int>(v[j]));
+          }
+        }
+        __threadfence();
+        epi_bar_sync();
+        if (threadIdx.x == 0) {
+          const unsigned int prev = atomicAdd(&counters[tile], 1u);
+          bar->last = (prev == static_cast<unsigned int>(splits - 1)) ? 1 : 0;
+        }
+        epi_bar_sync();
+        if (bar->last && nvalid) {
+          __threadfence();
+          for (int t0 = 0; t0 < M; t0 += 16) {
+            int a[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              a[j] = (t0 + j < M) ? __ldcg(partial + static_cast<long long>(t0 + j) * N + n) : 0;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int t = t0 + j;
+              if (t < M)
+                store_out<OM>(y, static_cast<long long>(t) * N + n, a[j] - rowsum[t],
+                              OM == 2 ? 0.0f : scale[t], gamma);
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, ncols);
+  }
+}
+
+}  // namespace bl

@@ -185,9 +185,11 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(
        rg * RPW < N; rg += warps_total) {
     const long long n = rg * RPW + rsel;
     const bool valid = n < N;
-    int acc[MT];
+    int acc4[MT][4];  // one chain per 4-trit group of a word: no long dp4a dependency
 #pragma unroll
-    for (int t = 0; t < MT; ++t) acc[t] = 0;
+    for (int t = 0; t < MT; ++t)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc4[t][j] = 0;
     if (valid) {
       const uint4* prow = reinterpret_cast<const uint4*>(packed + n * (K >> 2));
       for (int c0 = sub; c0 < CPR; c0 += LPR * kGemvUnroll) {
@@ -212,16 +214,19 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(
 #pragma unroll
               for (int t = 0; t < MT; ++t) {
                 const uint4 xv = xs4[t * xs_row_units + g * CPR + c];
-                acc[t] = __dp4a(r0, static_cast<int>(xv.x), acc[t]);
-                acc[t] = __dp4a(r1, static_cast<int>(xv.y), acc[t]);
-                acc[t] = __dp4a(r2, static_cast<int>(xv.z), acc[t]);
-                acc[t] = __dp4a(r3, static_cast<int>(xv.w), acc[t]);
+                acc4[t][0] = __dp4a(r0, static_cast<int>(xv.x), acc4[t][0]);
+                acc4[t][1] = __dp4a(r1, static_cast<int>(xv.y), acc4[t][1]);
+                acc4[t][2] = __dp4a(r2, static_cast<int>(xv.z), acc4[t][2]);
+                acc4[t][3] = __dp4a(r3, static_cast<int>(xv.w), acc4[t][3]);
               }
             }
           }
         }
       }
     }
+    int acc[MT];
+#pragma unroll
+    for (int t = 0; t < MT; ++t) acc[t] = (acc4[t][0] + acc4[t][1]) + (acc4[t][2] + acc4[t][3]);
     for (int off = LPR >> 1; off > 0; off >>= 1) {
 #pragma unroll
       for (int t = 0; t < MT; ++t) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], off);

@@ -92,6 +92,41 @@ def test_quantize_weights_exact_sum_edge_cases(kind):
         np.testing.assert_array_equal(packed.cpu().numpy(), ref_packed)
 
 
+def test_quantize_weights_rows_of_very_different_scale():
+    """Row blocks whose scale differs 100x: the per-block gamma guesses miss the final
+    threshold for many blocks, which then re-read their range. Codes stay exact."""
+    N, K = 2048, 1536
+    W = syn.weights(N, K, 1.0, seed=77)
+    scale = torch.where((torch.arange(N) // 64) % 2 == 0, 0.001, 0.1)
+    W = (W * scale[:, None]).contiguous()
+    packed, gamma = bl.quantize_weights(W.cuda())
+    ref_packed, ref_gamma = orc.quantize_weights(W.numpy(), 1e-5)
+    assert gamma.item() == float(ref_gamma)
+    np.testing.assert_array_equal(packed.cpu().numpy(), ref_packed)
+
+
+@pytest.mark.parametrize("ws_kind", ["full", "tiny"])
+def test_quantize_weights_many_ambiguous(ws_kind):
+    """Half of the weights sit within 1% of gamma/2: far more ambiguous entries than the
+    lists hold (always with the tiny workspace), so blocks fall back to a re-read."""
+    rng = np.random.default_rng(5)
+    N, K = 512, 2048
+    mag = np.where(rng.random(N * K) < 0.5, 0.5 * (1 + 0.01 * rng.uniform(-1, 1, N * K)), 1.5)
+    W = (mag * rng.choice([-1.0, 1.0], N * K) * 0.02).astype(np.float32).reshape(N, K)
+    Wd = torch.from_numpy(W).cuda()
+    lib = bl.load_library()
+    packed = torch.empty((N, K // 4), dtype=torch.uint8, device="cuda")
+    gamma = torch.empty(1, dtype=torch.float32, device="cuda")
+    ws = bl.workspace(1, N, K) if ws_kind == "full" else torch.empty(4096, dtype=torch.uint8, device="cuda")
+    rc = lib.bitlinear_quantize_weights(Wd.data_ptr(), 0, N, K, 1e-5, packed.data_ptr(),
+                                        gamma.data_ptr(), ws.data_ptr(), ws.numel(),
+                                        torch.cuda.current_stream().cuda_stream)
+    assert rc == 0
+    ref_packed, ref_gamma = orc.quantize_weights(W, 1e-5)
+    assert gamma.item() == float(ref_gamma)
+    np.testing.assert_array_equal(packed.cpu().numpy(), ref_packed)
+
+
 def test_ternarize_ties_on_device():
     """Weights exactly at 0.5 (gamma + eps) and one ulp either side."""
     d = np.float32(0.71875)
@@ -139,7 +174,8 @@ def test_quantize_acts_bit_exact(M, K, dtype, outliers):
 CONTRACT_SHAPES = [
     (1, 256, 256), (2, 293, 192), (3, 1000, 1536), (4, 777, 64),       # CUDA-core path
     (5, 300, 640), (16, 4096, 1536), (130, 293, 8640), (300, 520, 1536),  # tensor-core path
-    (129, 257, 128), (64, 64, 64),
+    (129, 257, 128), (64, 64, 64), (256, 1000, 3200), (257, 300, 640), (17, 8640, 3200),
+    (48, 129, 8640), (176, 520, 8192),
 ]
 
 
@@ -192,14 +228,17 @@ def test_forward_tiny_config_end_to_end():
     np.testing.assert_array_equal(y.cpu().numpy(), ref)
 
 
-def test_forward_paths_agree_at_the_switch():
-    """M = 4 runs the CUDA-core kernel, M = 5 the tensor-core GEMM: rows must agree."""
+@pytest.mark.parametrize("m_small,m_big", [(4, 5), (256, 257)])
+def test_forward_paths_agree_at_the_switch(m_small, m_big):
+    """M = 4 | 5 switches CUDA-core GEMV -> skinny tensor-core kernel; M = 256 | 257 switches
+    skinny -> prefill GEMM. Rows present in both calls must agree bit for bit (the per-token
+    quantization does not depend on the other tokens)."""
     W = syn.weights(1000, 1536, 0.02, seed=5)
-    x = syn.activations(5, 1536, seed=6)
+    x = syn.activations(m_big, 1536, seed=6)
     packed, gamma = bl.quantize_weights(W.cuda())
-    y5 = bl.forward(x.cuda(), packed, gamma, out_dtype=torch.float32)
-    y4 = bl.forward(x[:4].contiguous().cuda(), packed, gamma, out_dtype=torch.float32)
-    torch.testing.assert_close(y5[:4], y4, rtol=0, atol=0)
+    yb = bl.forward(x.cuda(), packed, gamma, out_dtype=torch.float32)
+    ys = bl.forward(x[:m_small].contiguous().cuda(), packed, gamma, out_dtype=torch.float32)
+    torch.testing.assert_close(yb[:m_small], ys, rtol=0, atol=0)
 
 
 # ----------------------------------------------------------------------------- full sizes
