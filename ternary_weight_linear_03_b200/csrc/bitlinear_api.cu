@@ -309,40 +309,35 @@ bl_status launch_act_quant(const void* x, int x_dtype, int M, int K, int8_t* xq,
 }
 
 // ------------------------------------------------------------------ weight quantization
-// Workspace of bitlinear_quantize_weights: the WqWorkspace header, then the per-block
-// lists of ambiguous weights (8 bytes each; room for n/32 of them in total). A smaller
-// workspace only makes more blocks re-read their range; results do not change.
-size_t wq_ws_bytes(long long n) {
-  return align_up(sizeof(WqWorkspace), 256) + align_up(static_cast<size_t>(n / 32) * 8, 256);
-}
+// Workspace of bitlinear_quantize_weights: the exponent buckets and the barrier counter.
+size_t wq_ws_bytes(long long) { return align_up(sizeof(WqWorkspace), 256); }
 
 template <bool kBf16>
 bl_status launch_weight_quant_t(const void* W, long long n, float eps, void* ws,
                                 size_t ws_bytes, float* gamma, uint32_t* packed,
                                 cudaStream_t s) {
   auto kern = bl::weight_quant_kernel<kBf16>;
+  constexpr int kSmem = bl::kWqStages * bl::kWqStageBytes;
   static int blocks_per_sm = 0;
   if (blocks_per_sm == 0) {
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_per_sm, kern, bl::kWqThreads, 0) !=
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) !=
             cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_per_sm, kern, bl::kWqThreads,
+                                                      kSmem) != cudaSuccess ||
         blocks_per_sm < 1)
       return BL_ERR_CUDA;
   }
-  const long long nwords = n / 16;
-  const long long want = (nwords + bl::kWqThreads * 4 - 1) / (bl::kWqThreads * 4);
+  // one block per 32 KB of weights at least, at most all resident blocks
+  const long long want = (n * (kBf16 ? 2 : 4) + 32767) / 32768;
   const int grid = static_cast<int>(
       std::max<long long>(1, std::min<long long>(want, 1ll * blocks_per_sm * num_sms())));
   WqWorkspace* hdr = static_cast<WqWorkspace*>(ws);
-  const size_t head = align_up(sizeof(WqWorkspace), 256);
-  unsigned long long* lists =
-      reinterpret_cast<unsigned long long*>(static_cast<char*>(ws) + head);
-  const long long room = (ws_bytes > head) ? static_cast<long long>((ws_bytes - head) / 8) : 0;
-  int cap = static_cast<int>(std::min<long long>(room / grid, 1ll << 30));
+  (void)ws_bytes;
   if (cudaMemsetAsync(hdr, 0, sizeof(WqWorkspace), s) != cudaSuccess) return BL_ERR_CUDA;
   unsigned long long limit = kWaitLimitNs;
-  void* args[] = {const_cast<void**>(&W), &n, &eps, &hdr, &lists, &cap, &gamma, &packed, &limit};
+  void* args[] = {const_cast<void**>(&W), &n, &eps, &hdr, &gamma, &packed, &limit};
   if (cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kern), dim3(grid),
-                                  dim3(bl::kWqThreads), args, 0, s) != cudaSuccess)
+                                  dim3(bl::kWqThreads), args, kSmem, s) != cudaSuccess)
     return BL_ERR_CUDA;
   return launch_status();
 }

@@ -5,12 +5,14 @@
 // integer "addition" of BitNet b1.58 (dmarx anthology record LIT-380, Key takeaways
 // bullet 4) in the same u = c + 1 form as the other kernels (acc = D - rowsum_t).
 //
-// Three shared-memory rings:
-//   W  packed weight super-tiles: 128 rows x 128 bytes (512 K, four K blocks), one TMA box
-//      with the 128-byte swizzle, so every row is fetched as one 128-byte burst;
-//   X  int8 token tiles: bnt rows x 128 (one K block), 128-byte swizzle;
-//   U  unpacked weight tiles: 128 rows x 128 int8 in the swizzled K-major layout the MMA
-//      reads (several in flight, so unpacking runs ahead of the MMAs).
+// Data path:
+//   W  packed weight super-tiles (128 rows x 128 bytes = 512 K, four K blocks) arrive by
+//      TMA with the 128-byte swizzle, so every row is one 128-byte burst;
+//   A  thread r of warps 0-3 unpacks its row's 128 trits of a K block in registers and
+//      writes them with one tcgen05.st into TMEM lane r (4 int8 per column): the MMA takes
+//      its A operand straight from tensor memory, so unpacked weights never touch shared
+//      memory (no shared-memory write/read traffic and no proxy fence for them);
+//   X  int8 token tiles (bnt rows x 128, one K block, 128-byte swizzle) in a deep ring.
 //
 // Work unit = (128-row weight tile, K range of whole super-tiles). When there are too few
 // weight tiles to fill the GPU, K is split across CTAs: each split adds its exact int32
@@ -18,9 +20,12 @@
 // split to finish (per-tile arrival counter) rescales the sums and writes y. Integer
 // adds, so the split does not change a single bit.
 //
-// 6 warps: warps 0-3 unpack (thread t owns weight row t) during the main loop and run
-// the epilogue (TMEM lanes 32*w .. 32*w+31) at the end; warp 4 issues the TMA loads;
-// warp 5 allocates TMEM and issues the MMAs.
+// The four MMAs of a K block write to up to four separate accumulators (summed in the
+// epilogue), so consecutive small-N MMAs do not serialize on one accumulator.
+//
+// 6 warps: warps 0-3 unpack (thread t owns weight row t, TMEM lane t) during the main loop
+// and run the epilogue at the end; warp 4 issues the TMA loads; warp 5 allocates TMEM and
+// issues the MMAs.
 #pragma once
 
 #include "common.cuh"
@@ -34,14 +39,15 @@ constexpr int BK = 128;                 // K per K block
 constexpr int KPS = 4;                  // K blocks per packed super-tile
 constexpr int MMA_K = 32;
 constexpr int WP_BYTES = BW * BK * KPS / 4;  // 16 KB packed super-tile
-constexpr int WU_BYTES = BW * BK;            // 16 KB unpacked tile
+constexpr int A_COLS = BK / 4;               // TMEM columns of one unpacked K block
+constexpr int SU = 4;                        // unpacked K blocks in flight (TMEM slots)
 constexpr int THREADS = 192;
-constexpr int MAX_SW = 4, MAX_SX = 8, MAX_SU = 4;
+constexpr int MAX_SW = 4, MAX_SX = 16;
 
 struct Barriers {
   uint64_t w_full[MAX_SW], w_empty[MAX_SW];
   uint64_t x_full[MAX_SX], x_empty[MAX_SX];
-  uint64_t u_full[MAX_SU], u_empty[MAX_SU];
+  uint64_t a_full[SU], a_empty[SU];
   uint64_t acc_full;
   uint64_t drain;
   uint32_t tmem_base;
@@ -50,7 +56,7 @@ struct Barriers {
 };
 
 struct Plan {
-  int sw, sx, su;
+  int sw, sx;
 };
 
 __host__ __device__ constexpr int x_tile_bytes(int bnt) { return bnt * BK; }
@@ -59,24 +65,29 @@ __host__ __device__ constexpr int smem_budget(int bnt) {
   return bnt <= 64 ? 110 * 1024 : 200 * 1024;
 }
 __host__ __device__ constexpr Plan plan_for(int bnt) {
-  // 2 packed super-tiles, 4 unpacked tiles if the token tiles still double-buffer
-  int su = MAX_SU, sx = 0;
-  const int sw = 2;
-  const int room = smem_budget(bnt) - 1024 - static_cast<int>(sizeof(Barriers));
-  while (true) {
-    sx = (room - sw * WP_BYTES - su * WU_BYTES) / x_tile_bytes(bnt);
-    if (sx >= 2 || su == 2) break;
-    --su;
-  }
-  if (sx > MAX_SX) sx = MAX_SX;
-  return Plan{sw, sx, su};
+  const int sw = bnt <= 64 ? 4 : 2;
+  const int room = smem_budget(bnt) - 1024 - static_cast<int>(sizeof(Barriers)) - sw * WP_BYTES;
+  const int sx = room / x_tile_bytes(bnt);
+  return Plan{sw, sx > MAX_SX ? MAX_SX : sx};
 }
 __host__ __device__ constexpr int smem_bytes(int bnt) {
   return 1024 + plan_for(bnt).sw * WP_BYTES + plan_for(bnt).sx * x_tile_bytes(bnt) +
-         plan_for(bnt).su * WU_BYTES + static_cast<int>(sizeof(Barriers));
+         static_cast<int>(sizeof(Barriers));
 }
-__host__ __device__ constexpr uint32_t tmem_cols(int bnt) {
+// Columns of one accumulator (bnt rounded up to a power of two, at least 32).
+__host__ __device__ constexpr uint32_t acc_cols(int bnt) {
   return bnt <= 32 ? 32u : bnt <= 64 ? 64u : bnt <= 128 ? 128u : 256u;
+}
+// Independent accumulators: the 4 MMAs of a K block go to different ones, so a small-N
+// MMA does not wait for the one before it to finish its read-modify-write of D. Chosen
+// so that the accumulators plus the SU unpacked A slots fit 256 TMEM columns for small
+// token tiles (two CTAs per SM) and 512 for large ones.
+__host__ __device__ constexpr int n_acc(int bnt) {
+  return bnt <= 32 ? 4 : bnt <= 128 ? 2 : 1;
+}
+// TMEM allocation: accumulators, then SU unpacked A slots; a power of two.
+__host__ __device__ constexpr uint32_t tmem_cols(int bnt) {
+  return n_acc(bnt) * acc_cols(bnt) + SU * A_COLS <= 256u ? 256u : 512u;
 }
 }  // namespace sk
 
@@ -89,6 +100,47 @@ __device__ __forceinline__ void tmem_ld_x16(uint32_t taddr, uint32_t (&r)[16]) {
         "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr)
       : "memory");
+}
+
+// Each thread of the warp writes 32 consecutive 32-bit columns of its own TMEM lane.
+__device__ __forceinline__ void tmem_st_x32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+      "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+// D[tmem] (+)= A[tmem] * B[smem]^T, int8 x int8 -> int32, one CTA.
+__device__ __forceinline__ void mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// 16 columns of this thread's TMEM lane, summed over the nacc accumulators (exact int32).
+__device__ __forceinline__ void ld_acc_sum(uint32_t taddr, int nacc, uint32_t acol,
+                                           uint32_t (&v)[16]) {
+  tmem_ld_x16(taddr, v);
+  tmem_ld_wait();
+  for (int i = 1; i < nacc; ++i) {
+    uint32_t w[16];
+    tmem_ld_x16(taddr + static_cast<uint32_t>(i) * acol, w);
+    tmem_ld_wait();
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[j] += w[j];
+  }
 }
 
 // Fire-and-forget atomic add (the result is not returned, so the issuer does not wait).
@@ -130,8 +182,7 @@ __global__ void __launch_bounds__(sk::THREADS, 1) gemm_skinny_kernel(
   const Plan pl = plan_for(bnt);
   const int XB = x_tile_bytes(bnt);
   unsigned char* sWp = smem;                    // SW x [128][128 B] swizzled
-  unsigned char* sWu = sWp + pl.sw * WP_BYTES;  // SU x [128][128] swizzled
-  unsigned char* sX = sWu + pl.su * WU_BYTES;   // SX x [bnt][128] swizzled
+  unsigned char* sX = sWp + pl.sw * WP_BYTES;   // SX x [bnt][128] swizzled
   Barriers* bar = reinterpret_cast<Barriers*>(sX + pl.sx * XB);
   volatile int* abort_flag = &bar->abort;
 
@@ -143,6 +194,9 @@ __global__ void __launch_bounds__(sk::THREADS, 1) gemm_skinny_kernel(
   const int kb0 = split * kb_per_split;
   const int kb1 = min(KB, kb0 + kb_per_split);
   const uint32_t ncols = tmem_cols(bnt);
+  const int nacc = n_acc(bnt);
+  const uint32_t acol = acc_cols(bnt);
+  const uint32_t a_col0 = nacc * acol;  // first TMEM column of the unpacked A slots
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < pl.sw; ++i) {
@@ -153,9 +207,9 @@ __global__ void __launch_bounds__(sk::THREADS, 1) gemm_skinny_kernel(
       mbar_init(&bar->x_full[i], 1);
       mbar_init(&bar->x_empty[i], 1);
     }
-    for (int i = 0; i < pl.su; ++i) {
-      mbar_init(&bar->u_full[i], 4);
-      mbar_init(&bar->u_empty[i], 1);
+    for (int i = 0; i < SU; ++i) {
+      mbar_init(&bar->a_full[i], 4);
+      mbar_init(&bar->a_empty[i], 1);
     }
     mbar_init(&bar->acc_full, 1);
     mbar_init(&bar->drain, 1);
@@ -212,19 +266,23 @@ __global__ void __launch_bounds__(sk::THREADS, 1) gemm_skinny_kernel(
       uint32_t uph = 0, xph = 0;
       bool ok = true, issued_any = false;
       for (int kb = kb0; kb < kb1; ++kb) {
-        if (!tc_wait(&bar->u_full[su], uph, limit_ns, abort_flag) ||
+        if (!tc_wait(&bar->a_full[su], uph, limit_ns, abort_flag) ||
             !tc_wait(&bar->x_full[sx], xph, limit_ns, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t a_addr = smem_u32(sWu + su * WU_BYTES);
+        const uint32_t a_tmem = tmem_base + a_col0 + static_cast<uint32_t>(su * A_COLS);
         const uint32_t b_addr = smem_u32(sX + sx * XB);
 #pragma unroll
-        for (int kk = 0; kk < BK / MMA_K; ++kk)
-          mma_i8(tmem_base, smem_desc_k128(a_addr + kk * MMA_K),
-                 smem_desc_k128(b_addr + kk * MMA_K), idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < BK / MMA_K; ++kk) {
+          const int ai = kk % nacc;  // accumulator of this MMA
+          mma_i8_ts(tmem_base + static_cast<uint32_t>(ai) * acol,
+                    a_tmem + static_cast<uint32_t>(kk * (MMA_K / 4)),
+                    smem_desc_k128(b_addr + kk * MMA_K), idesc,
+                    (kb > kb0 || kk >= nacc) ? 1u : 0u);
+        }
         issued_any = true;
-        mma_commit(&bar->u_empty[su]);
+        mma_commit(&bar->a_empty[su]);
         mma_commit(&bar->x_empty[sx]);
-        if (++su == pl.su) { su = 0; uph ^= 1u; }
+        if (++su == SU) { su = 0; uph ^= 1u; }
         if (++sx == pl.sx) { sx = 0; xph ^= 1u; }
       }
       if (ok) {
@@ -245,10 +303,11 @@ __global__ void __launch_bounds__(sk::THREADS, 1) gemm_skinny_kernel(
       const int q = (kb - kb0) & (KPS - 1);
       bool got = true;
       if (q == 0) got = tc_wait(&bar->w_full[sw], wph, limit_ns, abort_flag);
-      got = got && tc_wait(&bar->u_empty[su], uph ^ 1u, limit_ns, abort_flag);
+      got = got && tc_wait(&bar->a_empty[su], uph ^ 1u, limit_ns, abort_flag);
       if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+      tc_fence_after();
       const unsigned char* src = sWp + sw * WP_BYTES + r * 128;
-      unsigned char* dst = sWu + su * WU_BYTES + r * 128;
+      uint32_t a[32];  // the row's 128 unpacked codes of this K block, 4 per register
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         // logical 16-byte chunk 2q+h of the packed row = K block q, words 4h .. 4h+3
@@ -257,16 +316,21 @@ __global__ void __launch_bounds__(sk::THREADS, 1) gemm_skinny_kernel(
 #pragma unroll
         for (int mq = 0; mq < 4; ++mq) {
           const uint32_t w = words[mq];
-          const int chunk = 4 * h + mq;  // 16-trit group = 16-byte chunk of the unpacked row
-          const uint4 o = make_uint4(w & 0x03030303u, (w >> 2) & 0x03030303u,
-                                     (w >> 4) & 0x03030303u, (w >> 6) & 0x03030303u);
-          *reinterpret_cast<uint4*>(dst + ((chunk ^ rs) << 4)) = o;
+          const int c = 16 * h + 4 * mq;  // first column of this 16-trit group
+          a[c + 0] = w & 0x03030303u;
+          a[c + 1] = (w >> 2) & 0x03030303u;
+          a[c + 2] = (w >> 4) & 0x03030303u;
+          a[c + 3] = (w >> 6) & 0x03030303u;
         }
       }
-      fence_proxy_async_smem();
+      tmem_st_x32(tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + a_col0 +
+                      static_cast<uint32_t>(su * A_COLS),
+                  a);
+      tmem_st_wait();
+      tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bar->u_full[su]);
-      if (++su == pl.su) { su = 0; uph ^= 1u; }
+      if (lane == 0) mbar_arrive(&bar->a_full[su]);
+      if (++su == SU) { su = 0; uph ^= 1u; }
       if (q == KPS - 1 || kb == kb1 - 1) {  // done with this packed super-tile
         if (lane == 0) mbar_arrive(&bar->w_empty[sw]);
         if (++sw == pl.sw) { sw = 0; wph ^= 1u; }
@@ -283,8 +347,7 @@ __global__ void __launch_bounds__(sk::THREADS, 1) gemm_skinny_kernel(
       if (splits == 1) {
         for (int c0 = 0; c0 < bnt; c0 += 16) {
           uint32_t v[16];
-          tmem_ld_x16(taddr + c0, v);
-          tmem_ld_wait();
+          ld_acc_sum(taddr + c0, nacc, acol, v);
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int t = c0 + j;
@@ -298,8 +361,7 @@ __global__ void __launch_bounds__(sk::THREADS, 1) gemm_skinny_kernel(
         // exact int32 partial of this split, added into acc32[t][n] (zeroed by the host)
         for (int c0 = 0; c0 < bnt; c0 += 16) {
           uint32_t v[16];
-          tmem_ld_x16(taddr + c0, v);
-          tmem_ld_wait();
+          ld_acc_sum(taddr + c0, nacc, acol, v);
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int t = c0 + j;

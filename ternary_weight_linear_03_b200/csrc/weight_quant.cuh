@@ -2,20 +2,15 @@
 // takeaways bullet 1: weights constrained to {-1, 0, +1} by an absmean quantization
 // function; searcharxiv.com abstract page, Abstract: every weight is ternary).
 //
-// One cooperative kernel that reads W from HBM once:
-//   1  every block streams its own contiguous range of 16-weight words and
-//      a) adds every |w| into an exact sum (below),
-//      b) ternarizes provisionally against a bracket [T_lo, T_hi] of the final threshold,
-//         estimated from the block's first 4096 weights: |w| >= T_hi is +-1, |w| < T_lo is 0,
-//         anything in between is written as 0 and appended (index, value) to the block's
-//         list of ambiguous weights (a few percent),
-//      and writes its packed words.
+// One cooperative kernel, two lean passes over W (the second is served from L2 whenever W
+// fits there). Every block owns a contiguous range of 16-weight words and streams it
+// through a ring of 16 KB bulk copies (cp.async.bulk into shared memory, 4 in flight per
+// block); thread t handles the 16-byte chunks t + 256 i of each stage.
+//   A  exact sum of |w| (below) into exponent buckets;
 //   -- grid barrier (bounded wait) --
-//   2  every block turns the exact sum into gamma = fl32(fl64(S) / n) and the threshold T
-//   3  if T lies inside the block's bracket and its list did not overflow, only the listed
-//      weights are re-decided (atomicXor of their 2-bit fields); otherwise the block
-//      re-reads its range and ternarizes it again with T. Either way every code equals
-//      RoundClip(fl(w / (gamma + eps)), -1, 1).
+//      every block turns the buckets into gamma = fl32(fl64(S) / n) and the threshold T;
+//   B  code = (w >= T) - (-w >= T), stored as u = code + 1; the 4 (fp32) or 2 (bf16) lanes
+//      holding the chunks of one packed word merge their bits with shuffles.
 //
 // Threshold. RoundClip(fl(w/d), -1, 1) is +1 exactly when fl(w/d) > 0.5 (0.5 itself
 // rounds to the even 0, and every quotient >= 1.5 clips to 1). Correctly rounded
@@ -23,14 +18,15 @@
 // c = +1 iff w >= T, c = -1 iff -w >= T.
 //
 // Exact sum. Each warp fixes an exponent window [base, base + 20] from the largest
-// exponent in its first loads (base = that exponent - 17, at least 1). A float |w| in the
+// exponent in its first stage (base = that exponent - 17, at least 1). A float |w| in the
 // window is an integer multiple of u = 2^(base - 150) below 2^44 u, so up to 256 of them
-// add up exactly in a double; a thread keeps two such doubles (weights k % 2 of each
-// word, so the additions do not form one long dependency chain) and every 16 words
-// converts them to integers and adds those into 64-bit exponent buckets (low 32 bits at
-// exponent base, the rest at base + 32). Values outside the window (subnormals, far larger or smaller ones)
-// go straight into the buckets as (exponent, 24-bit mantissa). The buckets are summed
-// exactly, so gamma depends neither on the grid nor on the order of the atomic adds.
+// add up exactly in a double; a thread keeps two such doubles (alternate weights, so the
+// additions do not form one long dependency chain) and every 16 stages the warp converts
+// them to integers, sums those with shuffles and adds the result into 64-bit exponent
+// buckets (low 32 bits at exponent base, the rest at base + 32). Values outside the
+// window (subnormals, far larger or smaller ones) go straight into the buckets as
+// (exponent, 24-bit mantissa). The buckets are summed exactly, so gamma depends neither
+// on the grid nor on the order of the atomic adds.
 #pragma once
 
 #include "act_quant.cuh"
@@ -43,10 +39,8 @@ constexpr int kWqThreads = 256;
 constexpr int kWqLimbs = 14;     // 32-bit limbs of the exact sum (S * 2^149 < 2^448)
 constexpr int kWqWindow = 21;    // exponents covered by the fp64 window
 constexpr int kWqFlushWords = 16;  // words a thread sums in fp64 between bucket flushes
-constexpr float kWqBand = 0.03f;   // relative half-width of the per-block gamma bracket
 
-// Header of the quantize_weights workspace (zeroed by the host before each launch). It is
-// followed by gridDim.x lists of `cap` ambiguous-weight entries (uint64 each).
+// The quantize_weights workspace (zeroed by the host before each launch).
 struct WqWorkspace {
   unsigned long long buckets[kWqBuckets];
   unsigned int arrived;  // grid-barrier arrivals
@@ -66,15 +60,22 @@ __device__ __forceinline__ void wq_fallback(uint32_t bits, unsigned long long* s
   }
 }
 
-// Moves a thread's fp64 window sum into the buckets: acc is an integer multiple of
-// 2^(base-150) below 2^53 of those units, so the scaled conversion is exact.
-__device__ __forceinline__ void wq_flush(double& acc, int base, unsigned long long* sb) {
-  if (acc != 0.0) {
-    const double scale = __longlong_as_double(static_cast<long long>(1023 + 150 - base) << 52);
-    const unsigned long long u = __double2ull_rz(__dmul_rn(acc, scale));
+// Moves a warp's fp64 window sums into the buckets. Called by all 32 lanes together (the
+// window base is the same for the whole warp). Each lane's a0 + a1 is an integer multiple
+// of 2^(base-150) below 2^52 of those units, so the scaled conversion is exact; the warp
+// adds the 32 integers with shuffles (below 2^57) and one lane adds the low 32 bits at
+// exponent base and the rest at base + 32, so the shared buckets see 2 atomics per warp.
+__device__ __forceinline__ void wq_flush(double& a0, double& a1, int base,
+                                         unsigned long long* sb) {
+  const double scale = __longlong_as_double(static_cast<long long>(1023 + 150 - base) << 52);
+  unsigned long long u = __double2ull_rz(__dmul_rn(__dadd_rn(a0, a1), scale));
+  a0 = 0.0;
+  a1 = 0.0;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) u += __shfl_xor_sync(0xffffffffu, u, off);
+  if ((threadIdx.x & 31) == 0 && u != 0ull) {
     atomicAdd(&sb[base], u & 0xffffffffull);
     if (u >> 32) atomicAdd(&sb[base + 32], u >> 32);
-    acc = 0.0;
   }
 }
 
@@ -126,213 +127,201 @@ __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
   return v;
 }
 
-// The 16 weights of word wi as floats (fp32, or bf16 widened exactly).
-template <bool kBf16>
-__device__ __forceinline__ void wq_load_word(const uint4* v, long long wi, uint4 (&raw)[4]) {
-  if (kBf16) {
-    raw[0] = ld_stream_v4(v + 2 * wi);
-    raw[1] = ld_stream_v4(v + 2 * wi + 1);
-  } else {
-#pragma unroll
-    for (int q = 0; q < 4; ++q) raw[q] = ld_stream_v4(v + 4 * wi + q);
-  }
+// 1-D bulk copy global -> shared, completing on an mbarrier (no tensor map, no multicast).
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
 }
+
+constexpr int kWqStageBytes = 16384;  // one bulk copy
+constexpr int kWqStages = 4;          // ring depth per block
+constexpr int kWqChunks = kWqStageBytes / 16 / kWqThreads;  // 16-byte chunks per thread
+
+// The weights of one 16-byte chunk as floats: 4 fp32 or 8 bf16 (widened exactly).
 template <bool kBf16>
-__device__ __forceinline__ void wq_unpack_word(const uint4 (&raw)[4], float (&w)[16]) {
+__device__ __forceinline__ void wq_chunk_floats(const uint4 c, float (&w)[kBf16 ? 8 : 4]) {
   if (kBf16) {
-    const uint32_t h[8] = {raw[0].x, raw[0].y, raw[0].z, raw[0].w,
-                           raw[1].x, raw[1].y, raw[1].z, raw[1].w};
+    const uint32_t h[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
+    for (int q = 0; q < 4; ++q) {
       w[2 * q] = __uint_as_float(h[q] << 16);
       w[2 * q + 1] = __uint_as_float(h[q] & 0xffff0000u);
     }
   } else {
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      w[4 * q + 0] = __uint_as_float(raw[q].x);
-      w[4 * q + 1] = __uint_as_float(raw[q].y);
-      w[4 * q + 2] = __uint_as_float(raw[q].z);
-      w[4 * q + 3] = __uint_as_float(raw[q].w);
-    }
+    w[0] = __uint_as_float(c.x);
+    w[1] = __uint_as_float(c.y);
+    w[2] = __uint_as_float(c.z);
+    w[3] = __uint_as_float(c.w);
   }
 }
 
-// Exact codes of one word against the final threshold T.
-__device__ __forceinline__ uint32_t wq_pack16(const float (&w)[16], float T) {
-  uint32_t word = 0u;
-#pragma unroll
-  for (int k = 0; k < 16; ++k) {
-    const uint32_t u = 1u + (w[k] >= T ? 1u : 0u) - (-w[k] >= T ? 1u : 0u);
-    word |= u << wq_shift(k);
-  }
-  return word;
+// Position in its packed word of element e of a chunk: a word holds 16 weights = 4 fp32
+// chunks (chunk part p = 0..3) or 2 bf16 chunks (p = 0..1); relative index k = E*p + e.
+template <bool kBf16>
+__device__ __forceinline__ int wq_k(int part, int e) {
+  return (kBf16 ? 8 : 4) * part + e;
+}
+
+// OR of a value over the lanes that hold the parts of one packed word.
+template <bool kBf16>
+__device__ __forceinline__ uint32_t wq_or_parts(uint32_t v) {
+  v |= __shfl_xor_sync(0xffffffffu, v, 1);
+  if (!kBf16) v |= __shfl_xor_sync(0xffffffffu, v, 2);
+  return v;
+}
+
+// Streams the block's byte range [src, src + bytes) through the stage ring; `g` counts
+// the stages this block has consumed so far (slot and phase parity follow from it).
+struct WqRing {
+  unsigned char* stage;  // kWqStages x kWqStageBytes
+  uint64_t* full;        // kWqStages mbarriers
+  const char* src;
+  long long bytes;
+  int nst;               // stages of one pass over the range
+};
+
+// Issues stage st of a pass (bytes st * 16 KB ..) as the block's g-th stage overall.
+__device__ __forceinline__ void wq_issue(const WqRing& r, int st, int g) {
+  const uint32_t nb = static_cast<uint32_t>(
+      min(static_cast<long long>(kWqStageBytes), r.bytes - 1ll * st * kWqStageBytes));
+  const int slot = g % kWqStages;
+  mbar_arrive_expect_tx(&r.full[slot], nb);
+  bulk_load(r.stage + slot * kWqStageBytes, r.src + 1ll * st * kWqStageBytes, nb, &r.full[slot]);
 }
 
 // W holds n values (fp32, or bf16 if kBf16), n % 16 == 0, 16-byte aligned. Launched
-// cooperatively (all blocks resident). ws: header zeroed by the host, then gridDim.x
-// ambiguous lists of cap entries.
+// cooperatively (all blocks resident) with kWqStages * kWqStageBytes of dynamic shared
+// memory. ws is zeroed by the host.
 template <bool kBf16>
 __global__ void __launch_bounds__(kWqThreads) weight_quant_kernel(
     const void* __restrict__ W, long long n, float eps, WqWorkspace* __restrict__ ws,
-    unsigned long long* __restrict__ lists, int cap, float* __restrict__ gamma_out,
-    uint32_t* __restrict__ packed, unsigned long long limit_ns) {
+    float* __restrict__ gamma_out, uint32_t* __restrict__ packed, unsigned long long limit_ns) {
+  extern __shared__ __align__(128) unsigned char wq_stage[];  // kWqStages x 16 KB
   __shared__ unsigned long long sb[kWqBuckets];
   __shared__ unsigned long long col[kWqLimbs];
-  __shared__ float s_red[2][kWqThreads / 32];
-  __shared__ float s_Tlo, s_Thi, s_T;
-  __shared__ unsigned int s_cnt;
+  __shared__ uint64_t full[kWqStages];
+  __shared__ float s_T;
   __shared__ int s_ok;
-  for (int i = threadIdx.x; i < kWqBuckets; i += blockDim.x) sb[i] = 0ull;
-  if (threadIdx.x < kWqLimbs) col[threadIdx.x] = 0ull;
-  if (threadIdx.x == 0) s_cnt = 0u;
+  constexpr int E = kBf16 ? 8 : 4;   // weights per 16-byte chunk
+  constexpr int PARTS = 16 / E;      // chunks per packed word
+  constexpr int WORD_BYTES = kBf16 ? 32 : 64;
 
-  const uint4* __restrict__ v = static_cast<const uint4*>(W);
+  const int tid = threadIdx.x;
+  for (int i = tid; i < kWqBuckets; i += blockDim.x) sb[i] = 0ull;
+  if (tid < kWqLimbs) col[tid] = 0ull;
   const long long nwords = n / 16;
   const long long per_block = (nwords + gridDim.x - 1) / gridDim.x;
   const long long wb0 = min(nwords, static_cast<long long>(blockIdx.x) * per_block);
   const long long wb1 = min(nwords, wb0 + per_block);
-  unsigned long long* list = lists + static_cast<long long>(blockIdx.x) * cap;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-
-  // ---------------------------------------------------------------- first words
-  long long wi = wb0 + threadIdx.x;
-  uint4 cur[4] = {}, nxt[4] = {};
-  if (wi < wb1) wq_load_word<kBf16>(v, wi, cur);
-  float w[16];
-  wq_unpack_word<kBf16>(cur, w);
-  int emax = 0;
-  float asum = 0.0f, acnt = 0.0f;
-  if (wi < wb1) {
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      const uint32_t b = __float_as_uint(w[k]) & 0x7fffffffu;
-      const int e = static_cast<int>(b >> 23);
-      if (e != 255) {
-        emax = max(emax, e);
-        asum += __uint_as_float(b);
-        acnt += 1.0f;
-      }
-    }
-  }
-  emax = __reduce_max_sync(0xffffffffu, emax);
-  const int base = max(1, emax + 4 - kWqWindow);
-  const float lo_f = __uint_as_float(static_cast<uint32_t>(base) << 23);
-  const float hi_f = (base + kWqWindow <= 254)
-                         ? __uint_as_float(static_cast<uint32_t>(base + kWqWindow) << 23)
-                         : __int_as_float(0x7f800000);
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    asum += __shfl_xor_sync(0xffffffffu, asum, off);
-    acnt += __shfl_xor_sync(0xffffffffu, acnt, off);
-  }
-  if (lane == 0) {
-    s_red[0][warp] = asum;
-    s_red[1][warp] = acnt;
+  WqRing ring;
+  ring.stage = wq_stage;
+  ring.full = full;
+  ring.src = static_cast<const char*>(W) + wb0 * WORD_BYTES;
+  ring.bytes = (wb1 - wb0) * WORD_BYTES;
+  ring.nst = static_cast<int>((ring.bytes + kWqStageBytes - 1) / kWqStageBytes);
+  if (tid == 0) {
+    s_ok = 1;
+    for (int i = 0; i < kWqStages; ++i) mbar_init(&full[i], 1);
+    fence_mbar_init();
+    for (int st = 0; st < min(ring.nst, kWqStages); ++st) wq_issue(ring, st, st);
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    float sum = 0.0f, cnt = 0.0f;
-    for (int i = 0; i < kWqThreads / 32; ++i) {
-      sum += s_red[0][i];
-      cnt += s_red[1][i];
-    }
-    const float ghat = (cnt > 0.0f) ? sum / cnt : 0.0f;
-    s_Tlo = 0.5f * (ghat * (1.0f - kWqBand) + eps) * (1.0f - 1e-6f);
-    s_Thi = 0.5f * (ghat * (1.0f + kWqBand) + eps) * (1.0f + 1e-6f);
-  }
-  __syncthreads();
-  const float Tlo = s_Tlo, Thi = s_Thi;
 
-  // ---------------------------------------------------------------- phase 1: one pass
-  double acc[2] = {0.0, 0.0};  // two independent chains (k % 2)
+  // ---------------------------------------------------------------- pass A: exact sum
+  double acc0 = 0.0, acc1 = 0.0;
   bool nonfinite = false;
-  int since_flush = 0;
-  for (; wi < wb1; wi += kWqThreads) {
-    const long long wn = wi + kWqThreads;
-    if (wn < wb1) wq_load_word<kBf16>(v, wn, nxt);
-    // Common path, branch-free: fp64 window sum, provisional code, two any-flags.
-    uint32_t word = 0u;
-    bool out_any = false, amb_any = false;
+  int base = 1;
+  float lo_f = 0.0f, hi_f = 0.0f;
+  for (int st = 0; st < ring.nst; ++st) {
+    const int slot = st % kWqStages;
+    if (!mbar_wait(&full[slot], static_cast<uint32_t>((st / kWqStages) & 1), limit_ns)) s_ok = 0;
+    const uint4* stage = reinterpret_cast<const uint4*>(wq_stage + slot * kWqStageBytes);
+    const int nchunks = static_cast<int>(
+        min(static_cast<long long>(kWqStageBytes), ring.bytes - 1ll * st * kWqStageBytes) / 16);
+    uint4 ch[kWqChunks];
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      const float x = w[k];
-      const float a = abs_bits(x);
-      const bool in = (a >= lo_f) & (a < hi_f);
-      out_any |= !in;
-      acc[k & 1] += static_cast<double>(in ? a : 0.0f);  // exact: see the header
-      const bool big = a >= Thi;
-      const uint32_t neg = __float_as_uint(x) >> 31;
-      word += (big ? 2u - 2u * neg : 1u) << wq_shift(k);
-      amb_any |= (!big) & (a >= Tlo);
+    for (int i = 0; i < kWqChunks; ++i) {
+      const int c = tid + i * kWqThreads;
+      ch[i] = (c < nchunks) ? stage[c] : make_uint4(0u, 0u, 0u, 0u);  // zeros add nothing
     }
-    // Rare paths: weights outside the window (zeros included) and ambiguous weights.
-    if (out_any) {
+    if (st == 0) {  // exponent window of this warp
+      int emax = 0;
 #pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        const float a = abs_bits(w[k]);
-        if (!((a >= lo_f) & (a < hi_f)) && a != 0.0f)
-          wq_fallback(__float_as_uint(a), sb, nonfinite);
+      for (int i = 0; i < kWqChunks; ++i) {
+        float w[E];
+        wq_chunk_floats<kBf16>(ch[i], w);
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const int ex = static_cast<int>((__float_as_uint(w[e]) >> 23) & 0xffu);
+          if (ex != 255) emax = max(emax, ex);
+        }
       }
+      emax = __reduce_max_sync(0xffffffffu, emax);
+      base = max(1, emax + 4 - kWqWindow);
+      lo_f = __uint_as_float(static_cast<uint32_t>(base) << 23);
+      hi_f = (base + kWqWindow <= 254)
+                 ? __uint_as_float(static_cast<uint32_t>(base + kWqWindow) << 23)
+                 : __int_as_float(0x7f800000);
     }
-    if (amb_any) {
-      uint32_t m16 = 0u;
 #pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        const float a = abs_bits(w[k]);
-        m16 |= ((a < Thi) & (a >= Tlo) ? 1u : 0u) << k;
+    for (int i = 0; i < kWqChunks; ++i) {
+      float w[E];
+      wq_chunk_floats<kBf16>(ch[i], w);
+      bool out_any = false;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const float a = abs_bits(w[e]);
+        const bool in = (a >= lo_f) & (a < hi_f);
+        out_any |= !in;
+        if (e & 1) acc1 += static_cast<double>(in ? a : 0.0f);  // exact: see the header
+        else acc0 += static_cast<double>(in ? a : 0.0f);
       }
-      unsigned int slot = atomicAdd(&s_cnt, static_cast<unsigned int>(__popc(m16)));
+      if (out_any) {  // rare: zeros and values outside the window
 #pragma unroll
-      for (int k = 0; k < 16; ++k) {  // constant indices keep w[] in registers
-        if ((m16 >> k) & 1u) {
-          if (slot < static_cast<unsigned int>(cap))
-            list[slot] = (static_cast<unsigned long long>(__float_as_uint(w[k])) << 32) |
-                         (static_cast<unsigned long long>(wi) << 4) | static_cast<unsigned>(k);
-          ++slot;
+        for (int e = 0; e < E; ++e) {
+          const float a = abs_bits(w[e]);
+          if (!((a >= lo_f) & (a < hi_f)) && a != 0.0f)
+            wq_fallback(__float_as_uint(a), sb, nonfinite);
         }
       }
     }
-    packed[wi] = word;
-    if (++since_flush == kWqFlushWords) {
-#pragma unroll
-      for (int j = 0; j < 2; ++j) wq_flush(acc[j], base, sb);
-      since_flush = 0;
-    }
-#pragma unroll
-    for (int q = 0; q < 4; ++q) cur[q] = nxt[q];
-    wq_unpack_word<kBf16>(cur, w);
+    if ((st & 15) == 15) wq_flush(acc0, acc1, base, sb);
+    __syncthreads();  // every thread is done with this slot
+    if (tid == 0 && st + kWqStages < ring.nst) wq_issue(ring, st + kWqStages, st + kWqStages);
   }
-#pragma unroll
-  for (int j = 0; j < 2; ++j) wq_flush(acc[j], base, sb);
+  wq_flush(acc0, acc1, base, sb);
   if (nonfinite) record_status(kStatusNonfinite);
   __syncthreads();
-  for (int i = threadIdx.x; i < kWqBuckets; i += blockDim.x)
+  for (int i = tid; i < kWqBuckets; i += blockDim.x)
     if (sb[i]) atomicAdd(&ws->buckets[i], sb[i]);
+  // pass B starts streaming now; its stages do not depend on gamma
+  if (tid == 0)
+    for (int st = 0; st < min(ring.nst, kWqStages); ++st) wq_issue(ring, st, ring.nst + st);
 
   // ---------------------------------------------------------------- grid barrier
   __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) {
+  if (tid == 0) {
     atomicAdd(&ws->arrived, 1u);
-    int ok = 1;
     const uint64_t t0 = global_ns();
     while (ld_acquire_u32(&ws->arrived) < gridDim.x) {
       if (global_ns() - t0 > limit_ns) {
         record_status(kStatusTimeout);
-        ok = 0;
+        s_ok = 0;
         break;
       }
       __nanosleep(64);
     }
-    s_ok = ok;
   }
   __syncthreads();
-  if (!s_ok) return;
 
-  // ---------------------------------------------------------------- phase 2: gamma, T
+  // ---------------------------------------------------------------- gamma and T
   // Column sums: bucket e contributes B[e] << ((e-1) % 32) to limbs (e-1)/32 .. +2.
-  for (int e = 1 + threadIdx.x; e < kWqBuckets; e += blockDim.x) {
+  for (int e = 1 + tid; e < kWqBuckets; e += blockDim.x) {
     const unsigned long long b = __ldcg(&ws->buckets[e]);
     if (b == 0ull) continue;
     const int pos = e - 1, wd = pos >> 5, sh = pos & 31;
@@ -343,7 +332,7 @@ __global__ void __launch_bounds__(kWqThreads) weight_quant_kernel(
     if (p2) atomicAdd(&col[wd + 2], static_cast<unsigned long long>(p2));
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
+  if (tid == 0) {
     uint32_t L[kWqLimbs];
     unsigned long long carry = 0ull;
 #pragma unroll
@@ -359,27 +348,39 @@ __global__ void __launch_bounds__(kWqThreads) weight_quant_kernel(
   }
   __syncthreads();
 
-  // ---------------------------------------------------------------- phase 3: settle
+  // ---------------------------------------------------------------- pass B: codes
   const float T = s_T;
-  const unsigned int cnt = s_cnt;
-  if (T >= Tlo && T <= Thi && cnt <= static_cast<unsigned int>(cap)) {
-    for (unsigned int i = threadIdx.x; i < cnt; i += blockDim.x) {
-      const unsigned long long e = list[i];
-      const float x = __uint_as_float(static_cast<uint32_t>(e >> 32));
-      const long long widx = static_cast<long long>((e & 0xffffffffull) >> 4);
-      const int k = static_cast<int>(e & 15ull);
-      const uint32_t u = 1u + (x >= T ? 1u : 0u) - (-x >= T ? 1u : 0u);
-      if (u != 1u) atomicXor(&packed[widx], (1u ^ u) << wq_shift(k));
+  const int part = tid & (PARTS - 1);  // which part of its packed word this thread holds
+  uint32_t mul[E];                     // 1 << bit position of element e of this part
+#pragma unroll
+  for (int e = 0; e < E; ++e) mul[e] = 1u << wq_shift(wq_k<kBf16>(part, e));
+  for (int st = 0; st < ring.nst; ++st) {
+    const int g = ring.nst + st;  // stages consumed by this block so far
+    const int slot = g % kWqStages;
+    if (!mbar_wait(&full[slot], static_cast<uint32_t>((g / kWqStages) & 1), limit_ns)) s_ok = 0;
+    const uint4* stage = reinterpret_cast<const uint4*>(wq_stage + slot * kWqStageBytes);
+    const int nchunks = static_cast<int>(
+        min(static_cast<long long>(kWqStageBytes), ring.bytes - 1ll * st * kWqStageBytes) / 16);
+#pragma unroll
+    for (int i = 0; i < kWqChunks; ++i) {
+      const int c = tid + i * kWqThreads;
+      float w[E];
+      wq_chunk_floats<kBf16>((c < nchunks) ? stage[c] : make_uint4(0u, 0u, 0u, 0u), w);
+      uint32_t bits = 0u;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const uint32_t u = (abs_bits(w[e]) >= T) ? 2u - ((__float_as_uint(w[e]) >> 30) & 2u) : 1u;
+        bits += u * mul[e];
+      }
+      bits = wq_or_parts<kBf16>(bits);
+      if (c < nchunks && part == 0)
+        packed[wb0 + (1ll * st * kWqStageBytes + 16ll * c) / WORD_BYTES] = bits;
     }
-  } else {
-    for (long long wj = wb0 + threadIdx.x; wj < wb1; wj += kWqThreads) {
-      uint4 raw[4] = {};
-      float ww[16];
-      wq_load_word<kBf16>(v, wj, raw);
-      wq_unpack_word<kBf16>(raw, ww);
-      packed[wj] = wq_pack16(ww, T);
-    }
+    __syncthreads();
+    if (tid == 0 && st + kWqStages < ring.nst)
+      wq_issue(ring, st + kWqStages, ring.nst + st + kWqStages);
   }
+  (void)s_ok;
 }
 
 }  // namespace bl
