@@ -38,6 +38,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+from ternary_weight_linear_03_b200 import dist as bldist  # noqa: E402
 from ternary_weight_linear_03_b200 import synthetic as syn  # noqa: E402
 
 METRIC = "BitLinear tokens/s; decode HBM GB/s and prefill INT8 TOPS as % of roofline"
@@ -55,6 +56,22 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     return p.parse_args()
+
+
+def ncu_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu capture, or None when the
+    capture was of another workload or the kernel source changed since it was taken."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    src = os.path.join(ROOT, "ternary_weight_linear_03_b200", "csrc", "weight_quant.cuh")
+    try:
+        rec = json.load(open(path))[kernel]
+        sha = hashlib.sha1(open(src, "rb").read()).hexdigest()
+    except (OSError, KeyError, ValueError):
+        return None
+    if rec.get("workload") != workload or rec.get("source_sha1") != sha:
+        return None
+    return rec["dram_bytes_per_launch"]
 
 
 def peaks():
@@ -208,9 +225,7 @@ def main():
 
     import ternary_weight_linear_03_b200 as bl
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, world, local = bldist.rank_env()
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device (no CPU fallback)")
     torch.cuda.set_device(local)
@@ -227,7 +242,7 @@ def main():
     N, K = wl["N"], wl["K"]
     w_bytes = N * K * 4
     copies = max(2, math.ceil(2 * L2_BYTES / w_bytes))
-    N, K, Ws, xs = make_inputs(name, M, device, copies, seed_offset=7919 * rank)
+    N, K, Ws, xs = make_inputs(name, M, device, copies, seed_offset=bldist.seed_offset(rank))
     packed = torch.empty((N, K // 4), dtype=torch.uint8, device=device)
     gamma = torch.empty(1, dtype=torch.float32, device=device)
     y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
@@ -277,11 +292,7 @@ def main():
         torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
-    elapsed_ms = start.elapsed_time(end)
-    if dist is not None:
-        t = torch.tensor([elapsed_ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = t.item()
+    elapsed_ms = bldist.max_over_ranks(start.elapsed_time(end), dist, device)
     status = bl.get_device_status()
     if status != 0:
         raise SystemExit(f"device status {bl.status_string(status)} after the timed region")
@@ -294,12 +305,13 @@ def main():
     fw_bytes = N * K // 4 + M * K * 2 + M * N * 2
     if wq_ms >= fw_ms:
         dom = {"kernel": "bitlinear_quantize_weights (absmean + ternarize/pack)",
-               "bytes": wq_bytes, "ms": wq_ms}
+               "bytes": wq_bytes, "ms": wq_ms,
+               "traffic": ncu_traffic("weight_quant_kernel", name)}
     else:
-        dom = {"kernel": "bitlinear_forward", "bytes": fw_bytes, "ms": fw_ms}
+        dom = {"kernel": "bitlinear_forward", "bytes": fw_bytes, "ms": fw_ms, "traffic": None}
     achieved = dom["bytes"] / (dom["ms"] * 1e-3) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                "frac": achieved / hbm_peak, "traffic": None, "peak_source": peak_kind,
+                "frac": achieved / hbm_peak, "traffic": dom["traffic"], "peak_source": peak_kind,
                 "kernel": dom["kernel"], "algorithmic_bytes": dom["bytes"],
                 "ms_per_launch": dom["ms"],
                 "others": {"quantize_weights_ms": wq_ms, "forward_ms": fw_ms,
@@ -337,11 +349,7 @@ def main():
             y_h.copy_(y, non_blocking=True)
         e2.record(stream)
         torch.cuda.synchronize()
-        e_ms = s2.elapsed_time(e2)
-        if dist is not None:
-            t = torch.tensor([e_ms], device=device)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = t.item()
+        e_ms = bldist.max_over_ranks(s2.elapsed_time(e2), dist, device)
         e2e = {"value": M * e2e_steps * world / (e_ms * 1e-3), "unit": "tokens/s",
                "h2d_bytes_per_step": W_h.numel() * 4 + x_h.numel() * x_h.element_size(),
                "d2h_bytes_per_step": y_h.numel() * 2, "steps": e2e_steps}
