@@ -262,6 +262,8 @@ __global__ void __launch_bounds__(sk::THREADS, 1) gemm_skinny_kernel(
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc = idesc_i8(BW, bnt);
+      // built once; a stage or K step only moves the 14-bit start-address field
+      const uint64_t x_desc0 = smem_desc_k128(smem_u32(sX));
       int su = 0, sx = 0;
       uint32_t uph = 0, xph = 0;
       bool ok = true, issued_any = false;
@@ -270,13 +272,13 @@ __global__ void __launch_bounds__(sk::THREADS, 1) gemm_skinny_kernel(
             !tc_wait(&bar->x_full[sx], xph, limit_ns, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t a_tmem = tmem_base + a_col0 + static_cast<uint32_t>(su * A_COLS);
-        const uint32_t b_addr = smem_u32(sX + sx * XB);
+        const uint64_t b_desc = x_desc0 + static_cast<uint64_t>(sx * (XB >> 4));
 #pragma unroll
         for (int kk = 0; kk < BK / MMA_K; ++kk) {
           const int ai = kk % nacc;  // accumulator of this MMA
           mma_i8_ts(tmem_base + static_cast<uint32_t>(ai) * acol,
                     a_tmem + static_cast<uint32_t>(kk * (MMA_K / 4)),
-                    smem_desc_k128(b_addr + kk * MMA_K), idesc,
+                    b_desc + static_cast<uint64_t>(kk * (MMA_K >> 4)), idesc,
                     (kb > kb0 || kk >= nacc) ? 1u : 0u);
         }
         issued_any = true;

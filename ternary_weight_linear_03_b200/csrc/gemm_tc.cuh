@@ -156,6 +156,10 @@ __global__ void __launch_bounds__(tc::THREADS, 1) gemm_tc_kernel(
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
+      // Descriptors are built once; a stage or K step only moves the 14-bit start-address
+      // field (16-byte units), which keeps the single issuing thread's work per MMA tiny.
+      const uint64_t a_desc0 = smem_desc_k128(smem_u32(sA));
+      const uint64_t b_desc0 = smem_desc_k128(smem_u32(sBu));
       int s = 0, u = 0, ab = 0;
       uint32_t ph = 0, uph = 0, aph = 0;
       bool ok = true, issued_any = false;
@@ -167,12 +171,13 @@ __global__ void __launch_bounds__(tc::THREADS, 1) gemm_tc_kernel(
           if (!tc_wait(&bar->full_unp[u], uph, limit_ns, abort_flag) ||
               !tc_wait(&bar->full_tma[s], ph, limit_ns, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(sA + s * A_BYTES);
-          const uint32_t b_addr = smem_u32(sBu + u * BU_BYTES);
+          const uint64_t a_desc = a_desc0 + static_cast<uint64_t>(s * (A_BYTES >> 4));
+          const uint64_t b_desc = b_desc0 + static_cast<uint64_t>(u * (BU_BYTES >> 4));
 #pragma unroll
           for (int kk = 0; kk < BK / MMA_K; ++kk) {
-            mma_i8(d_tmem, smem_desc_k128(a_addr + kk * MMA_K), smem_desc_k128(b_addr + kk * MMA_K),
-                   IDESC, (kb | kk) != 0 ? 1u : 0u);
+            mma_i8(d_tmem, a_desc + static_cast<uint64_t>(kk * (MMA_K >> 4)),
+                   b_desc + static_cast<uint64_t>(kk * (MMA_K >> 4)), IDESC,
+                   (kb | kk) != 0 ? 1u : 0u);
           }
           issued_any = true;
           mma_commit(&bar->empty_tma[s]);
