@@ -20,12 +20,16 @@
 // split to finish (per-tile arrival counter) rescales the sums and writes y. Integer
 // adds, so the split does not change a single bit.
 //
-// The four MMAs of a K block write to up to four separate accumulators (summed in the
-// epilogue), so consecutive small-N MMAs do not serialize on one accumulator.
+// The loop moves in groups of KG = 2 K blocks. Per group the four unpack warps write
+// their rows' codes to TMEM, meet at a named barrier (bar.sync of 128 threads, far cheaper
+// than an mbarrier arrive/poll round trip), and warp 0 then issues the group's 8 MMAs and
+// one commit; its barrier (done ring) frees the A slot and the token tile. At small M
+// each MMA is a few tens of cycles of tensor work, so the kernel's pace is set by these
+// per-group synchronisation hops, not by bandwidth.
 //
-// 6 warps: warps 0-3 unpack (thread t owns weight row t, TMEM lane t) during the main loop
-// and run the epilogue at the end; warp 4 issues the TMA loads; warp 5 allocates TMEM and
-// issues the MMAs.
+// 5 warps: warps 0-3 unpack (thread t owns weight row t, TMEM lane t), warp 0 also issues
+// the MMAs (whole-warp loop, one elected lane issues, operands precomputed) and owns the
+// TMEM allocation; the four run the epilogue at the end. Warp 4 issues the TMA loads.
 #pragma once
 
 #include "common.cuh"
@@ -35,19 +39,35 @@ namespace bl {
 
 namespace sk {
 constexpr int BW = 128;                 // weight rows per tile (MMA M)
-constexpr int BK = 128;                 // K per K block
+constexpr int BK = 128;                 // K per K block (one 128-byte swizzle row of int8)
 constexpr int KPS = 4;                  // K blocks per packed super-tile
+constexpr int KG = 2;                   // K blocks per group (one synchronisation round)
 constexpr int MMA_K = 32;
 constexpr int WP_BYTES = BW * BK * KPS / 4;  // 16 KB packed super-tile
 constexpr int A_COLS = BK / 4;               // TMEM columns of one unpacked K block
-constexpr int SU = 4;                        // unpacked K blocks in flight (TMEM slots)
-constexpr int THREADS = 192;
+constexpr int G_COLS = KG * A_COLS;          // TMEM columns of one unpacked group
+constexpr int MAX_SU = 8;                    // unpacked groups in flight (TMEM slots), at most
+constexpr int THREADS = 160;
 constexpr int MAX_SW = 4, MAX_SX = 16;
+#ifndef SK_PREFETCH
+#define SK_PREFETCH 8
+#endif
+// W super-tiles prefetched into L2 ahead of the one being loaded: HBM latency under load
+// needs far more bytes in flight than the shared-memory ring holds.
+constexpr int PF = SK_PREFETCH;
+static_assert(KPS % KG == 0, "groups tile a super-tile");
+// Ring of per-group completion barriers. Group g's MMAs arrive on done[g % SD]; the
+// unpackers wait for group g - SU before reusing A slot g % SU, the producer for group
+// g - SX before reusing token slot g % SX. SD >= SU and SD >= SX make a waited-for phase
+// unable to be overtaken by the next phase of the same barrier (that one needs the
+// waiter's own later work first), and every waiter waits on every index in order.
+constexpr int SD = 16;
+static_assert(SD >= MAX_SU && SD >= MAX_SX && (SD & (SD - 1)) == 0, "done ring");
 
 struct Barriers {
   uint64_t w_full[MAX_SW], w_empty[MAX_SW];
-  uint64_t x_full[MAX_SX], x_empty[MAX_SX];
-  uint64_t a_full[SU], a_empty[SU];
+  uint64_t x_full[MAX_SX];
+  uint64_t done[SD];
   uint64_t acc_full;
   uint64_t drain;
   uint32_t tmem_base;
@@ -59,7 +79,9 @@ struct Plan {
   int sw, sx;
 };
 
+// One token tile of a K block: bnt rows x 128 bytes; a group holds KG of them.
 __host__ __device__ constexpr int x_tile_bytes(int bnt) { return bnt * BK; }
+__host__ __device__ constexpr int x_group_bytes(int bnt) { return KG * x_tile_bytes(bnt); }
 // Shared memory per CTA: small token tiles keep two CTAs per SM, large ones use one.
 __host__ __device__ constexpr int smem_budget(int bnt) {
   return bnt <= 64 ? 110 * 1024 : 200 * 1024;
@@ -67,28 +89,27 @@ __host__ __device__ constexpr int smem_budget(int bnt) {
 __host__ __device__ constexpr Plan plan_for(int bnt) {
   const int sw = bnt <= 64 ? 4 : 2;
   const int room = smem_budget(bnt) - 1024 - static_cast<int>(sizeof(Barriers)) - sw * WP_BYTES;
-  const int sx = room / x_tile_bytes(bnt);
+  const int sx = room / x_group_bytes(bnt);
   return Plan{sw, sx > MAX_SX ? MAX_SX : sx};
 }
 __host__ __device__ constexpr int smem_bytes(int bnt) {
-  return 1024 + plan_for(bnt).sw * WP_BYTES + plan_for(bnt).sx * x_tile_bytes(bnt) +
+  return 1024 + plan_for(bnt).sw * WP_BYTES + plan_for(bnt).sx * x_group_bytes(bnt) +
          static_cast<int>(sizeof(Barriers));
 }
-// Columns of one accumulator (bnt rounded up to a power of two, at least 32).
+// Columns of the accumulator (bnt rounded up to a power of two, at least 32).
 __host__ __device__ constexpr uint32_t acc_cols(int bnt) {
   return bnt <= 32 ? 32u : bnt <= 64 ? 64u : bnt <= 128 ? 128u : 256u;
 }
-// Independent accumulators: the 4 MMAs of a K block go to different ones, so a small-N
-// MMA does not wait for the one before it to finish its read-modify-write of D. Chosen
-// so that the accumulators plus the SU unpacked A slots fit 256 TMEM columns for small
-// token tiles (two CTAs per SM) and 512 for large ones.
-__host__ __device__ constexpr int n_acc(int bnt) {
-  return bnt <= 32 ? 4 : bnt <= 128 ? 2 : 1;
+// TMEM allocation: 256 columns for small token tiles (two CTAs per SM), else 512.
+__host__ __device__ constexpr uint32_t tmem_cols(int bnt) { return bnt <= 64 ? 256u : 512u; }
+// Unpacked A slots in flight: the rest of the allocation after the accumulator.
+__host__ __device__ constexpr int n_slots(int bnt) {
+  return (static_cast<int>(tmem_cols(bnt)) - static_cast<int>(acc_cols(bnt))) / G_COLS > MAX_SU
+             ? MAX_SU
+             : (static_cast<int>(tmem_cols(bnt)) - static_cast<int>(acc_cols(bnt))) / G_COLS;
 }
-// TMEM allocation: accumulators, then SU unpacked A slots; a power of two.
-__host__ __device__ constexpr uint32_t tmem_cols(int bnt) {
-  return n_acc(bnt) * acc_cols(bnt) + SU * A_COLS <= 256u ? 256u : 512u;
-}
+static_assert(n_slots(16) >= 3 && n_slots(64) >= 3 && n_slots(128) >= 4 && n_slots(256) >= 4,
+              "TMEM slot budget");
 }  // namespace sk
 
 __device__ __forceinline__ void tmem_ld_x16(uint32_t taddr, uint32_t (&r)[16]) {
@@ -118,29 +139,24 @@ __device__ __forceinline__ void tmem_st_x32(uint32_t taddr, const uint32_t (&r)[
 __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
-// D[tmem] (+)= A[tmem] * B[smem]^T, int8 x int8 -> int32, one CTA.
-__device__ __forceinline__ void mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                          uint32_t idesc, uint32_t accumulate) {
+// D[tmem] (+)= A[tmem] * B[smem]^T, int8 x int8 -> int32, one CTA; warp-collective like
+// mma_i8_elect (one elected lane issues).
+__device__ __forceinline__ void mma_i8_ts_elect(uint32_t d_tmem, uint32_t a_tmem,
+                                                uint64_t b_desc, uint32_t idesc,
+                                                uint32_t accumulate) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "@e tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
-// 16 columns of this thread's TMEM lane, summed over the nacc accumulators (exact int32).
-__device__ __forceinline__ void ld_acc_sum(uint32_t taddr, int nacc, uint32_t acol,
-                                           uint32_t (&v)[16]) {
+// 16 consecutive accumulator columns of this thread's TMEM lane.
+__device__ __forceinline__ void ld_acc16(uint32_t taddr, uint32_t (&v)[16]) {
   tmem_ld_x16(taddr, v);
   tmem_ld_wait();
-  for (int i = 1; i < nacc; ++i) {
-    uint32_t w[16];
-    tmem_ld_x16(taddr + static_cast<uint32_t>(i) * acol, w);
-    tmem_ld_wait();
-#pragma unroll
-    for (int j = 0; j < 16; ++j) v[j] += w[j];
-  }
 }
 
 // Fire-and-forget atomic add (the result is not returned, so the issuer does not wait).
@@ -150,6 +166,20 @@ __device__ __forceinline__ void red_add_s32(int* p, int v) {
 
 __device__ __forceinline__ void epi_bar_sync() {  // the 4 unpack/epilogue warps only
   asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+// Named barrier of the 4 unpack/epilogue warps that also returns the OR of every thread's
+// flag, so that all 128 threads take the same branch afterwards.
+__device__ __forceinline__ bool epi_bar_or(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v))
+      : "memory");
+  return r != 0;
 }
 
 // Rescales one accumulator and stores it. OM: 0 fp32, 1 bf16, 2 int32 (acc only).
@@ -167,7 +197,8 @@ __device__ __forceinline__ void store_out(void* y, long long o, int a, float sca
 
 // bnt = token tile (multiple of 16, >= M). grid = n_tiles * splits; CTA u handles weight
 // tile u / splits and the K blocks [split * kbps, min(KB, (split + 1) * kbps)), kbps a
-// multiple of KPS.
+// multiple of KPS. A trailing partial group reads K blocks past KB, which the tensor maps
+// fill with zeros (their products vanish).
 template <int OM>
 __global__ void __launch_bounds__(sk::THREADS, 1) gemm_skinny_kernel(
     const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w,
@@ -181,9 +212,10 @@ __global__ void __launch_bounds__(sk::THREADS, 1) gemm_skinny_kernel(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const Plan pl = plan_for(bnt);
   const int XB = x_tile_bytes(bnt);
+  const int XG = x_group_bytes(bnt);
   unsigned char* sWp = smem;                    // SW x [128][128 B] swizzled
-  unsigned char* sX = sWp + pl.sw * WP_BYTES;   // SX x [bnt][128] swizzled
-  Barriers* bar = reinterpret_cast<Barriers*>(sX + pl.sx * XB);
+  unsigned char* sX = sWp + pl.sw * WP_BYTES;   // SX x KG x [bnt][128] swizzled
+  Barriers* bar = reinterpret_cast<Barriers*>(sX + pl.sx * XG);
   volatile int* abort_flag = &bar->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -193,31 +225,25 @@ __global__ void __launch_bounds__(sk::THREADS, 1) gemm_skinny_kernel(
   const int KB = (K + BK - 1) / BK;
   const int kb0 = split * kb_per_split;
   const int kb1 = min(KB, kb0 + kb_per_split);
+  const int ng = (kb1 - kb0 + KG - 1) / KG;  // groups of this CTA
   const uint32_t ncols = tmem_cols(bnt);
-  const int nacc = n_acc(bnt);
-  const uint32_t acol = acc_cols(bnt);
-  const uint32_t a_col0 = nacc * acol;  // first TMEM column of the unpacked A slots
+  const uint32_t a_col0 = acc_cols(bnt);  // first TMEM column of the unpacked A slots
+  const int SU = n_slots(bnt);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < pl.sw; ++i) {
       mbar_init(&bar->w_full[i], 1);
-      mbar_init(&bar->w_empty[i], 4);
+      mbar_init(&bar->w_empty[i], 1);
     }
-    for (int i = 0; i < pl.sx; ++i) {
-      mbar_init(&bar->x_full[i], 1);
-      mbar_init(&bar->x_empty[i], 1);
-    }
-    for (int i = 0; i < SU; ++i) {
-      mbar_init(&bar->a_full[i], 4);
-      mbar_init(&bar->a_empty[i], 1);
-    }
+    for (int i = 0; i < pl.sx; ++i) mbar_init(&bar->x_full[i], 1);
+    for (int i = 0; i < SD; ++i) mbar_init(&bar->done[i], 1);
     mbar_init(&bar->acc_full, 1);
     mbar_init(&bar->drain, 1);
     bar->abort = 0;
     bar->last = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == 0) {
     tmem_alloc(&bar->tmem_base, ncols);
     tmem_relinquish();
   }
@@ -232,24 +258,42 @@ __global__ void __launch_bounds__(sk::THREADS, 1) gemm_skinny_kernel(
       prefetch_tmap(&map_x);
       prefetch_tmap(&map_w);
       int sw = 0, sx = 0;
-      uint32_t wph = 0, xph = 0;
+      uint32_t wph = 0;
       long long w_issued = 0, x_issued = 0;
       bool ok = true;
-      for (int kb = kb0; kb < kb1; ++kb) {
-        if (((kb - kb0) & (KPS - 1)) == 0) {
+      const int nst = (kb1 - kb0 + KPS - 1) / KPS;  // super-tiles of this CTA
+      for (int i = 0; i < PF && i < nst; ++i)
+        tma_prefetch_l2_2d(&map_w, (kb0 + i * KPS) * (BK / 4), n0);
+      for (int g = 0; g < ng; ++g) {
+        const int kb = kb0 + g * KG;
+        if (((g * KG) & (KPS - 1)) == 0) {
+          const int st = (g * KG) / KPS;
+          if (st + PF < nst) tma_prefetch_l2_2d(&map_w, (kb0 + (st + PF) * KPS) * (BK / 4), n0);
           if (!tc_wait(&bar->w_empty[sw], wph ^ 1u, limit_ns, abort_flag)) { ok = false; break; }
           mbar_arrive_expect_tx(&bar->w_full[sw], WP_BYTES);
           tma_load_2d(sWp + sw * WP_BYTES, &map_w, kb * (BK / 4), n0, &bar->w_full[sw]);
           ++w_issued;
           if (++sw == pl.sw) { sw = 0; wph ^= 1u; }
         }
-        if (!tc_wait(&bar->x_empty[sx], xph ^ 1u, limit_ns, abort_flag)) { ok = false; break; }
-        mbar_arrive_expect_tx(&bar->x_full[sx], XB);
-        tma_load_2d(sX + sx * XB, &map_x, kb * BK, 0, &bar->x_full[sx]);
+        if (g >= pl.sx) {  // token slot sx is free once group g - SX has been consumed
+          const int i = g - pl.sx;
+          if (!tc_wait(&bar->done[i & (SD - 1)], static_cast<uint32_t>((i / SD) & 1), limit_ns,
+                       abort_flag)) { ok = false; break; }
+        }
+        mbar_arrive_expect_tx(&bar->x_full[sx], XG);
+#pragma unroll
+        for (int kq = 0; kq < KG; ++kq)
+          tma_load_2d(sX + sx * XG + kq * XB, &map_x, (kb + kq) * BK, 0, &bar->x_full[sx]);
         ++x_issued;
-        if (++sx == pl.sx) { sx = 0; xph ^= 1u; }
+        if (++sx == pl.sx) sx = 0;
       }
-      if (!ok) {  // wait (bounded) for the copies still in flight
+      if (ok) {
+        // The last commits' arrivals land on done[] asynchronously: see each barrier's final
+        // phase before the CTA can exit, so no arrival reaches a later CTA's shared memory.
+        for (int i = max(0, ng - SD); i < ng; ++i)
+          if (!tc_wait(&bar->done[i & (SD - 1)], static_cast<uint32_t>((i / SD) & 1), limit_ns,
+                       abort_flag)) break;
+      } else {  // wait (bounded) for the copies still in flight
         for (long long i = w_issued - 1; i >= 0 && i > w_issued - 1 - pl.sw; --i)
           mbar_wait(&bar->w_full[i % pl.sw], static_cast<uint32_t>((i / pl.sw) & 1),
                     100000000ull);
@@ -258,89 +302,104 @@ __global__ void __launch_bounds__(sk::THREADS, 1) gemm_skinny_kernel(
                     100000000ull);
       }
     }
-  } else if (warp == 5) {
-    // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc = idesc_i8(BW, bnt);
-      // built once; a stage or K step only moves the 14-bit start-address field
-      const uint64_t x_desc0 = smem_desc_k128(smem_u32(sX));
-      int su = 0, sx = 0;
-      uint32_t uph = 0, xph = 0;
-      bool ok = true, issued_any = false;
-      for (int kb = kb0; kb < kb1; ++kb) {
-        if (!tc_wait(&bar->a_full[su], uph, limit_ns, abort_flag) ||
-            !tc_wait(&bar->x_full[sx], xph, limit_ns, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t a_tmem = tmem_base + a_col0 + static_cast<uint32_t>(su * A_COLS);
-        const uint64_t b_desc = x_desc0 + static_cast<uint64_t>(sx * (XB >> 4));
-#pragma unroll
-        for (int kk = 0; kk < BK / MMA_K; ++kk) {
-          const int ai = kk % nacc;  // accumulator of this MMA
-          mma_i8_ts(tmem_base + static_cast<uint32_t>(ai) * acol,
-                    a_tmem + static_cast<uint32_t>(kk * (MMA_K / 4)),
-                    b_desc + static_cast<uint64_t>(kk * (MMA_K >> 4)), idesc,
-                    (kb > kb0 || kk >= nacc) ? 1u : 0u);
-        }
-        issued_any = true;
-        mma_commit(&bar->a_empty[su]);
-        mma_commit(&bar->x_empty[sx]);
-        if (++su == SU) { su = 0; uph ^= 1u; }
-        if (++sx == pl.sx) { sx = 0; xph ^= 1u; }
-      }
-      if (ok) {
-        mma_commit(&bar->acc_full);
-      } else if (issued_any) {
-        mma_commit(&bar->drain);
-        mbar_wait(&bar->drain, 0u, 100000000ull);
-      }
-    }
   } else {
     // ------------------------------------------------------------------ warps 0-3
     const int r = threadIdx.x;  // weight row of the tile owned by this thread (0..127)
     const int rs = r & 7;       // its 128-byte swizzle phase
-    int sw = 0, su = 0;
-    uint32_t wph = 0, uph = 0;
-    bool ok = true;
-    for (int kb = kb0; kb < kb1; ++kb) {
-      const int q = (kb - kb0) & (KPS - 1);
+    const uint32_t a_lane = tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + a_col0;
+    // MMA operands (used by warp 0): built once; a stage or K step only moves the
+    // descriptor's 14-bit start-address field or the TMEM column
+    const uint32_t idesc = idesc_i8(BW, bnt);
+    const uint64_t x_desc0 = smem_desc_k128(smem_u32(sX));
+    const uint32_t a_tmem0 = tmem_base + a_col0;
+    int sw = 0, su = 0, sx = 0;
+    uint32_t wph = 0, xph = 0;
+    int g = 0;
+    for (; g < ng; ++g) {
+      const int q0 = (g * KG) & (KPS - 1);  // first K block of the group in its super-tile
+      // lane 0 waits for the warp; __syncwarp then orders the other lanes after it. A warp
+      // whose wait fails skips its work but still meets the others at the named barrier.
       bool got = true;
-      if (q == 0) got = tc_wait(&bar->w_full[sw], wph, limit_ns, abort_flag);
-      got = got && tc_wait(&bar->a_empty[su], uph ^ 1u, limit_ns, abort_flag);
-      if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-      tc_fence_after();
-      const unsigned char* src = sWp + sw * WP_BYTES + r * 128;
-      uint32_t a[32];  // the row's 128 unpacked codes of this K block, 4 per register
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        // logical 16-byte chunk 2q+h of the packed row = K block q, words 4h .. 4h+3
-        const uint4 p = *reinterpret_cast<const uint4*>(src + (((2 * q + h) ^ rs) << 4));
-        const uint32_t words[4] = {p.x, p.y, p.z, p.w};
-#pragma unroll
-        for (int mq = 0; mq < 4; ++mq) {
-          const uint32_t w = words[mq];
-          const int c = 16 * h + 4 * mq;  // first column of this 16-trit group
-          a[c + 0] = w & 0x03030303u;
-          a[c + 1] = (w >> 2) & 0x03030303u;
-          a[c + 2] = (w >> 4) & 0x03030303u;
-          a[c + 3] = (w >> 6) & 0x03030303u;
+      if (lane == 0) {
+        if (q0 == 0) got = tc_wait(&bar->w_full[sw], wph, limit_ns, abort_flag);
+        if (g >= SU) {  // A slot su is free once group g - SU has been consumed
+          const int i = g - SU;
+          got = got && tc_wait(&bar->done[i & (SD - 1)], static_cast<uint32_t>((i / SD) & 1),
+                               limit_ns, abort_flag);
         }
       }
-      tmem_st_x32(tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + a_col0 +
-                      static_cast<uint32_t>(su * A_COLS),
-                  a);
-      tmem_st_wait();
-      tc_fence_before();
+      got = __shfl_sync(0xffffffffu, got, 0);
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bar->a_full[su]);
-      if (++su == SU) { su = 0; uph ^= 1u; }
-      if (q == KPS - 1 || kb == kb1 - 1) {  // done with this packed super-tile
-        if (lane == 0) mbar_arrive(&bar->w_empty[sw]);
-        if (++sw == pl.sw) { sw = 0; wph ^= 1u; }
+      if (got) {
+        tc_fence_after();
+        const unsigned char* src = sWp + sw * WP_BYTES + r * 128;
+#pragma unroll
+        for (int kq = 0; kq < KG; ++kq) {
+          const int q = q0 + kq;
+          uint32_t a[32];  // the row's 128 unpacked codes of K block q, 4 per register
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            // logical 16-byte chunk 2q+h of the packed row = K block q, words 4h .. 4h+3
+            const uint4 p = *reinterpret_cast<const uint4*>(src + (((2 * q + h) ^ rs) << 4));
+            const uint32_t words[4] = {p.x, p.y, p.z, p.w};
+#pragma unroll
+            for (int mq = 0; mq < 4; ++mq) {
+              const uint32_t w = words[mq];
+              const int c = 16 * h + 4 * mq;  // first column of this 16-trit group
+              a[c + 0] = w & 0x03030303u;
+              a[c + 1] = (w >> 2) & 0x03030303u;
+              a[c + 2] = (w >> 4) & 0x03030303u;
+              a[c + 3] = (w >> 6) & 0x03030303u;
+            }
+          }
+          tmem_st_x32(a_lane + static_cast<uint32_t>(su * G_COLS + kq * A_COLS), a);
+        }
+        tmem_st_wait();
+      }
+      tc_fence_before();
+      // all 128 rows of group g are in TMEM, unless some warp failed (a uniform decision)
+      if (epi_bar_or(!got || *abort_flag != 0)) break;
+      const bool last_of_tile = (q0 + KG == KPS) || (g == ng - 1);
+      if (warp == 0) {
+        bool xok = true;
+        if (lane == 0) {
+          xok = tc_wait(&bar->x_full[sx], xph, limit_ns, abort_flag);
+          if (last_of_tile) mbar_arrive(&bar->w_empty[sw]);  // all rows read this super-tile
+        }
+        xok = __shfl_sync(0xffffffffu, xok, 0);
+        __syncwarp();
+        if (xok) {
+          tc_fence_after();
+          const uint32_t a_tmem = a_tmem0 + static_cast<uint32_t>(su * G_COLS);
+          const uint64_t b_desc = x_desc0 + static_cast<uint64_t>(sx * (XG >> 4));
+#pragma unroll
+          for (int kq = 0; kq < KG; ++kq)
+#pragma unroll
+            for (int kk = 0; kk < BK / MMA_K; ++kk)
+              mma_i8_ts_elect(tmem_base,
+                              a_tmem + static_cast<uint32_t>(kq * A_COLS + kk * (MMA_K / 4)),
+                              b_desc + static_cast<uint64_t>(kq * (XB >> 4) + kk * (MMA_K >> 4)),
+                              idesc, (g | kq | kk) != 0 ? 1u : 0u);
+          mma_commit_elect(&bar->done[g & (SD - 1)]);
+        }
+      }
+      if (++su == SU) su = 0;
+      if (++sx == pl.sx) { sx = 0; xph ^= 1u; }
+      if (last_of_tile && ++sw == pl.sw) { sw = 0; wph ^= 1u; }
+    }
+    const bool ok = (g == ng);
+    if (warp == 0) {
+      if (ok) {
+        mma_commit_elect(&bar->acc_full);
+      } else if (g > 0) {
+        mma_commit_elect(&bar->drain);  // completes once every MMA issued above has finished
+        if (lane == 0) mbar_wait(&bar->drain, 0u, 100000000ull);
+        __syncwarp();
       }
     }
     // ---------------------------------------------------------------- epilogue
     const bool got = ok && tc_wait(&bar->acc_full, 0u, limit_ns, abort_flag);
-    if (__all_sync(0xffffffffu, got)) {
+    if (!epi_bar_or(!got)) {  // the same decision in all four warps
       tc_fence_after();
       const int n = n0 + warp * 32 + lane;  // this thread's TMEM lane = weight row
       const bool nvalid = n < N;
@@ -349,7 +408,7 @@ __global__ void __launch_bounds__(sk::THREADS, 1) gemm_skinny_kernel(
       if (splits == 1) {
         for (int c0 = 0; c0 < bnt; c0 += 16) {
           uint32_t v[16];
-          ld_acc_sum(taddr + c0, nacc, acol, v);
+          ld_acc16(taddr + c0, v);
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int t = c0 + j;
@@ -363,7 +422,7 @@ __global__ void __launch_bounds__(sk::THREADS, 1) gemm_skinny_kernel(
         // exact int32 partial of this split, added into acc32[t][n] (zeroed by the host)
         for (int c0 = 0; c0 < bnt; c0 += 16) {
           uint32_t v[16];
-          ld_acc_sum(taddr + c0, nacc, acol, v);
+          ld_acc16(taddr + c0, v);
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int t = c0 + j;
@@ -400,7 +459,7 @@ __global__ void __launch_bounds__(sk::THREADS, 1) gemm_skinny_kernel(
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 0) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem_base, ncols);
