@@ -21,15 +21,17 @@
 // adds, so the split does not change a single bit.
 //
 // The loop moves in groups of KG = 2 K blocks. Per group the four unpack warps write
-// their rows' codes to TMEM, meet at a named barrier (bar.sync of 128 threads, far cheaper
-// than an mbarrier arrive/poll round trip), and warp 0 then issues the group's 8 MMAs and
-// one commit; its barrier (done ring) frees the A slot and the token tile. At small M
-// each MMA is a few tens of cycles of tensor work, so the kernel's pace is set by these
-// per-group synchronisation hops, not by bandwidth.
+// their rows' codes to TMEM and meet the MMA warp at a hardware named barrier (bar.red of
+// 160 threads, far cheaper than an mbarrier arrive/poll round trip; the reduction also
+// makes every abort decision uniform, so no participant can be left waiting). The MMA
+// warp then issues the group's 8 MMAs and one commit while the unpack warps go on to the
+// next group; the commit's barrier (done ring) frees the A slot and the token tile. At
+// small M each MMA is a few tens of cycles of tensor work, so these per-group handoffs,
+// not bandwidth, set the pace.
 //
-// 5 warps: warps 0-3 unpack (thread t owns weight row t, TMEM lane t), warp 0 also issues
-// the MMAs (whole-warp loop, one elected lane issues, operands precomputed) and owns the
-// TMEM allocation; the four run the epilogue at the end. Warp 4 issues the TMA loads.
+// 6 warps: warps 0-3 unpack (thread t owns weight row t, TMEM lane t) and run the
+// epilogue at the end; warp 4 issues the TMA loads; warp 5 owns the TMEM allocation and
+// issues the MMAs (whole-warp loop, one elected lane issues, operands precomputed).
 #pragma once
 
 #include "common.cuh"
@@ -47,14 +49,9 @@ constexpr int WP_BYTES = BW * BK * KPS / 4;  // 16 KB packed super-tile
 constexpr int A_COLS = BK / 4;               // TMEM columns of one unpacked K block
 constexpr int G_COLS = KG * A_COLS;          // TMEM columns of one unpacked group
 constexpr int MAX_SU = 8;                    // unpacked groups in flight (TMEM slots), at most
-constexpr int THREADS = 160;
+constexpr int THREADS = 192;
 constexpr int MAX_SW = 4, MAX_SX = 16;
-#ifndef SK_PREFETCH
-#define SK_PREFETCH 8
-#endif
-// W super-tiles prefetched into L2 ahead of the one being loaded: HBM latency under load
-// needs far more bytes in flight than the shared-memory ring holds.
-constexpr int PF = SK_PREFETCH;
+
 static_assert(KPS % KG == 0, "groups tile a super-tile");
 // Ring of per-group completion barriers. Group g's MMAs arrive on done[g % SD]; the
 // unpackers wait for group g - SU before reusing A slot g % SU, the producer for group
@@ -167,20 +164,24 @@ __device__ __forceinline__ void red_add_s32(int* p, int v) {
 __device__ __forceinline__ void epi_bar_sync() {  // the 4 unpack/epilogue warps only
   asm volatile("bar.sync 1, 128;" ::: "memory");
 }
-// Named barrier of the 4 unpack/epilogue warps that also returns the OR of every thread's
-// flag, so that all 128 threads take the same branch afterwards.
-__device__ __forceinline__ bool epi_bar_or(bool v) {
+// Named barriers that also return the OR of every participant's flag, so that all of them
+// take the same branch afterwards: id 1 = the 4 unpack/epilogue warps, id 2 = those and
+// the MMA warp (the per-group handoff).
+template <int ID, int COUNT>
+__device__ __forceinline__ bool bar_or(bool v) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, 1, 128, p;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
-      : "r"(static_cast<uint32_t>(v))
+      : "r"(static_cast<uint32_t>(v)), "n"(ID), "n"(COUNT)
       : "memory");
   return r != 0;
 }
+__device__ __forceinline__ bool epi_bar_or(bool v) { return bar_or<1, 128>(v); }
+__device__ __forceinline__ bool group_bar_or(bool v) { return bar_or<2, 160>(v); }
 
 // Rescales one accumulator and stores it. OM: 0 fp32, 1 bf16, 2 int32 (acc only).
 template <int OM>
@@ -243,7 +244,7 @@ __global__ void __launch_bounds__(sk::THREADS, 1) gemm_skinny_kernel(
     bar->last = 0;
     fence_mbar_init();
   }
-  if (warp == 0) {
+  if (warp == 5) {
     tmem_alloc(&bar->tmem_base, ncols);
     tmem_relinquish();
   }
@@ -261,14 +262,9 @@ __global__ void __launch_bounds__(sk::THREADS, 1) gemm_skinny_kernel(
       uint32_t wph = 0;
       long long w_issued = 0, x_issued = 0;
       bool ok = true;
-      const int nst = (kb1 - kb0 + KPS - 1) / KPS;  // super-tiles of this CTA
-      for (int i = 0; i < PF && i < nst; ++i)
-        tma_prefetch_l2_2d(&map_w, (kb0 + i * KPS) * (BK / 4), n0);
       for (int g = 0; g < ng; ++g) {
         const int kb = kb0 + g * KG;
         if (((g * KG) & (KPS - 1)) == 0) {
-          const int st = (g * KG) / KPS;
-          if (st + PF < nst) tma_prefetch_l2_2d(&map_w, (kb0 + (st + PF) * KPS) * (BK / 4), n0);
           if (!tc_wait(&bar->w_empty[sw], wph ^ 1u, limit_ns, abort_flag)) { ok = false; break; }
           mbar_arrive_expect_tx(&bar->w_full[sw], WP_BYTES);
           tma_load_2d(sWp + sw * WP_BYTES, &map_w, kb * (BK / 4), n0, &bar->w_full[sw]);
@@ -302,23 +298,68 @@ __global__ void __launch_bounds__(sk::THREADS, 1) gemm_skinny_kernel(
                     100000000ull);
       }
     }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------------ MMA issuer
+    const uint32_t idesc = idesc_i8(BW, bnt);
+    // built once; a stage or K step only moves the 14-bit start-address field
+    const uint64_t x_desc0 = smem_desc_k128(smem_u32(sX));
+    const uint32_t a_tmem0 = tmem_base + a_col0;
+    int su = 0, sx = 0, sw = 0;
+    uint32_t xph = 0;
+    bool failed = false;  // a token-tile wait gave up (the abort flag is set)
+    int g = 0;
+    for (; g < ng; ++g) {
+      if (group_bar_or(*abort_flag != 0)) break;  // group g's rows are in TMEM
+      const int q0 = (g * KG) & (KPS - 1);
+      const bool last_of_tile = (q0 + KG == KPS) || (g == ng - 1);
+      bool xok = true;
+      if (lane == 0) {
+        xok = tc_wait(&bar->x_full[sx], xph, limit_ns, abort_flag);
+        if (last_of_tile) mbar_arrive(&bar->w_empty[sw]);  // every row has read this super-tile
+      }
+      xok = __shfl_sync(0xffffffffu, xok, 0);
+      __syncwarp();
+      if (xok) {
+        tc_fence_after();
+        const uint32_t a_tmem = a_tmem0 + static_cast<uint32_t>(su * G_COLS);
+        const uint64_t b_desc = x_desc0 + static_cast<uint64_t>(sx * (XG >> 4));
+#pragma unroll
+        for (int kq = 0; kq < KG; ++kq)
+#pragma unroll
+          for (int kk = 0; kk < BK / MMA_K; ++kk)
+            mma_i8_ts_elect(tmem_base,
+                            a_tmem + static_cast<uint32_t>(kq * A_COLS + kk * (MMA_K / 4)),
+                            b_desc + static_cast<uint64_t>(kq * (XB >> 4) + kk * (MMA_K >> 4)),
+                            idesc, (g | kq | kk) != 0 ? 1u : 0u);
+        mma_commit_elect(&bar->done[g & (SD - 1)]);
+      } else {
+        // stay in step with the unpack warps: the next handoff sees the abort flag and
+        // every participant leaves the loop there
+        failed = true;
+      }
+      if (++su == SU) su = 0;
+      if (++sx == pl.sx) { sx = 0; xph ^= 1u; }
+      if (last_of_tile && ++sw == pl.sw) sw = 0;
+    }
+    if (g == ng && !failed) {
+      mma_commit_elect(&bar->acc_full);
+    } else if (g > 0) {
+      mma_commit_elect(&bar->drain);  // completes once every MMA issued above has finished
+      if (lane == 0) mbar_wait(&bar->drain, 0u, 100000000ull);
+      __syncwarp();
+    }
   } else {
     // ------------------------------------------------------------------ warps 0-3
     const int r = threadIdx.x;  // weight row of the tile owned by this thread (0..127)
     const int rs = r & 7;       // its 128-byte swizzle phase
     const uint32_t a_lane = tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + a_col0;
-    // MMA operands (used by warp 0): built once; a stage or K step only moves the
-    // descriptor's 14-bit start-address field or the TMEM column
-    const uint32_t idesc = idesc_i8(BW, bnt);
-    const uint64_t x_desc0 = smem_desc_k128(smem_u32(sX));
-    const uint32_t a_tmem0 = tmem_base + a_col0;
-    int sw = 0, su = 0, sx = 0;
-    uint32_t wph = 0, xph = 0;
+    int sw = 0, su = 0;
+    uint32_t wph = 0;
     int g = 0;
     for (; g < ng; ++g) {
       const int q0 = (g * KG) & (KPS - 1);  // first K block of the group in its super-tile
       // lane 0 waits for the warp; __syncwarp then orders the other lanes after it. A warp
-      // whose wait fails skips its work but still meets the others at the named barrier.
+      // whose wait fails skips its work but still meets the others at the handoff.
       bool got = true;
       if (lane == 0) {
         if (q0 == 0) got = tc_wait(&bar->w_full[sw], wph, limit_ns, abort_flag);
@@ -357,46 +398,12 @@ __global__ void __launch_bounds__(sk::THREADS, 1) gemm_skinny_kernel(
         tmem_st_wait();
       }
       tc_fence_before();
-      // all 128 rows of group g are in TMEM, unless some warp failed (a uniform decision)
-      if (epi_bar_or(!got || *abort_flag != 0)) break;
+      if (group_bar_or(!got || *abort_flag != 0)) break;  // hand group g to the MMA warp
       const bool last_of_tile = (q0 + KG == KPS) || (g == ng - 1);
-      if (warp == 0) {
-        bool xok = true;
-        if (lane == 0) {
-          xok = tc_wait(&bar->x_full[sx], xph, limit_ns, abort_flag);
-          if (last_of_tile) mbar_arrive(&bar->w_empty[sw]);  // all rows read this super-tile
-        }
-        xok = __shfl_sync(0xffffffffu, xok, 0);
-        __syncwarp();
-        if (xok) {
-          tc_fence_after();
-          const uint32_t a_tmem = a_tmem0 + static_cast<uint32_t>(su * G_COLS);
-          const uint64_t b_desc = x_desc0 + static_cast<uint64_t>(sx * (XG >> 4));
-#pragma unroll
-          for (int kq = 0; kq < KG; ++kq)
-#pragma unroll
-            for (int kk = 0; kk < BK / MMA_K; ++kk)
-              mma_i8_ts_elect(tmem_base,
-                              a_tmem + static_cast<uint32_t>(kq * A_COLS + kk * (MMA_K / 4)),
-                              b_desc + static_cast<uint64_t>(kq * (XB >> 4) + kk * (MMA_K >> 4)),
-                              idesc, (g | kq | kk) != 0 ? 1u : 0u);
-          mma_commit_elect(&bar->done[g & (SD - 1)]);
-        }
-      }
       if (++su == SU) su = 0;
-      if (++sx == pl.sx) { sx = 0; xph ^= 1u; }
       if (last_of_tile && ++sw == pl.sw) { sw = 0; wph ^= 1u; }
     }
     const bool ok = (g == ng);
-    if (warp == 0) {
-      if (ok) {
-        mma_commit_elect(&bar->acc_full);
-      } else if (g > 0) {
-        mma_commit_elect(&bar->drain);  // completes once every MMA issued above has finished
-        if (lane == 0) mbar_wait(&bar->drain, 0u, 100000000ull);
-        __syncwarp();
-      }
-    }
     // ---------------------------------------------------------------- epilogue
     const bool got = ok && tc_wait(&bar->acc_full, 0u, limit_ns, abort_flag);
     if (!epi_bar_or(!got)) {  // the same decision in all four warps
@@ -459,7 +466,7 @@ __global__ void __launch_bounds__(sk::THREADS, 1) gemm_skinny_kernel(
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 5) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem_base, ncols);

@@ -12,9 +12,8 @@
 //                 weight tile [256 rows x 32 bytes] into a STAGES-deep ring
 //   warps 2,3,8,9 unpack: 2-bit codes -> one int8 per trit (shift + mask), written in the
 //                 128-byte swizzled K-major layout the MMA reads, USTAGES-deep ring
-//   warp 1        allocates 512 TMEM columns and issues 4 MMAs (K = 32 each) per stage
-//                 into a double-buffered 128 x 256 int32 accumulator (whole-warp loop,
-//                 one elected lane issues)
+//   warp 1        allocates 512 TMEM columns; one lane issues 4 MMAs (K = 32 each) per
+//                 stage into a double-buffered 128 x 256 int32 accumulator
 //   warps 4..7    epilogue: tcgen05.ld of their 32 TMEM lanes, subtract rowsum, rescale,
 //                 store, while the MMA fills the other accumulator buffer
 // Every mbarrier wait is bounded; on a timeout the kernel records BL_ERR_TIMEOUT, waits
@@ -63,12 +62,8 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, uint64_t
   const uint64_t t0 = global_ns();
   while (true) {
 #pragma unroll 1
-    for (int i = 0; i < 32; ++i) {
+    for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(bar, parity)) return true;
-#ifdef TC_WAIT_BACKOFF_NS
-      __nanosleep(TC_WAIT_BACKOFF_NS);
-#endif
-    }
     if (*abort) return false;
     if (global_ns() - t0 > limit_ns) {
       record_status(kStatusTimeout);
@@ -160,53 +155,44 @@ __global__ void __launch_bounds__(tc::THREADS, 1) gemm_tc_kernel(
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
-    // The whole warp runs this loop (operands stay warp-uniform); lane 0 polls the
-    // barriers and one elected lane issues each tcgen05 instruction. Descriptors are built
-    // once; a stage or K step only moves the 14-bit start-address field (16-byte units).
-    const uint64_t a_desc0 = smem_desc_k128(smem_u32(sA));
-    const uint64_t b_desc0 = smem_desc_k128(smem_u32(sBu));
-    int s = 0, u = 0, ab = 0;
-    uint32_t ph = 0, uph = 0, aph = 0;
-    bool ok = true, issued_any = false;
-    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-      bool got = true;
-      if (lane == 0) got = tc_wait(&bar->tmem_empty[ab], aph ^ 1u, limit_ns, abort_flag);
-      got = __shfl_sync(0xffffffffu, got, 0);
-      __syncwarp();
-      if (!got) { ok = false; break; }
-      tc_fence_after();
-      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(ab * BN);
-      for (int kb = 0; kb < KB; ++kb) {
-        got = true;
-        if (lane == 0)
-          got = tc_wait(&bar->full_unp[u], uph, limit_ns, abort_flag) &&
-                tc_wait(&bar->full_tma[s], ph, limit_ns, abort_flag);
-        got = __shfl_sync(0xffffffffu, got, 0);
-        __syncwarp();
-        if (!got) { ok = false; break; }
+    if (lane == 0) {
+      // Descriptors are built once; a stage or K step only moves the 14-bit start-address
+      // field (16-byte units), which keeps the single issuing thread's work per MMA tiny.
+      const uint64_t a_desc0 = smem_desc_k128(smem_u32(sA));
+      const uint64_t b_desc0 = smem_desc_k128(smem_u32(sBu));
+      int s = 0, u = 0, ab = 0;
+      uint32_t ph = 0, uph = 0, aph = 0;
+      bool ok = true, issued_any = false;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        if (!tc_wait(&bar->tmem_empty[ab], aph ^ 1u, limit_ns, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        const uint64_t a_desc = a_desc0 + static_cast<uint64_t>(s * (A_BYTES >> 4));
-        const uint64_t b_desc = b_desc0 + static_cast<uint64_t>(u * (BU_BYTES >> 4));
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(ab * BN);
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!tc_wait(&bar->full_unp[u], uph, limit_ns, abort_flag) ||
+              !tc_wait(&bar->full_tma[s], ph, limit_ns, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t a_desc = a_desc0 + static_cast<uint64_t>(s * (A_BYTES >> 4));
+          const uint64_t b_desc = b_desc0 + static_cast<uint64_t>(u * (BU_BYTES >> 4));
 #pragma unroll
-        for (int kk = 0; kk < BK / MMA_K; ++kk) {
-          mma_i8_elect(d_tmem, a_desc + static_cast<uint64_t>(kk * (MMA_K >> 4)),
-                       b_desc + static_cast<uint64_t>(kk * (MMA_K >> 4)), IDESC,
-                       (kb | kk) != 0 ? 1u : 0u);
+          for (int kk = 0; kk < BK / MMA_K; ++kk) {
+            mma_i8(d_tmem, a_desc + static_cast<uint64_t>(kk * (MMA_K >> 4)),
+                   b_desc + static_cast<uint64_t>(kk * (MMA_K >> 4)), IDESC,
+                   (kb | kk) != 0 ? 1u : 0u);
+          }
+          issued_any = true;
+          mma_commit(&bar->empty_tma[s]);
+          mma_commit(&bar->empty_unp[u]);
+          if (++s == STAGES) { s = 0; ph ^= 1u; }
+          if (++u == USTAGES) { u = 0; uph ^= 1u; }
         }
-        issued_any = true;
-        mma_commit_elect(&bar->empty_tma[s]);
-        mma_commit_elect(&bar->empty_unp[u]);
-        if (++s == STAGES) { s = 0; ph ^= 1u; }
-        if (++u == USTAGES) { u = 0; uph ^= 1u; }
+        if (!ok) break;
+        mma_commit(&bar->tmem_full[ab]);
+        if (++ab == 2) { ab = 0; aph ^= 1u; }
       }
-      if (!ok) break;
-      mma_commit_elect(&bar->tmem_full[ab]);
-      if (++ab == 2) { ab = 0; aph ^= 1u; }
-    }
-    if (!ok && issued_any) {
-      mma_commit_elect(&bar->drain);  // completes once every MMA issued above has finished
-      if (lane == 0) mbar_wait(&bar->drain, 0u, 100000000ull);
-      __syncwarp();
+      if (!ok && issued_any) {
+        mma_commit(&bar->drain);  // completes once every MMA issued above has finished
+        mbar_wait(&bar->drain, 0u, 100000000ull);
+      }
     }
   } else if (warp >= 4 && warp < 8) {
     // ------------------------------------------------------------------ epilogue
