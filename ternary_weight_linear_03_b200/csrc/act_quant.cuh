@@ -64,13 +64,25 @@ __device__ __forceinline__ float abs_bits(float x) {
   return __uint_as_float(__float_as_uint(x) & 0x7fffffffu);
 }
 
-// grid = M blocks, K % 8 == 0. rowsum may be null.
+// Zeroes n16 16-byte words at z with the whole grid (the split-K sums and counters of the
+// tensor-core kernel that follows, so that no separate memset sits between the two).
+__device__ __forceinline__ void grid_zero(uint4* __restrict__ z, long long n16) {
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n16;
+       i += static_cast<long long>(gridDim.x) * blockDim.x)
+    z[i] = make_uint4(0u, 0u, 0u, 0u);
+}
+
+// grid = M blocks, K % 8 == 0. rowsum may be null; zero/zero_n16 name an extra region to
+// clear (may be null/0). Lets the dependent kernel launch at once (it waits for this
+// grid's completion before reading any of these outputs).
 template <bool kBf16>
 __global__ void __launch_bounds__(kAqThreads) act_quant_kernel(
     const void* __restrict__ x, int K, int8_t* __restrict__ xq, float* __restrict__ scale,
-    int* __restrict__ rowsum) {
+    int* __restrict__ rowsum, uint4* __restrict__ zero, long long zero_n16) {
   __shared__ float redf[32];
   __shared__ int redi[32];
+  allow_dependent_launch();
+  grid_zero(zero, zero_n16);
   const int t = blockIdx.x;
   const char* row = static_cast<const char*>(x) + static_cast<size_t>(t) * K * (kBf16 ? 2 : 4);
   const int nc = K / 8;
@@ -112,9 +124,14 @@ __global__ void __launch_bounds__(kAqThreads) act_quant_kernel(
 }
 
 // rowsum_t = sum_k xq[t,k] for int8 input given directly (the integer test hook).
+// zero/zero_n16 as for act_quant_kernel.
 __global__ void __launch_bounds__(kAqThreads) rowsum_i8_kernel(const int8_t* __restrict__ xq,
-                                                              int K, int* __restrict__ rowsum) {
+                                                              int K, int* __restrict__ rowsum,
+                                                              uint4* __restrict__ zero,
+                                                              long long zero_n16) {
   __shared__ int redi[32];
+  allow_dependent_launch();
+  grid_zero(zero, zero_n16);
   const int t = blockIdx.x;
   const int4* row = reinterpret_cast<const int4*>(xq + static_cast<size_t>(t) * K);
   int sum = 0;

@@ -267,16 +267,35 @@ bl_status launch_skinny_t(const int8_t* xq, const uint8_t* packed, const int* ro
       return BL_ERR_CUDA;
     configured = true;
   }
-  if (p.splits > 1 &&
-      cudaMemsetAsync(w.partial, 0,
-                      reinterpret_cast<char*>(w.counters + p.tiles) -
-                          reinterpret_cast<char*>(w.partial),
-                      s) != cudaSuccess)
+  // Programmatic dependent launch: the kernel may start while the quantization kernel before
+  // it (which also zeroed the split-K sums and counters) is still running; it loads W and
+  // sets up TMEM meanwhile and waits for that grid before touching its outputs.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(p.tiles * p.splits));
+  cfg.blockDim = dim3(bl::sk::THREADS);
+  cfg.dynamicSmemBytes = static_cast<size_t>(bl::sk::smem_bytes(p.bnt));
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, map_x, map_w, rowsum, scale, gamma, y, w.partial,
+                         w.counters, M, N, K, p.bnt, p.splits, p.kbps, kWaitLimitNs) !=
+      cudaSuccess)
     return BL_ERR_CUDA;
-  kern<<<p.tiles * p.splits, bl::sk::THREADS, bl::sk::smem_bytes(p.bnt), s>>>(
-      map_x, map_w, rowsum, scale, gamma, y, w.partial, w.counters, M, N, K, p.bnt, p.splits,
-      p.kbps, kWaitLimitNs);
   return launch_status();
+}
+
+// The part of the workspace the skinny kernel needs zeroed (split-K sums and counters; a
+// multiple of 256 bytes), empty when K is not split. The kernel launched just before the
+// skinny one clears it.
+void skinny_zero_region(void* ws, int M, int N, int K, uint4** z, long long* n16) {
+  const SkinnyPlan p = skinny_plan(M, N, K);
+  const SkinnyWs w = skinny_ws_layout(ws, M, N, K, p);
+  const size_t head = fwd_ws_layout(nullptr, M, K).bytes;
+  *z = (p.splits > 1) ? reinterpret_cast<uint4*>(w.partial) : nullptr;
+  *n16 = (p.splits > 1) ? static_cast<long long>((w.bytes - head) / 16) : 0;
 }
 
 bl_status launch_skinny(const int8_t* xq, const uint8_t* packed, const int* rowsum,
@@ -300,16 +319,19 @@ size_t fwd_ws_bytes(int M, int N, int K) {
 }
 
 bl_status launch_act_quant(const void* x, int x_dtype, int M, int K, int8_t* xq, float* scale,
-                           int* rowsum, cudaStream_t s) {
+                           int* rowsum, cudaStream_t s, uint4* zero = nullptr,
+                           long long zero_n16 = 0) {
   if (x_dtype == BL_BF16)
-    bl::act_quant_kernel<true><<<M, bl::kAqThreads, 0, s>>>(x, K, xq, scale, rowsum);
+    bl::act_quant_kernel<true><<<M, bl::kAqThreads, 0, s>>>(x, K, xq, scale, rowsum, zero,
+                                                            zero_n16);
   else
-    bl::act_quant_kernel<false><<<M, bl::kAqThreads, 0, s>>>(x, K, xq, scale, rowsum);
+    bl::act_quant_kernel<false><<<M, bl::kAqThreads, 0, s>>>(x, K, xq, scale, rowsum, zero,
+                                                             zero_n16);
   return launch_status();
 }
 
 // ------------------------------------------------------------------ weight quantization
-// Workspace of bitlinear_quantize_weights: the exponent buckets and the barrier counter.
+// Workspace of bitlinear_quantize_weights: the exact-sum columns and the barrier counters.
 size_t wq_ws_bytes(long long) { return align_up(sizeof(WqWorkspace), 256); }
 
 template <bool kBf16>
@@ -446,7 +468,10 @@ bl_status bitlinear_forward(const void* x, int x_dtype, const uint8_t* packed,
   if (!aligned16(ws)) return BL_ERR_MISALIGNED;
   if (ws_bytes < fwd_ws_bytes(M, N, K)) return BL_ERR_WORKSPACE;
   FwdWs w = fwd_ws_layout(ws, M, K);
-  bl_status st = launch_act_quant(x, x_dtype, M, K, w.xq, w.scale, w.rowsum, s);
+  uint4* zero = nullptr;
+  long long zero_n16 = 0;
+  if (M <= kSkinnyMaxM) skinny_zero_region(ws, M, N, K, &zero, &zero_n16);
+  bl_status st = launch_act_quant(x, x_dtype, M, K, w.xq, w.scale, w.rowsum, s, zero, zero_n16);
   if (st != BL_OK) return st;
   if (M <= kSkinnyMaxM)
     return launch_skinny(w.xq, packed, w.rowsum, w.scale, gamma, y, y_dtype, M, N, K, ws, s);
@@ -464,7 +489,10 @@ bl_status bitlinear_contract_i32(const int8_t* xq, const uint8_t* packed, int32_
   if (!aligned16(ws)) return BL_ERR_MISALIGNED;
   if (ws_bytes < fwd_ws_bytes(M, N, K)) return BL_ERR_WORKSPACE;
   FwdWs w = fwd_ws_layout(ws, M, K);
-  bl::rowsum_i8_kernel<<<M, bl::kAqThreads, 0, s>>>(xq, K, w.rowsum);
+  uint4* zero = nullptr;
+  long long zero_n16 = 0;
+  if (M <= kSkinnyMaxM) skinny_zero_region(ws, M, N, K, &zero, &zero_n16);
+  bl::rowsum_i8_kernel<<<M, bl::kAqThreads, 0, s>>>(xq, K, w.rowsum, zero, zero_n16);
   if (launch_status() != BL_OK) return BL_ERR_CUDA;
   if (M <= kSkinnyMaxM)
     return launch_skinny(xq, packed, w.rowsum, nullptr, nullptr, acc, BL_I32, M, N, K, ws, s);

@@ -77,6 +77,19 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
 }
 
 // ---------------------------------------------------------------------------------------
+// Programmatic dependent launch. A kernel launched with programmatic stream serialization
+// may start while the kernel before it in the stream is still running; it must call
+// grid_dependency_wait() before touching anything that kernel writes. The earlier kernel
+// calls allow_dependent_launch() to let it start early. Without the launch attribute the
+// wait returns at once.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void allow_dependent_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------------------
 // TMA (no multicast anywhere in this library)
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1,
                                             uint64_t* bar) {

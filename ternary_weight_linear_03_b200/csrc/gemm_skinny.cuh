@@ -262,13 +262,25 @@ __global__ void __launch_bounds__(sk::THREADS, 1) gemm_skinny_kernel(
       uint32_t wph = 0;
       long long w_issued = 0, x_issued = 0;
       bool ok = true;
+      // The first W super-tiles fill the empty ring before the wait for the kernel that
+      // produced the token tiles (programmatic dependent launch): W does not depend on it.
+      const int nst = (kb1 - kb0 + KPS - 1) / KPS;
+      const int pre = min(pl.sw, nst);
+      for (int i = 0; i < pre; ++i) {
+        mbar_arrive_expect_tx(&bar->w_full[i], WP_BYTES);
+        tma_load_2d(sWp + i * WP_BYTES, &map_w, (kb0 + i * KPS) * (BK / 4), n0, &bar->w_full[i]);
+      }
+      w_issued = pre;
+      grid_dependency_wait();
       for (int g = 0; g < ng; ++g) {
         const int kb = kb0 + g * KG;
         if (((g * KG) & (KPS - 1)) == 0) {
-          if (!tc_wait(&bar->w_empty[sw], wph ^ 1u, limit_ns, abort_flag)) { ok = false; break; }
-          mbar_arrive_expect_tx(&bar->w_full[sw], WP_BYTES);
-          tma_load_2d(sWp + sw * WP_BYTES, &map_w, kb * (BK / 4), n0, &bar->w_full[sw]);
-          ++w_issued;
+          if ((g * KG) / KPS >= pre) {  // not one of the super-tiles issued above
+            if (!tc_wait(&bar->w_empty[sw], wph ^ 1u, limit_ns, abort_flag)) { ok = false; break; }
+            mbar_arrive_expect_tx(&bar->w_full[sw], WP_BYTES);
+            tma_load_2d(sWp + sw * WP_BYTES, &map_w, kb * (BK / 4), n0, &bar->w_full[sw]);
+            ++w_issued;
+          }
           if (++sw == pl.sw) { sw = 0; wph ^= 1u; }
         }
         if (g >= pl.sx) {  // token slot sx is free once group g - SX has been consumed
@@ -405,6 +417,7 @@ __global__ void __launch_bounds__(sk::THREADS, 1) gemm_skinny_kernel(
     }
     const bool ok = (g == ng);
     // ---------------------------------------------------------------- epilogue
+    grid_dependency_wait();  // rowsum, scale and the zeroed split-K sums come from it
     const bool got = ok && tc_wait(&bar->acc_full, 0u, limit_ns, abort_flag);
     if (!epi_bar_or(!got)) {  // the same decision in all four warps
       tc_fence_after();

@@ -2,8 +2,9 @@
 // takeaways bullet 1: weights constrained to {-1, 0, +1} by an absmean quantization
 // function; searcharxiv.com abstract page, Abstract: every weight is ternary).
 //
-// One cooperative kernel, two lean passes over W (the second is served from L2 whenever W
-// fits there). Every block owns a contiguous range of 16-weight words and streams it
+// One cooperative kernel, two lean passes over W. The second pass reads the stages still
+// held in shared memory when a block's whole range fits its ring, and is otherwise served
+// from L2 whenever W fits there. Every block owns a contiguous range of 16-weight words and streams it
 // through a ring of 16 KB bulk copies (cp.async.bulk into shared memory, 4 in flight per
 // block); thread t handles the 16-byte chunks t + 256 i of each stage.
 //   A  exact sum of |w| (below) into exponent buckets;
@@ -25,7 +26,11 @@
 // them to integers, sums those with shuffles and adds the result into 64-bit exponent
 // buckets (low 32 bits at exponent base, the rest at base + 32). Values outside the
 // window (subnormals, far larger or smaller ones) go straight into the buckets as
-// (exponent, 24-bit mantissa). The buckets are summed exactly, so gamma depends neither
+// (exponent, 24-bit mantissa). Each block then folds its buckets into the 14 column sums
+// of a 448-bit integer (bucket e adds B[e] << ((e - 1) % 32) at 32-bit limb (e - 1) / 32)
+// and adds the non-zero ones into one of kWqCopies copies in the workspace (spreading the
+// same-address atomics); after the grid barrier every block adds the copies, propagates
+// the carries and rounds once. All of it is integer arithmetic, so gamma depends neither
 // on the grid nor on the order of the atomic adds.
 #pragma once
 
@@ -39,12 +44,13 @@ constexpr int kWqThreads = 256;
 constexpr int kWqLimbs = 14;     // 32-bit limbs of the exact sum (S * 2^149 < 2^448)
 constexpr int kWqWindow = 21;    // exponents covered by the fp64 window
 constexpr int kWqFlushWords = 16;  // words a thread sums in fp64 between bucket flushes
+constexpr int kWqCopies = 8;       // copies of the column sums and arrival counters
 
-// The quantize_weights workspace (zeroed by the host before each launch).
+// The quantize_weights workspace (zeroed by the host before each launch). Block b adds
+// into copy b % kWqCopies.
 struct WqWorkspace {
-  unsigned long long buckets[kWqBuckets];
-  unsigned int arrived;  // grid-barrier arrivals
-  unsigned int pad[3];
+  unsigned long long cols[kWqCopies][kWqLimbs];  // column sums (below 2^39 per block)
+  unsigned int arrived[kWqCopies];               // grid-barrier arrivals
 };
 
 // |w| outside the fp64 window: added as (exponent, mantissa) into the shared buckets.
@@ -107,17 +113,16 @@ __device__ double wq_limbs_to_double(const uint32_t* L) {
 }
 
 // Smallest float t with fl(t / d) > 0.5, +inf when no finite t qualifies (d == 0 or inf).
+// For d > 0, correctly rounded division gives fl(t / d) > 0.5 exactly when t / d lies
+// above the midpoint 0.5 + 2^-25 between 0.5 and the next float (at the midpoint itself
+// the tie goes to the even 0.5), i.e. when t > m = d * (0.5 + 2^-25). m has at most
+// 24 + 26 significant bits, so the double product is exact, and t is the smallest float
+// strictly above m: m rounded up, stepped once more if m is itself a float.
 __device__ float wq_threshold(float d) {
   if (!(d > 0.0f) || isinf(d)) return __int_as_float(0x7f800000);
-  float t = __fmul_rn(0.5f, d);
-  for (int i = 0; i < 64 && t > 0.0f; ++i) {  // step down while the predecessor qualifies
-    const float prev = __int_as_float(__float_as_int(t) - 1);
-    if (__fdiv_rn(prev, d) > 0.5f) t = prev; else break;
-  }
-  for (int i = 0; i < 64; ++i) {  // step up until t qualifies
-    if (__fdiv_rn(t, d) > 0.5f) break;
-    t = __int_as_float(__float_as_int(t) + 1);
-  }
+  const double m = __dmul_rn(static_cast<double>(d), 0.5 + 0x1p-25);
+  float t = __double2float_ru(m);
+  if (static_cast<double>(t) == m) t = __int_as_float(__float_as_int(t) + 1);  // m > 0
   return t;
 }
 
@@ -296,19 +301,39 @@ __global__ void __launch_bounds__(kWqThreads) weight_quant_kernel(
   wq_flush(acc0, acc1, base, sb);
   if (nonfinite) record_status(kStatusNonfinite);
   __syncthreads();
-  for (int i = tid; i < kWqBuckets; i += blockDim.x)
-    if (sb[i]) atomicAdd(&ws->buckets[i], sb[i]);
-  // pass B starts streaming now; its stages do not depend on gamma
-  if (tid == 0)
-    for (int st = 0; st < min(ring.nst, kWqStages); ++st) wq_issue(ring, st, ring.nst + st);
+  // Column sums of this block: bucket e contributes B[e] << ((e-1) % 32) to limbs
+  // (e-1)/32 .. +2, each part below 2^32, so a column of one block stays below 2^39.
+  for (int e = 1 + tid; e < kWqBuckets; e += blockDim.x) {
+    const unsigned long long b = sb[e];
+    if (b == 0ull) continue;
+    const int pos = e - 1, wd = pos >> 5, sh = pos & 31;
+    const uint32_t lo = static_cast<uint32_t>(b), hi = static_cast<uint32_t>(b >> 32);
+    atomicAdd(&col[wd], static_cast<unsigned long long>(lo << sh));
+    atomicAdd(&col[wd + 1], static_cast<unsigned long long>(__funnelshift_l(lo, hi, sh)));
+    const uint32_t p2 = __funnelshift_l(hi, 0u, sh);
+    if (p2) atomicAdd(&col[wd + 2], static_cast<unsigned long long>(p2));
+  }
+  __syncthreads();
+  const int copy = static_cast<int>(blockIdx.x % kWqCopies);
+  if (tid < kWqLimbs && col[tid] != 0ull) atomicAdd(&ws->cols[copy][tid], col[tid]);
+  // When the block's whole range fits the ring, pass A left every stage in its slot
+  // (stage st in slot st) and pass B reads them there; otherwise pass B streams the range
+  // again, starting now (its stages do not depend on gamma).
+  const bool resident = ring.nst <= kWqStages;
+  if (tid == 0 && !resident)
+    for (int st = 0; st < kWqStages; ++st) wq_issue(ring, st, ring.nst + st);
 
   // ---------------------------------------------------------------- grid barrier
-  __threadfence();
-  __syncthreads();
+  __syncthreads();  // this block's column adds are issued; thread 0 fences for all
   if (tid == 0) {
-    atomicAdd(&ws->arrived, 1u);
+    __threadfence();
+    atomicAdd(&ws->arrived[copy], 1u);
     const uint64_t t0 = global_ns();
-    while (ld_acquire_u32(&ws->arrived) < gridDim.x) {
+    while (true) {
+      unsigned int total = 0u;
+#pragma unroll
+      for (int c = 0; c < kWqCopies; ++c) total += ld_acquire_u32(&ws->arrived[c]);
+      if (total >= gridDim.x) break;
       if (global_ns() - t0 > limit_ns) {
         record_status(kStatusTimeout);
         s_ok = 0;
@@ -320,16 +345,11 @@ __global__ void __launch_bounds__(kWqThreads) weight_quant_kernel(
   __syncthreads();
 
   // ---------------------------------------------------------------- gamma and T
-  // Column sums: bucket e contributes B[e] << ((e-1) % 32) to limbs (e-1)/32 .. +2.
-  for (int e = 1 + tid; e < kWqBuckets; e += blockDim.x) {
-    const unsigned long long b = __ldcg(&ws->buckets[e]);
-    if (b == 0ull) continue;
-    const int pos = e - 1, wd = pos >> 5, sh = pos & 31;
-    const uint32_t lo = static_cast<uint32_t>(b), hi = static_cast<uint32_t>(b >> 32);
-    atomicAdd(&col[wd], static_cast<unsigned long long>(lo << sh));
-    atomicAdd(&col[wd + 1], static_cast<unsigned long long>(__funnelshift_l(lo, hi, sh)));
-    const uint32_t p2 = __funnelshift_l(hi, 0u, sh);
-    if (p2) atomicAdd(&col[wd + 2], static_cast<unsigned long long>(p2));
+  if (tid < kWqLimbs) {
+    unsigned long long t = 0ull;  // below 2^39 times the grid size: far from 2^64
+#pragma unroll
+    for (int c = 0; c < kWqCopies; ++c) t += __ldcg(&ws->cols[c][tid]);
+    col[tid] = t;
   }
   __syncthreads();
   if (tid == 0) {
@@ -337,7 +357,7 @@ __global__ void __launch_bounds__(kWqThreads) weight_quant_kernel(
     unsigned long long carry = 0ull;
 #pragma unroll
     for (int j = 0; j < kWqLimbs; ++j) {
-      const unsigned long long t = col[j] + carry;
+      const unsigned long long t = col[j] + carry;  // no overflow (see above)
       L[j] = static_cast<uint32_t>(t);
       carry = t >> 32;
     }
@@ -356,8 +376,9 @@ __global__ void __launch_bounds__(kWqThreads) weight_quant_kernel(
   for (int e = 0; e < E; ++e) mul[e] = 1u << wq_shift(wq_k<kBf16>(part, e));
   for (int st = 0; st < ring.nst; ++st) {
     const int g = ring.nst + st;  // stages consumed by this block so far
-    const int slot = g % kWqStages;
-    if (!mbar_wait(&full[slot], static_cast<uint32_t>((g / kWqStages) & 1), limit_ns)) s_ok = 0;
+    const int slot = resident ? st : g % kWqStages;
+    if (!resident && !mbar_wait(&full[slot], static_cast<uint32_t>((g / kWqStages) & 1), limit_ns))
+      s_ok = 0;
     const uint4* stage = reinterpret_cast<const uint4*>(wq_stage + slot * kWqStageBytes);
     const int nchunks = static_cast<int>(
         min(static_cast<long long>(kWqStageBytes), ring.bytes - 1ll * st * kWqStageBytes) / 16);
@@ -376,6 +397,7 @@ __global__ void __launch_bounds__(kWqThreads) weight_quant_kernel(
       if (c < nchunks && part == 0)
         packed[wb0 + (1ll * st * kWqStageBytes + 16ll * c) / WORD_BYTES] = bits;
     }
+    if (resident) continue;
     __syncthreads();
     if (tid == 0 && st + kWqStages < ring.nst)
       wq_issue(ring, st + kWqStages, ring.nst + st + kWqStages);
