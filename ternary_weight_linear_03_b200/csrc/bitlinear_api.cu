@@ -164,10 +164,10 @@ int choose_lpr_log2(int cpr) {
   return best;
 }
 
-template <int MT, int XM, int OM>
+template <int MT, int XM, int OM, bool XR>
 bl_status launch_gemv_t(const void* x, const uint8_t* packed, const float* gamma, void* y,
                         int N, int K, cudaStream_t s) {
-  auto kern = bl::gemv_kernel<MT, XM, OM>;
+  auto kern = bl::gemv_kernel<MT, XM, OM, XR>;
   const int smem = MT * K;
   static int configured_smem = -1;
   static int blocks_per_sm = 1;
@@ -189,14 +189,25 @@ bl_status launch_gemv_t(const void* x, const uint8_t* packed, const float* gamma
   return launch_status();
 }
 
+// Activations stay in registers for one token when a lane owns at most kGemvRegChunks
+// chunks of a row (two tokens would spill).
+bool gemv_x_in_registers(int M, int K) {
+  const int cpr = K / 64;
+  const int lpr = 1 << choose_lpr_log2(cpr);
+  return M == 1 && (cpr + lpr - 1) / lpr <= bl::kGemvRegChunks;
+}
+
 template <int XM, int OM>
 bl_status launch_gemv_m(const void* x, const uint8_t* packed, const float* gamma, void* y,
                         int M, int N, int K, cudaStream_t s) {
+  const bool xr = gemv_x_in_registers(M, K);
   switch (M) {
-    case 1: return launch_gemv_t<1, XM, OM>(x, packed, gamma, y, N, K, s);
-    case 2: return launch_gemv_t<2, XM, OM>(x, packed, gamma, y, N, K, s);
-    case 3: return launch_gemv_t<3, XM, OM>(x, packed, gamma, y, N, K, s);
-    case 4: return launch_gemv_t<4, XM, OM>(x, packed, gamma, y, N, K, s);
+    case 1:
+      return xr ? launch_gemv_t<1, XM, OM, true>(x, packed, gamma, y, N, K, s)
+                : launch_gemv_t<1, XM, OM, false>(x, packed, gamma, y, N, K, s);
+    case 2: return launch_gemv_t<2, XM, OM, false>(x, packed, gamma, y, N, K, s);
+    case 3: return launch_gemv_t<3, XM, OM, false>(x, packed, gamma, y, N, K, s);
+    case 4: return launch_gemv_t<4, XM, OM, false>(x, packed, gamma, y, N, K, s);
     default: return BL_ERR_UNSUPPORTED_SHAPE;
   }
 }

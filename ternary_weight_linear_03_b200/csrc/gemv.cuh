@@ -6,8 +6,15 @@
 //   acc[t,n] = sum_k c[n,k] q[t,k] = sum_k u[n,k] q[t,k] - rowsum_t,
 // and one packed 32-bit word (16 trits) unpacks to four int8x4 registers with one shift
 // and one mask each (the packed layout puts trits 16g+4j .. 16g+4j+3 in bits 2j of the
-// four bytes). The byte products run on dp4a; rowsum_t = sum_k q[t,k] comes from the
-// prologue.
+// four bytes). The shift is not even needed: w & (3 << 2j) holds 4^j u per byte, so the
+// dp4a of group j accumulates 4^j times the wanted sum in its own register, and the four
+// chains are recombined with exact arithmetic shifts. rowsum_t = sum_k q[t,k] comes from
+// the prologue.
+//
+// When a lane's activation chunks fit in registers (one token, at most kGemvRegChunks
+// chunks), they are loaded once and every weight row reuses them (no shared-memory
+// traffic in the inner loop), and the next row's weights are loaded while the current
+// row is being summed.
 //
 // Layout. Each lane owns 16-byte chunks (64 trits) of a weight row; LPR lanes share a row
 // and reduce with warp shuffles. The quantized activations live in shared memory with
@@ -24,6 +31,27 @@ namespace bl {
 constexpr int kGemvThreads = 512;
 constexpr int kGemvWarps = kGemvThreads / 32;
 constexpr int kGemvUnroll = 4;
+constexpr int kGemvRegChunks = 4;  // chunks per lane whose activations stay in registers
+
+// dp4a with the first operand's bytes unsigned (weights masked in place reach 128).
+__device__ __forceinline__ int dp4a_us(uint32_t a, int b, int c) {
+  int d;
+  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+// Adds one packed word's 16 trits times 16 int8 activations into the four chains
+// (chain j holds 4^j times its part of the sum).
+__device__ __forceinline__ void gemv_word(uint32_t w, const uint4& xv, int (&a)[4]) {
+  a[0] = __dp4a(static_cast<int>(w & 0x03030303u), static_cast<int>(xv.x), a[0]);
+  a[1] = __dp4a(static_cast<int>(w & 0x0C0C0C0Cu), static_cast<int>(xv.y), a[1]);
+  a[2] = __dp4a(static_cast<int>(w & 0x30303030u), static_cast<int>(xv.z), a[2]);
+  a[3] = dp4a_us(w & 0xC0C0C0C0u, static_cast<int>(xv.w), a[3]);
+}
+// The exact sum of the four chains.
+__device__ __forceinline__ int gemv_combine(const int (&a)[4]) {
+  return a[0] + (a[1] >> 2) + (a[2] >> 4) + (a[3] >> 6);
+}
 
 enum XMode { kXf32 = 0, kXbf16 = 1, kXi8 = 2 };
 enum OMode { kOf32 = 0, kObf16 = 1, kOi32 = 2 };
@@ -58,7 +86,7 @@ __device__ __forceinline__ void load16(const void* x, long long off, float (&v)[
   }
 }
 
-template <int MT, int XM, int OM>
+template <int MT, int XM, int OM, bool XR>
 __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(
     const void* __restrict__ x, const uint8_t* __restrict__ packed,
     const float* __restrict__ gamma_ptr, void* __restrict__ y, int N, int K, int lpr_log2) {
@@ -181,11 +209,79 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(
   const uint4* xs4 = reinterpret_cast<const uint4*>(xs_raw);
   const int xs_row_units = K >> 4;
 
+  if (XR) {
+    // ------------------------------------------------------------ activations in registers
+    uint4 xr[MT][kGemvRegChunks][4];
+#pragma unroll
+    for (int t = 0; t < MT; ++t)
+#pragma unroll
+      for (int u = 0; u < kGemvRegChunks; ++u) {
+        const int c = sub + u * LPR;
+#pragma unroll
+        for (int g = 0; g < 4; ++g)
+          xr[t][u][g] = (c < CPR) ? xs4[t * xs_row_units + g * CPR + c] : make_uint4(0u, 0u, 0u, 0u);
+      }
+    const long long stride = warps_total * RPW;  // rows between two turns of this warp
+    const long long rows_of = (static_cast<long long>(blockIdx.x) * kGemvWarps + warp) * RPW;
+    uint4 wv[kGemvRegChunks];
+    auto load_row = [&](long long row, uint4 (&w)[kGemvRegChunks]) {
+      const uint4* prow = reinterpret_cast<const uint4*>(packed + row * (K >> 2));
+#pragma unroll
+      for (int u = 0; u < kGemvRegChunks; ++u) {
+        const int c = sub + u * LPR;
+        w[u] = (row < N && c < CPR) ? ld_stream_v4(prow + c) : make_uint4(0u, 0u, 0u, 0u);
+      }
+    };
+    load_row(rows_of + rsel, wv);
+    for (long long rbase = rows_of; rbase < N; rbase += stride) {
+      const long long n = rbase + rsel;
+      uint4 wn[kGemvRegChunks];
+      load_row(n + stride, wn);  // next turn's row, in flight while this one is summed
+      int ch[MT][4];
+#pragma unroll
+      for (int t = 0; t < MT; ++t)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) ch[t][j] = 0;
+#pragma unroll
+      for (int u = 0; u < kGemvRegChunks; ++u) {
+        const uint32_t words[4] = {wv[u].x, wv[u].y, wv[u].z, wv[u].w};
+#pragma unroll
+        for (int g = 0; g < 4; ++g)
+#pragma unroll
+          for (int t = 0; t < MT; ++t) gemv_word(words[g], xr[t][u][g], ch[t]);
+      }
+      int acc[MT];
+#pragma unroll
+      for (int t = 0; t < MT; ++t) acc[t] = gemv_combine(ch[t]);
+      for (int off = LPR >> 1; off > 0; off >>= 1) {
+#pragma unroll
+        for (int t = 0; t < MT; ++t) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], off);
+      }
+      if (n < N && sub == 0) {
+#pragma unroll
+        for (int t = 0; t < MT; ++t) {
+          const int a = acc[t] - sh.rowsum[t];
+          const long long o = static_cast<long long>(t) * N + n;
+          if (OM == kOi32) {
+            static_cast<int*>(y)[o] = a;
+          } else {
+            const float v = __fmul_rn(__int2float_rn(a), sh.f[t]);
+            if (OM == kOf32) static_cast<float*>(y)[o] = v;
+            else static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(v);
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kGemvRegChunks; ++u) wv[u] = wn[u];
+    }
+    return;
+  }
+
   for (long long rg = static_cast<long long>(blockIdx.x) * kGemvWarps + warp;
        rg * RPW < N; rg += warps_total) {
     const long long n = rg * RPW + rsel;
     const bool valid = n < N;
-    int acc4[MT][4];  // one chain per 4-trit group of a word: no long dp4a dependency
+    int acc4[MT][4];  // chain j of token t (4^j times its part: see the header)
 #pragma unroll
     for (int t = 0; t < MT; ++t)
 #pragma unroll
@@ -205,28 +301,17 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(
           if (c < CPR) {
             const uint32_t words[4] = {wv[u].x, wv[u].y, wv[u].z, wv[u].w};
 #pragma unroll
-            for (int g = 0; g < 4; ++g) {
-              const uint32_t wd = words[g];
-              const int r0 = static_cast<int>(wd & 0x03030303u);
-              const int r1 = static_cast<int>((wd >> 2) & 0x03030303u);
-              const int r2 = static_cast<int>((wd >> 4) & 0x03030303u);
-              const int r3 = static_cast<int>((wd >> 6) & 0x03030303u);
+            for (int g = 0; g < 4; ++g)
 #pragma unroll
-              for (int t = 0; t < MT; ++t) {
-                const uint4 xv = xs4[t * xs_row_units + g * CPR + c];
-                acc4[t][0] = __dp4a(r0, static_cast<int>(xv.x), acc4[t][0]);
-                acc4[t][1] = __dp4a(r1, static_cast<int>(xv.y), acc4[t][1]);
-                acc4[t][2] = __dp4a(r2, static_cast<int>(xv.z), acc4[t][2]);
-                acc4[t][3] = __dp4a(r3, static_cast<int>(xv.w), acc4[t][3]);
-              }
-            }
+              for (int t = 0; t < MT; ++t)
+                gemv_word(words[g], xs4[t * xs_row_units + g * CPR + c], acc4[t]);
           }
         }
       }
     }
     int acc[MT];
 #pragma unroll
-    for (int t = 0; t < MT; ++t) acc[t] = (acc4[t][0] + acc4[t][1]) + (acc4[t][2] + acc4[t][3]);
+    for (int t = 0; t < MT; ++t) acc[t] = gemv_combine(acc4[t]);
     for (int off = LPR >> 1; off > 0; off >>= 1) {
 #pragma unroll
       for (int t = 0; t < MT; ++t) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], off);
