@@ -209,7 +209,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(
   const uint4* xs4 = reinterpret_cast<const uint4*>(xs_raw);
   const int xs_row_units = K >> 4;
 
-  if (XR) {
+  if constexpr (XR) {
     // ------------------------------------------------------------ activations in registers
     uint4 xr[MT][kGemvRegChunks][4];
 #pragma unroll
@@ -274,59 +274,58 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(
 #pragma unroll
       for (int u = 0; u < kGemvRegChunks; ++u) wv[u] = wn[u];
     }
-    return;
-  }
-
-  for (long long rg = static_cast<long long>(blockIdx.x) * kGemvWarps + warp;
-       rg * RPW < N; rg += warps_total) {
-    const long long n = rg * RPW + rsel;
-    const bool valid = n < N;
-    int acc4[MT][4];  // chain j of token t (4^j times its part: see the header)
+  } else {
+    for (long long rg = static_cast<long long>(blockIdx.x) * kGemvWarps + warp;
+         rg * RPW < N; rg += warps_total) {
+      const long long n = rg * RPW + rsel;
+      const bool valid = n < N;
+      int acc4[MT][4];  // chain j of token t (4^j times its part: see the header)
 #pragma unroll
-    for (int t = 0; t < MT; ++t)
+      for (int t = 0; t < MT; ++t)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) acc4[t][j] = 0;
-    if (valid) {
-      const uint4* prow = reinterpret_cast<const uint4*>(packed + n * (K >> 2));
-      for (int c0 = sub; c0 < CPR; c0 += LPR * kGemvUnroll) {
-        uint4 wv[kGemvUnroll];
+        for (int j = 0; j < 4; ++j) acc4[t][j] = 0;
+      if (valid) {
+        const uint4* prow = reinterpret_cast<const uint4*>(packed + n * (K >> 2));
+        for (int c0 = sub; c0 < CPR; c0 += LPR * kGemvUnroll) {
+          uint4 wv[kGemvUnroll];
 #pragma unroll
-        for (int u = 0; u < kGemvUnroll; ++u) {
-          const int c = c0 + u * LPR;
-          wv[u] = (c < CPR) ? ld_stream_v4(prow + c) : make_uint4(0u, 0u, 0u, 0u);
-        }
+          for (int u = 0; u < kGemvUnroll; ++u) {
+            const int c = c0 + u * LPR;
+            wv[u] = (c < CPR) ? ld_stream_v4(prow + c) : make_uint4(0u, 0u, 0u, 0u);
+          }
 #pragma unroll
-        for (int u = 0; u < kGemvUnroll; ++u) {
-          const int c = c0 + u * LPR;
-          if (c < CPR) {
-            const uint32_t words[4] = {wv[u].x, wv[u].y, wv[u].z, wv[u].w};
+          for (int u = 0; u < kGemvUnroll; ++u) {
+            const int c = c0 + u * LPR;
+            if (c < CPR) {
+              const uint32_t words[4] = {wv[u].x, wv[u].y, wv[u].z, wv[u].w};
 #pragma unroll
-            for (int g = 0; g < 4; ++g)
+              for (int g = 0; g < 4; ++g)
 #pragma unroll
-              for (int t = 0; t < MT; ++t)
-                gemv_word(words[g], xs4[t * xs_row_units + g * CPR + c], acc4[t]);
+                for (int t = 0; t < MT; ++t)
+                  gemv_word(words[g], xs4[t * xs_row_units + g * CPR + c], acc4[t]);
+            }
           }
         }
       }
-    }
-    int acc[MT];
+      int acc[MT];
 #pragma unroll
-    for (int t = 0; t < MT; ++t) acc[t] = gemv_combine(acc4[t]);
-    for (int off = LPR >> 1; off > 0; off >>= 1) {
+      for (int t = 0; t < MT; ++t) acc[t] = gemv_combine(acc4[t]);
+      for (int off = LPR >> 1; off > 0; off >>= 1) {
 #pragma unroll
-      for (int t = 0; t < MT; ++t) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], off);
-    }
-    if (valid && sub == 0) {
+        for (int t = 0; t < MT; ++t) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], off);
+      }
+      if (valid && sub == 0) {
 #pragma unroll
-      for (int t = 0; t < MT; ++t) {
-        const int a = acc[t] - sh.rowsum[t];
-        const long long o = static_cast<long long>(t) * N + n;
-        if (OM == kOi32) {
-          static_cast<int*>(y)[o] = a;
-        } else {
-          const float v = __fmul_rn(__int2float_rn(a), sh.f[t]);
-          if (OM == kOf32) static_cast<float*>(y)[o] = v;
-          else static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(v);
+        for (int t = 0; t < MT; ++t) {
+          const int a = acc[t] - sh.rowsum[t];
+          const long long o = static_cast<long long>(t) * N + n;
+          if (OM == kOi32) {
+            static_cast<int*>(y)[o] = a;
+          } else {
+            const float v = __fmul_rn(__int2float_rn(a), sh.f[t]);
+            if (OM == kOf32) static_cast<float*>(y)[o] = v;
+            else static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(v);
+          }
         }
       }
     }
