@@ -164,10 +164,10 @@ int choose_lpr_log2(int cpr) {
   return best;
 }
 
-template <int MT, int XM, int OM, bool XR>
+template <int MT, int XM, int OM, bool XR, int R>
 bl_status launch_gemv_t(const void* x, const uint8_t* packed, const float* gamma, void* y,
                         int N, int K, cudaStream_t s) {
-  auto kern = bl::gemv_kernel<MT, XM, OM, XR>;
+  auto kern = bl::gemv_kernel<MT, XM, OM, XR, R>;
   const int smem = MT * K;
   static int configured_smem = -1;
   static int blocks_per_sm = 1;
@@ -182,7 +182,7 @@ bl_status launch_gemv_t(const void* x, const uint8_t* packed, const float* gamma
       blocks_per_sm < 1)
     blocks_per_sm = 1;
   const int lpr_log2 = choose_lpr_log2(K / 64);
-  const long long rows_per_block = static_cast<long long>(bl::kGemvWarps) * (32 >> lpr_log2);
+  const long long rows_per_block = static_cast<long long>(bl::kGemvWarps) * (32 >> lpr_log2) * R;
   const long long need = (N + rows_per_block - 1) / rows_per_block;
   const int grid = static_cast<int>(std::min<long long>(need, 1ll * blocks_per_sm * num_sms()));
   kern<<<grid, bl::kGemvThreads, smem, s>>>(x, packed, gamma, y, N, K, lpr_log2);
@@ -197,17 +197,30 @@ bool gemv_x_in_registers(int M, int K) {
   return M == 1 && (cpr + lpr - 1) / lpr <= bl::kGemvRegChunks;
 }
 
+// Rows summed at once per warp on the shared-memory path: two when one warp covers a
+// whole row (large K) and there are rows enough for every warp of the GPU twice over.
+bool gemv_two_rows(int N, int K) {
+  return choose_lpr_log2(K / 64) == 5 && N >= 2 * bl::kGemvWarps * num_sms();
+}
+
+template <int MT, int XM, int OM>
+bl_status launch_gemv_r(const void* x, const uint8_t* packed, const float* gamma, void* y,
+                        int N, int K, cudaStream_t s) {
+  return gemv_two_rows(N, K) ? launch_gemv_t<MT, XM, OM, false, 2>(x, packed, gamma, y, N, K, s)
+                             : launch_gemv_t<MT, XM, OM, false, 1>(x, packed, gamma, y, N, K, s);
+}
+
 template <int XM, int OM>
 bl_status launch_gemv_m(const void* x, const uint8_t* packed, const float* gamma, void* y,
                         int M, int N, int K, cudaStream_t s) {
-  const bool xr = gemv_x_in_registers(M, K);
   switch (M) {
     case 1:
-      return xr ? launch_gemv_t<1, XM, OM, true>(x, packed, gamma, y, N, K, s)
-                : launch_gemv_t<1, XM, OM, false>(x, packed, gamma, y, N, K, s);
-    case 2: return launch_gemv_t<2, XM, OM, false>(x, packed, gamma, y, N, K, s);
-    case 3: return launch_gemv_t<3, XM, OM, false>(x, packed, gamma, y, N, K, s);
-    case 4: return launch_gemv_t<4, XM, OM, false>(x, packed, gamma, y, N, K, s);
+      return gemv_x_in_registers(M, K)
+                 ? launch_gemv_t<1, XM, OM, true, 1>(x, packed, gamma, y, N, K, s)
+                 : launch_gemv_r<1, XM, OM>(x, packed, gamma, y, N, K, s);
+    case 2: return launch_gemv_r<2, XM, OM>(x, packed, gamma, y, N, K, s);
+    case 3: return launch_gemv_r<3, XM, OM>(x, packed, gamma, y, N, K, s);
+    case 4: return launch_gemv_r<4, XM, OM>(x, packed, gamma, y, N, K, s);
     default: return BL_ERR_UNSUPPORTED_SHAPE;
   }
 }

@@ -86,7 +86,9 @@ __device__ __forceinline__ void load16(const void* x, long long off, float (&v)[
   }
 }
 
-template <int MT, int XM, int OM, bool XR>
+// XR: activations in registers (one token). R: rows a warp sums at once on the shared-
+// memory path (2 lets every activation load feed two rows; worth it only with many rows).
+template <int MT, int XM, int OM, bool XR, int R>
 __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(
     const void* __restrict__ x, const uint8_t* __restrict__ packed,
     const float* __restrict__ gamma_ptr, void* __restrict__ y, int N, int K, int lpr_log2) {
@@ -275,56 +277,76 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(
       for (int u = 0; u < kGemvRegChunks; ++u) wv[u] = wn[u];
     }
   } else {
+    // ------------------------------------------------------------ activations in smem
+    // A warp sums R rows at once (rg, rg + warps_total, ...), so every activation load from
+    // shared memory feeds R rows.
     for (long long rg = static_cast<long long>(blockIdx.x) * kGemvWarps + warp;
-         rg * RPW < N; rg += warps_total) {
-      const long long n = rg * RPW + rsel;
-      const bool valid = n < N;
-      int acc4[MT][4];  // chain j of token t (4^j times its part: see the header)
+         rg * RPW < N; rg += R * warps_total) {
+      long long n[R];
+      bool valid[R];
+      const uint4* prow[R];
 #pragma unroll
-      for (int t = 0; t < MT; ++t)
+      for (int q = 0; q < R; ++q) {
+        n[q] = (rg + q * warps_total) * RPW + rsel;
+        valid[q] = n[q] < N;
+        prow[q] = reinterpret_cast<const uint4*>(packed + (valid[q] ? n[q] : 0) * (K >> 2));
+      }
+      int acc4[R][MT][4];  // chain j of token t (4^j times its part: see the header)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc4[t][j] = 0;
-      if (valid) {
-        const uint4* prow = reinterpret_cast<const uint4*>(packed + n * (K >> 2));
-        for (int c0 = sub; c0 < CPR; c0 += LPR * kGemvUnroll) {
-          uint4 wv[kGemvUnroll];
+      for (int q = 0; q < R; ++q)
+#pragma unroll
+        for (int t = 0; t < MT; ++t)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) acc4[q][t][j] = 0;
+      for (int c0 = sub; c0 < CPR; c0 += LPR * kGemvUnroll) {
+        uint4 wv[R][kGemvUnroll];
+#pragma unroll
+        for (int q = 0; q < R; ++q)
 #pragma unroll
           for (int u = 0; u < kGemvUnroll; ++u) {
             const int c = c0 + u * LPR;
-            wv[u] = (c < CPR) ? ld_stream_v4(prow + c) : make_uint4(0u, 0u, 0u, 0u);
+            wv[q][u] = (valid[q] && c < CPR) ? ld_stream_v4(prow[q] + c) : make_uint4(0u, 0u, 0u, 0u);
           }
 #pragma unroll
-          for (int u = 0; u < kGemvUnroll; ++u) {
-            const int c = c0 + u * LPR;
-            if (c < CPR) {
-              const uint32_t words[4] = {wv[u].x, wv[u].y, wv[u].z, wv[u].w};
+        for (int u = 0; u < kGemvUnroll; ++u) {
+          const int c = c0 + u * LPR;
+          if (c < CPR) {
 #pragma unroll
-              for (int g = 0; g < 4; ++g)
+            for (int g = 0; g < 4; ++g)
 #pragma unroll
-                for (int t = 0; t < MT; ++t)
-                  gemv_word(words[g], xs4[t * xs_row_units + g * CPR + c], acc4[t]);
-            }
+              for (int t = 0; t < MT; ++t) {
+                const uint4 xv = xs4[t * xs_row_units + g * CPR + c];
+#pragma unroll
+                for (int q = 0; q < R; ++q) {
+                  const uint32_t w = g == 0 ? wv[q][u].x : g == 1 ? wv[q][u].y
+                                   : g == 2 ? wv[q][u].z : wv[q][u].w;
+                  gemv_word(w, xv, acc4[q][t]);
+                }
+              }
           }
         }
       }
-      int acc[MT];
 #pragma unroll
-      for (int t = 0; t < MT; ++t) acc[t] = gemv_combine(acc4[t]);
-      for (int off = LPR >> 1; off > 0; off >>= 1) {
+      for (int q = 0; q < R; ++q) {
+        int acc[MT];
 #pragma unroll
-        for (int t = 0; t < MT; ++t) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], off);
-      }
-      if (valid && sub == 0) {
+        for (int t = 0; t < MT; ++t) acc[t] = gemv_combine(acc4[q][t]);
+        for (int off = LPR >> 1; off > 0; off >>= 1) {
 #pragma unroll
-        for (int t = 0; t < MT; ++t) {
-          const int a = acc[t] - sh.rowsum[t];
-          const long long o = static_cast<long long>(t) * N + n;
-          if (OM == kOi32) {
-            static_cast<int*>(y)[o] = a;
-          } else {
-            const float v = __fmul_rn(__int2float_rn(a), sh.f[t]);
-            if (OM == kOf32) static_cast<float*>(y)[o] = v;
-            else static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(v);
+          for (int t = 0; t < MT; ++t) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], off);
+        }
+        if (valid[q] && sub == 0) {
+#pragma unroll
+          for (int t = 0; t < MT; ++t) {
+            const int a = acc[t] - sh.rowsum[t];
+            const long long o = static_cast<long long>(t) * N + n[q];
+            if (OM == kOi32) {
+              static_cast<int*>(y)[o] = a;
+            } else {
+              const float v = __fmul_rn(__int2float_rn(a), sh.f[t]);
+              if (OM == kOf32) static_cast<float*>(y)[o] = v;
+              else static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(v);
+            }
           }
         }
       }
