@@ -58,12 +58,16 @@ def parse():
     return p.parse_args()
 
 
+KERNEL_SOURCES = {"weight_quant_kernel": "weight_quant.cuh", "gemm_tc_kernel": "gemm_tc.cuh",
+                  "gemm_skinny_kernel": "gemm_skinny.cuh", "gemv_kernel": "gemv.cuh"}
+
+
 def ncu_traffic(kernel: str, workload: str):
     """DRAM bytes per launch of `kernel` from the committed ncu capture, or None when the
     capture was of another workload or the kernel source changed since it was taken."""
     import hashlib
     path = os.path.join(ROOT, "profiles", "traffic.json")
-    src = os.path.join(ROOT, "ternary_weight_linear_03_b200", "csrc", "weight_quant.cuh")
+    src = os.path.join(ROOT, "ternary_weight_linear_03_b200", "csrc", KERNEL_SOURCES[kernel])
     try:
         rec = json.load(open(path))[kernel]
         sha = hashlib.sha1(open(src, "rb").read()).hexdigest()
@@ -300,22 +304,38 @@ def main():
     # per-launch times: the event nodes of each copy's graph as of its last replay
     wq_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     fw_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
-    hbm_peak, _, peak_kind = peaks()
+    hbm_peak, bf16_peak, peak_kind = peaks()
     wq_bytes = N * K * 4 + N * K // 4
     fw_bytes = N * K // 4 + M * K * 2 + M * N * 2
+    fw_ops = 2.0 * M * N * K
+    others = {"quantize_weights_ms": wq_ms, "forward_ms": fw_ms,
+              "forward_GBps": fw_bytes / (fw_ms * 1e-3) / 1e9,
+              "forward_TOPS": fw_ops / (fw_ms * 1e-3) / 1e12}
     if wq_ms >= fw_ms:
-        dom = {"kernel": "bitlinear_quantize_weights (absmean + ternarize/pack)",
-               "bytes": wq_bytes, "ms": wq_ms,
-               "traffic": ncu_traffic("weight_quant_kernel", name)}
+        achieved = wq_bytes / (wq_ms * 1e-3) / 1e9
+        roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                    "frac": achieved / hbm_peak,
+                    "traffic": ncu_traffic("weight_quant_kernel", name),
+                    "peak_source": f"{peak_kind} HBM copy",
+                    "kernel": "bitlinear_quantize_weights (absmean + ternarize/pack)",
+                    "algorithmic_bytes": wq_bytes, "ms_per_launch": wq_ms}
+    elif M > 256:
+        # the tcgen05 int8 GEMM: a dense contraction, measured against the int8 tensor peak
+        # (the measured bf16 burst figure times the nominal int8:bf16 ratio of 2)
+        i8_peak = 2.0 * bf16_peak
+        achieved = fw_ops / (fw_ms * 1e-3) / 1e12
+        roofline = {"bound": "tensor", "achieved": achieved, "peak": i8_peak, "unit": "TFLOP/s",
+                    "frac": achieved / i8_peak, "traffic": ncu_traffic("gemm_tc_kernel", name),
+                    "peak_source": f"{peak_kind} bf16 burst x 2 (int8)",
+                    "kernel": "bitlinear_forward (activation quant + tcgen05 int8 GEMM)",
+                    "algorithmic_ops": fw_ops, "ms_per_launch": fw_ms}
     else:
-        dom = {"kernel": "bitlinear_forward", "bytes": fw_bytes, "ms": fw_ms, "traffic": None}
-    achieved = dom["bytes"] / (dom["ms"] * 1e-3) / 1e9
-    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                "frac": achieved / hbm_peak, "traffic": dom["traffic"], "peak_source": peak_kind,
-                "kernel": dom["kernel"], "algorithmic_bytes": dom["bytes"],
-                "ms_per_launch": dom["ms"],
-                "others": {"quantize_weights_ms": wq_ms, "forward_ms": fw_ms,
-                           "forward_GBps": fw_bytes / (fw_ms * 1e-3) / 1e9}}
+        achieved = fw_bytes / (fw_ms * 1e-3) / 1e9
+        roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                    "frac": achieved / hbm_peak, "traffic": None,
+                    "peak_source": f"{peak_kind} HBM copy", "kernel": "bitlinear_forward",
+                    "algorithmic_bytes": fw_bytes, "ms_per_launch": fw_ms}
+    roofline["others"] = others
 
     tokens = M * args.steps * world
     value = tokens / (elapsed_ms * 1e-3)
