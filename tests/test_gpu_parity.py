@@ -173,6 +173,8 @@ def test_quantize_acts_bit_exact(M, K, dtype, outliers):
 
 CONTRACT_SHAPES = [
     (1, 256, 256), (2, 293, 192), (3, 1000, 1536), (4, 777, 64),       # CUDA-core path
+    (1, 4099, 8192), (1, 3001, 2048),            # one token, activations in registers
+    (1, 5000, 28672), (2, 4800, 2048), (4, 4737, 4096),  # large K: two rows per warp
     (5, 300, 640), (16, 4096, 1536), (130, 293, 8640), (300, 520, 1536),  # tensor-core path
     (129, 257, 128), (64, 64, 64), (256, 1000, 3200), (257, 300, 640), (17, 8640, 3200),
     (48, 129, 8640), (176, 520, 8192),
