@@ -27,7 +27,11 @@
 // warp then issues the group's 8 MMAs and one commit while the unpack warps go on to the
 // next group; the commit's barrier (done ring) frees the A slot and the token tile. At
 // small M each MMA is a few tens of cycles of tensor work, so these per-group handoffs,
-// not bandwidth, set the pace.
+// not bandwidth, set the pace, and the unpack warps are the critical path: every mbarrier
+// wait (a hundred to three hundred cycles on B200 even for a completed phase) is done by
+// the MMA warp, which has slack. Before the handoff of group g it makes sure that group
+// g + 1 may start (its W super-tile has landed, the MMAs that last read its A slot are
+// done), so the unpack warps never wait on an mbarrier.
 //
 // 6 warps: warps 0-3 unpack (thread t owns weight row t, TMEM lane t) and run the
 // epilogue at the end; warp 4 issues the TMA loads; warp 5 owns the TMEM allocation and
@@ -318,10 +322,29 @@ __global__ void __launch_bounds__(sk::THREADS, 1) gemm_skinny_kernel(
     const uint32_t a_tmem0 = tmem_base + a_col0;
     int su = 0, sx = 0, sw = 0;
     uint32_t xph = 0;
-    bool failed = false;  // a token-tile wait gave up (the abort flag is set)
+    bool failed = false;  // a wait gave up (the abort flag is set)
+    // Waits (all lanes) until group gn may be unpacked: its W super-tile has landed and the
+    // MMAs of group gn - SU, the last readers of its A slot, are done.
+    auto prepare = [&](int gn) -> bool {
+      bool ok = true;
+      if (((gn * KG) & (KPS - 1)) == 0) {
+        const int st = (gn * KG) / KPS;  // super-tiles before this one
+        ok = tc_wait(&bar->w_full[st % pl.sw], static_cast<uint32_t>((st / pl.sw) & 1),
+                     limit_ns, abort_flag);
+      }
+      if (gn >= SU) {
+        const int i = gn - SU;
+        ok = ok && tc_wait(&bar->done[i & (SD - 1)], static_cast<uint32_t>((i / SD) & 1),
+                           limit_ns, abort_flag);
+      }
+      return __all_sync(0xffffffffu, ok);
+    };
+    bool stop = group_bar_or(ng > 0 && !prepare(0));  // group 0 may start
     int g = 0;
-    for (; g < ng; ++g) {
-      if (group_bar_or(*abort_flag != 0)) break;  // group g's rows are in TMEM
+    for (; !stop && g < ng; ++g) {
+      const bool next_ok = (g + 1 < ng) ? prepare(g + 1) : true;
+      tc_fence_before();
+      if (group_bar_or(!next_ok || *abort_flag != 0)) break;  // group g's rows are in TMEM
       const int q0 = (g * KG) & (KPS - 1);
       const bool last_of_tile = (q0 + KG == KPS) || (g == ng - 1);
       bool xok = true;
@@ -362,58 +385,45 @@ __global__ void __launch_bounds__(sk::THREADS, 1) gemm_skinny_kernel(
     }
   } else {
     // ------------------------------------------------------------------ warps 0-3
+    // No mbarrier waits here: passing the handoff before group g means the MMA warp has
+    // seen group g's W super-tile land and its A slot freed.
     const int r = threadIdx.x;  // weight row of the tile owned by this thread (0..127)
     const int rs = r & 7;       // its 128-byte swizzle phase
     const uint32_t a_lane = tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + a_col0;
     int sw = 0, su = 0;
-    uint32_t wph = 0;
+    bool stop = group_bar_or(false);  // group 0 may start
     int g = 0;
-    for (; g < ng; ++g) {
+    for (; !stop && g < ng; ++g) {
       const int q0 = (g * KG) & (KPS - 1);  // first K block of the group in its super-tile
-      // lane 0 waits for the warp; __syncwarp then orders the other lanes after it. A warp
-      // whose wait fails skips its work but still meets the others at the handoff.
-      bool got = true;
-      if (lane == 0) {
-        if (q0 == 0) got = tc_wait(&bar->w_full[sw], wph, limit_ns, abort_flag);
-        if (g >= SU) {  // A slot su is free once group g - SU has been consumed
-          const int i = g - SU;
-          got = got && tc_wait(&bar->done[i & (SD - 1)], static_cast<uint32_t>((i / SD) & 1),
-                               limit_ns, abort_flag);
-        }
-      }
-      got = __shfl_sync(0xffffffffu, got, 0);
-      __syncwarp();
-      if (got) {
-        tc_fence_after();
-        const unsigned char* src = sWp + sw * WP_BYTES + r * 128;
+      tc_fence_after();
+      const unsigned char* src = sWp + sw * WP_BYTES + r * 128;
 #pragma unroll
-        for (int kq = 0; kq < KG; ++kq) {
-          const int q = q0 + kq;
-          uint32_t a[32];  // the row's 128 unpacked codes of K block q, 4 per register
+      for (int kq = 0; kq < KG; ++kq) {
+        const int q = q0 + kq;
+        uint32_t a[32];  // the row's 128 unpacked codes of K block q, 4 per register
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            // logical 16-byte chunk 2q+h of the packed row = K block q, words 4h .. 4h+3
-            const uint4 p = *reinterpret_cast<const uint4*>(src + (((2 * q + h) ^ rs) << 4));
-            const uint32_t words[4] = {p.x, p.y, p.z, p.w};
+        for (int h = 0; h < 2; ++h) {
+          // logical 16-byte chunk 2q+h of the packed row = K block q, words 4h .. 4h+3
+          const uint4 p = *reinterpret_cast<const uint4*>(src + (((2 * q + h) ^ rs) << 4));
+          const uint32_t words[4] = {p.x, p.y, p.z, p.w};
 #pragma unroll
-            for (int mq = 0; mq < 4; ++mq) {
-              const uint32_t w = words[mq];
-              const int c = 16 * h + 4 * mq;  // first column of this 16-trit group
-              a[c + 0] = w & 0x03030303u;
-              a[c + 1] = (w >> 2) & 0x03030303u;
-              a[c + 2] = (w >> 4) & 0x03030303u;
-              a[c + 3] = (w >> 6) & 0x03030303u;
-            }
+          for (int mq = 0; mq < 4; ++mq) {
+            const uint32_t w = words[mq];
+            const int c = 16 * h + 4 * mq;  // first column of this 16-trit group
+            a[c + 0] = w & 0x03030303u;
+            a[c + 1] = (w >> 2) & 0x03030303u;
+            a[c + 2] = (w >> 4) & 0x03030303u;
+            a[c + 3] = (w >> 6) & 0x03030303u;
           }
-          tmem_st_x32(a_lane + static_cast<uint32_t>(su * G_COLS + kq * A_COLS), a);
         }
-        tmem_st_wait();
+        tmem_st_x32(a_lane + static_cast<uint32_t>(su * G_COLS + kq * A_COLS), a);
       }
+      tmem_st_wait();
       tc_fence_before();
-      if (group_bar_or(!got || *abort_flag != 0)) break;  // hand group g to the MMA warp
+      if (group_bar_or(*abort_flag != 0)) break;  // hand group g to the MMA warp
       const bool last_of_tile = (q0 + KG == KPS) || (g == ng - 1);
       if (++su == SU) su = 0;
-      if (last_of_tile && ++sw == pl.sw) { sw = 0; wph ^= 1u; }
+      if (last_of_tile && ++sw == pl.sw) sw = 0;
     }
     const bool ok = (g == ng);
     // ---------------------------------------------------------------- epilogue
