@@ -5,6 +5,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <mutex>
@@ -25,6 +26,7 @@ constexpr int kGemvMaxM = 4;            // M above this runs a tensor-core kerne
 constexpr int kSkinnyMaxM = 256;        // M above this runs the prefill GEMM
 constexpr int kGemvMaxSmem = 200 * 1024;  // xq rows held in shared memory by the GEMV
 constexpr unsigned long long kWaitLimitNs = 4000000000ull;  // 4 s per mbarrier wait
+constexpr int kMinKbPerSplit = 8;  // skinny split-K: K blocks per split, at least
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -81,11 +83,17 @@ SkinnyPlan skinny_plan(int M, int N, int K) {
   p.bnt = (M + 15) / 16 * 16;
   p.tiles = (N + bl::sk::BW - 1) / bl::sk::BW;
   const int KB = (K + bl::sk::BK - 1) / bl::sk::BK;
-  // Split K only when the weight tiles alone leave most SMs idle, and keep at least 4
-  // K blocks per split so that each CTA streams long enough to cover its fixed costs.
+  // Split K only when the weight tiles alone leave most SMs idle; keep at least
+  // kMinKbPerSplit K blocks per split so that each CTA streams long enough to cover its
+  // fixed costs, and keep the int32 sums the splits exchange (M x N x 4 bytes each)
+  // within a quarter of the packed weight bytes (measured on B200: beyond that the
+  // reduction costs more than the extra SMs bring).
   long long splits = 1;
   if (p.tiles < num_sms()) splits = (num_sms() + p.tiles - 1) / p.tiles;
-  splits = std::max<long long>(1, std::min<long long>(splits, std::max(1, KB / 4)));
+  const long long by_traffic = static_cast<long long>(
+      (static_cast<double>(N) * K / 4.0) / (4.0 * 4.0 * static_cast<double>(M) * N));
+  splits = std::max<long long>(
+      1, std::min<long long>({splits, std::max(1, KB / kMinKbPerSplit), by_traffic}));
   p.kbps = static_cast<int>((KB + splits - 1) / splits);
   p.kbps = (p.kbps + bl::sk::KPS - 1) / bl::sk::KPS * bl::sk::KPS;  // whole super-tiles
   p.splits = (KB + p.kbps - 1) / p.kbps;                          // no empty split
