@@ -45,10 +45,8 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 // Test of phase completion that may suspend the thread for a hardware-chosen time while
-// the phase is incomplete. A suspended waiter takes no issue slots, so a spinning role
-// does not slow the warps it shares an SM sub-partition with (measured: with the
-// non-suspending test_wait form, the waiting MMA-issuing warp slowed the unpack warp beside
-// it by about 1 us per K block).
+// the phase is incomplete (a suspended waiter takes no issue slots; the non-suspending
+// test_wait form measured the same in these kernels).
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
