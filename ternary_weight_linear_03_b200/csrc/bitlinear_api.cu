@@ -49,7 +49,13 @@ int num_sms() {
   return sms;
 }
 
-bool use_gemv(int M, int K) { return M <= kGemvMaxM && static_cast<long long>(M) * K <= kGemvMaxSmem; }
+// The CUDA-core GEMV for one or two tokens, and for up to kGemvMaxM tokens when the packed
+// weights are small (at most 2 MB, where the tensor-core kernel's fixed latency dominates);
+// measured on B200 against the skinny tensor-core kernel on the decode shapes.
+bool use_gemv(int M, int N, int K) {
+  if (static_cast<long long>(M) * K > kGemvMaxSmem) return false;
+  return M <= 2 || (M <= kGemvMaxM && static_cast<long long>(N) * K / 4 <= (2ll << 20));
+}
 
 // Workspace layout of the forward / contract paths that run the GEMM:
 //   [xq M*K int8][scale M fp32][rowsum M int32], each 256-byte aligned.
@@ -345,7 +351,7 @@ bl_status launch_skinny(const int8_t* xq, const uint8_t* packed, const int* rows
 
 // Workspace bytes the forward / contract paths need for (M, N, K).
 size_t fwd_ws_bytes(int M, int N, int K) {
-  if (use_gemv(M, K)) return 0;
+  if (use_gemv(M, N, K)) return 0;
   if (M <= kSkinnyMaxM) return skinny_ws_layout(nullptr, M, N, K, skinny_plan(M, N, K)).bytes;
   return fwd_ws_layout(nullptr, M, K).bytes;
 }
@@ -491,7 +497,7 @@ bl_status bitlinear_forward(const void* x, int x_dtype, const uint8_t* packed,
   if (!aligned16(x) || !aligned16(packed) || !aligned16(gamma) || !aligned16(y))
     return BL_ERR_MISALIGNED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (use_gemv(M, K)) {
+  if (use_gemv(M, N, K)) {
     if (x_dtype == BL_BF16)
       return launch_gemv_x<bl::kXbf16>(x, packed, gamma, y, y_dtype, M, N, K, s);
     return launch_gemv_x<bl::kXf32>(x, packed, gamma, y, y_dtype, M, N, K, s);
@@ -516,7 +522,7 @@ bl_status bitlinear_contract_i32(const int8_t* xq, const uint8_t* packed, int32_
   if (!shape_ok(M, N, K)) return BL_ERR_UNSUPPORTED_SHAPE;
   if (!aligned16(xq) || !aligned16(packed) || !aligned16(acc)) return BL_ERR_MISALIGNED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (use_gemv(M, K)) return launch_gemv_x<bl::kXi8>(xq, packed, nullptr, acc, BL_I32, M, N, K, s);
+  if (use_gemv(M, N, K)) return launch_gemv_x<bl::kXi8>(xq, packed, nullptr, acc, BL_I32, M, N, K, s);
   if (!ws) return BL_ERR_WORKSPACE;
   if (!aligned16(ws)) return BL_ERR_MISALIGNED;
   if (ws_bytes < fwd_ws_bytes(M, N, K)) return BL_ERR_WORKSPACE;
@@ -559,7 +565,7 @@ bl_status bitlinear_forward_noalloc(const void* x, int x_dtype, const uint8_t* p
   if (!aligned16(x) || !aligned16(packed) || !aligned16(gamma) || !aligned16(y))
     return BL_ERR_MISALIGNED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (use_gemv(M, K)) {
+  if (use_gemv(M, N, K)) {
     if (x_dtype == BL_BF16)
       return launch_gemv_x<bl::kXbf16>(x, packed, gamma, y, y_dtype, M, N, K, s);
     return launch_gemv_x<bl::kXf32>(x, packed, gamma, y, y_dtype, M, N, K, s);

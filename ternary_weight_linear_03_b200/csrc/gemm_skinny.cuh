@@ -1,4 +1,5 @@
-// Skinny BitLinear (4 < M <= 256 tokens) on the tcgen05 tensor cores, operands swapped:
+// Skinny BitLinear (up to 256 tokens, above the GEMV range) on the tcgen05 tensor cores,
+// operands swapped:
 //   D[n][t] = sum_k u[n][k] * xq[t][k]     (A = 128 unpacked weight rows, B = the M tokens)
 // so the weights fill the MMA's 128-row slot and the few tokens its N slot (16..256), and
 // every weight tile is unpacked once no matter how many tokens there are. This is the

@@ -230,13 +230,15 @@ def test_forward_tiny_config_end_to_end():
     np.testing.assert_array_equal(y.cpu().numpy(), ref)
 
 
-@pytest.mark.parametrize("m_small,m_big", [(4, 5), (256, 257)])
-def test_forward_paths_agree_at_the_switch(m_small, m_big):
-    """M = 4 | 5 switches CUDA-core GEMV -> skinny tensor-core kernel; M = 256 | 257 switches
-    skinny -> prefill GEMM. Rows present in both calls must agree bit for bit (the per-token
-    quantization does not depend on the other tokens)."""
-    W = syn.weights(1000, 1536, 0.02, seed=5)
-    x = syn.activations(m_big, 1536, seed=6)
+@pytest.mark.parametrize("m_small,m_big,N,K", [(4, 5, 1000, 1536), (2, 3, 4800, 2048),
+                                               (256, 257, 1000, 1536)])
+def test_forward_paths_agree_at_the_switch(m_small, m_big, N, K):
+    """CUDA-core GEMV -> skinny tensor-core kernel at M = 4 | 5 for small packed weights and
+    at M = 2 | 3 for larger ones; skinny -> prefill GEMM at M = 256 | 257. Rows present in
+    both calls must agree bit for bit (the per-token quantization does not depend on the
+    other tokens)."""
+    W = syn.weights(N, K, 0.02, seed=5)
+    x = syn.activations(m_big, K, seed=6)
     packed, gamma = bl.quantize_weights(W.cuda())
     yb = bl.forward(x.cuda(), packed, gamma, out_dtype=torch.float32)
     ys = bl.forward(x[:m_small].contiguous().cuda(), packed, gamma, out_dtype=torch.float32)
