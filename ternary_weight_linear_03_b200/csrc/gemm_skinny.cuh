@@ -13,7 +13,8 @@
 //      writes them with one tcgen05.st into TMEM lane r (4 int8 per column): the MMA takes
 //      its A operand straight from tensor memory, so unpacked weights never touch shared
 //      memory (no shared-memory write/read traffic and no proxy fence for them);
-//   X  int8 token tiles (bnt rows x 128, one K block, 128-byte swizzle) in a deep ring.
+//   X  int8 token tiles (bnt rows x 128 per K block, 128-byte swizzle), one ring slot per
+//      group of K blocks.
 //
 // Work unit = (128-row weight tile, K range of whole super-tiles). When there are too few
 // weight tiles to fill the GPU, K is split across CTAs: each split adds its exact int32
@@ -58,11 +59,12 @@ constexpr int THREADS = 192;
 constexpr int MAX_SW = 4, MAX_SX = 16;
 
 static_assert(KPS % KG == 0, "groups tile a super-tile");
-// Ring of per-group completion barriers. Group g's MMAs arrive on done[g % SD]; the
-// unpackers wait for group g - SU before reusing A slot g % SU, the producer for group
-// g - SX before reusing token slot g % SX. SD >= SU and SD >= SX make a waited-for phase
-// unable to be overtaken by the next phase of the same barrier (that one needs the
-// waiter's own later work first), and every waiter waits on every index in order.
+// Ring of per-group completion barriers. Group g's MMAs arrive on done[g % SD]; the MMA
+// warp waits for group g - SU before group g may be unpacked into A slot g % SU, the
+// producer for group g - SX before reusing token slot g % SX. SD >= SU and SD >= SX make a
+// waited-for phase unable to be overtaken by the next phase of the same barrier (that one
+// needs the waiter's own later work first), and every waiter waits on every index in
+// order.
 constexpr int SD = 16;
 static_assert(SD >= MAX_SU && SD >= MAX_SX && (SD & (SD - 1)) == 0, "done ring");
 
