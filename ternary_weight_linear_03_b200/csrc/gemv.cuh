@@ -14,7 +14,9 @@
 // When a lane's activation chunks fit in registers (one token, at most kGemvRegChunks
 // chunks), they are loaded once and every weight row reuses them (no shared-memory
 // traffic in the inner loop), and the next row's weights are loaded while the current
-// row is being summed.
+// row is being summed. Otherwise the activations are read from shared memory, and when
+// one warp covers a whole row and rows are plentiful a warp sums two rows at once, so
+// each activation load feeds both.
 //
 // Layout. Each lane owns 16-byte chunks (64 trits) of a weight row; LPR lanes share a row
 // and reduce with warp shuffles. The quantized activations live in shared memory with

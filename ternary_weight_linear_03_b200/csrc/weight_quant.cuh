@@ -4,12 +4,13 @@
 //
 // One cooperative kernel, two lean passes over W. The second pass reads the stages still
 // held in shared memory when a block's whole range fits its ring, and is otherwise served
-// from L2 whenever W fits there. Every block owns a contiguous range of 16-weight words and streams it
-// through a ring of 16 KB bulk copies (cp.async.bulk into shared memory, 4 in flight per
-// block); thread t handles the 16-byte chunks t + 256 i of each stage.
-//   A  exact sum of |w| (below) into exponent buckets;
+// from L2 whenever W fits there. Every block owns a contiguous range of 16-weight words
+// and streams it through a ring of 16 KB bulk copies (cp.async.bulk into shared memory, 4
+// in flight per block); thread t handles the 16-byte chunks t + 256 i of each stage.
+//   A  exact sum of |w| (below) into exponent buckets, folded into column sums;
 //   -- grid barrier (bounded wait) --
-//      every block turns the buckets into gamma = fl32(fl64(S) / n) and the threshold T;
+//      every block turns the column sums into gamma = fl32(fl64(S) / n) and the
+//      threshold T;
 //   B  code = (w >= T) - (-w >= T), stored as u = code + 1; the 4 (fp32) or 2 (bf16) lanes
 //      holding the chunks of one packed word merge their bits with shuffles.
 //
