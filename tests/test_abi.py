@@ -21,7 +21,8 @@ def lib():
 
 
 def header_symbols():
-    text = open(HEADER).read()
+    with open(HEADER) as f:
+        text = f.read()
     return sorted(set(re.findall(r"\b(bitlinear_\w+)\s*\(", text)))
 
 

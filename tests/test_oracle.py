@@ -26,7 +26,8 @@ def _fsum_gamma(w: np.ndarray) -> np.float32:
 
 def test_hand_worked_example():
     """Every stage of the hand-worked 2x16 example (tests/golden/hand_worked_2x16.json)."""
-    d = json.load(open(os.path.join(GOLDEN, "hand_worked_2x16.json")))
+    with open(os.path.join(GOLDEN, "hand_worked_2x16.json")) as f:
+        d = json.load(f)
     W = np.array(d["W"], np.float32)
     x = np.array(d["x"], np.float32)
     gamma = orc.absmean(W)

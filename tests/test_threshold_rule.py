@@ -46,9 +46,11 @@ def test_threshold_rule_random_and_neighbours():
         below = np.nextafter(t, np.float32(0))
         assert not qualifies(below, d), (d, t, below)
         # the rule itself on a few floats around the threshold
+        tb = int(t.view(np.uint32))
         for k in range(-3, 4):
-            x = t.view(np.uint32) + np.uint32(k) if k >= 0 else t.view(np.uint32) - np.uint32(-k)
-            x = np.uint32(x).view(np.float32)
+            if not 0 < tb + k < 0x7f800000:  # positive finite floats only
+                continue
+            x = np.uint32(tb + k).view(np.float32)
             rule = np.float64(x) > np.float64(d) * (0.5 + 2.0 ** -25)
             assert rule == qualifies(x, d), (d, x)
 
