@@ -26,7 +26,7 @@ EXPORTS = (
     "bitlinear_workspace_size", "bitlinear_quantize_weights", "bitlinear_quantize_acts",
     "bitlinear_forward", "bitlinear_forward_noalloc", "bitlinear_contract_i32",
     "bitlinear_get_device_status",
-    "bitlinear_debug_timeout_probe", "bitlinear_status_string",
+    "bitlinear_debug_timeout_probe", "bitlinear_debug_plan", "bitlinear_status_string",
 )
 
 
@@ -66,6 +66,8 @@ def load_library() -> ctypes.CDLL:
     lib.bitlinear_get_device_status.restype = i
     lib.bitlinear_debug_timeout_probe.argtypes = [u64, p]
     lib.bitlinear_debug_timeout_probe.restype = i
+    lib.bitlinear_debug_plan.argtypes = [i, i, i, i, p, p]
+    lib.bitlinear_debug_plan.restype = i
     lib.bitlinear_status_string.argtypes = [i]
     lib.bitlinear_status_string.restype = ctypes.c_char_p
     _lib = lib
@@ -204,6 +206,17 @@ def get_device_status(stream=None) -> int:
 def debug_timeout_probe(timeout_ns: int, stream=None) -> None:
     _check(load_library().bitlinear_debug_timeout_probe(int(timeout_ns), _stream(stream)),
            "bitlinear_debug_timeout_probe")
+
+
+PATHS = ("gemv", "skinny", "prefill")
+
+
+def debug_plan(M: int, N: int, K: int, sms: int = 148) -> tuple[str, int]:
+    """The kernel a forward of this shape runs and its K splits (host only, no device)."""
+    path, splits = ctypes.c_int(-1), ctypes.c_int(0)
+    _check(load_library().bitlinear_debug_plan(M, N, K, sms, ctypes.byref(path),
+                                               ctypes.byref(splits)), "bitlinear_debug_plan")
+    return PATHS[path.value], splits.value
 
 
 def status_string(status: int) -> str:

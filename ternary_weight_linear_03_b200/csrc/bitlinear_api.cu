@@ -84,7 +84,7 @@ struct SkinnyPlan {
   int splits;  // K ranges per tile
   int kbps;    // 128-wide K blocks per split
 };
-SkinnyPlan skinny_plan(int M, int N, int K) {
+SkinnyPlan skinny_plan_for(int M, int N, int K, int sms) {
   SkinnyPlan p{};
   p.bnt = (M + 15) / 16 * 16;
   p.tiles = (N + bl::sk::BW - 1) / bl::sk::BW;
@@ -95,7 +95,7 @@ SkinnyPlan skinny_plan(int M, int N, int K) {
   // within a quarter of the packed weight bytes (measured on B200: beyond that the
   // reduction costs more than the extra SMs bring).
   long long splits = 1;
-  if (p.tiles < num_sms()) splits = (num_sms() + p.tiles - 1) / p.tiles;
+  if (p.tiles < sms) splits = (sms + p.tiles - 1) / p.tiles;
   const long long by_traffic = static_cast<long long>(
       (static_cast<double>(N) * K / 4.0) / (4.0 * 4.0 * static_cast<double>(M) * N));
   splits = std::max<long long>(
@@ -105,6 +105,7 @@ SkinnyPlan skinny_plan(int M, int N, int K) {
   p.splits = (KB + p.kbps - 1) / p.kbps;                          // no empty split
   return p;
 }
+SkinnyPlan skinny_plan(int M, int N, int K) { return skinny_plan_for(M, N, K, num_sms()); }
 
 // Workspace of the skinny path: the FwdWs part, then (only when splits > 1) the int32
 // sums [M][N] and one arrival counter per weight tile, contiguous so one memset clears
@@ -584,6 +585,21 @@ bl_status bitlinear_debug_timeout_probe(uint64_t timeout_ns, void* stream) {
   if (timeout_ns < 1000ull || timeout_ns > 5000000000ull) return BL_ERR_INVALID_ARG;
   timeout_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(timeout_ns);
   return launch_status();
+}
+
+bl_status bitlinear_debug_plan(int M, int N, int K, int sms, int* path, int* k_splits) {
+  if (!path || !k_splits || sms < 1) return BL_ERR_INVALID_ARG;
+  if (!shape_ok(M, N, K)) return BL_ERR_UNSUPPORTED_SHAPE;
+  *k_splits = 1;
+  if (use_gemv(M, N, K)) {
+    *path = 0;
+  } else if (M <= kSkinnyMaxM) {
+    *path = 1;
+    *k_splits = skinny_plan_for(M, N, K, sms).splits;
+  } else {
+    *path = 2;
+  }
+  return BL_OK;
 }
 
 const char* bitlinear_status_string(bl_status status) {
