@@ -1,21 +1,21 @@
 #!/usr/bin/env python3
-"""BitLinear forward benchmark on B200: one JSON line per run (rank 0).
+"""BitLinear benchmark on B200: one JSON line per run (rank 0).
 
-A step is one pass of the whole BitLinear hot path over one batch: absmean ternary
-quantization of the fp32 weight matrix (gamma, codes, 2-bit packing), per-token int8
-quantization of the activations, the int32 contraction and the rescale to bf16.
+Headline (the default): the 70B-class prefill BitLinear, M = 4096 tokens of bf16
+activations against a 28672 x 8192 ternary weight matrix (K = 8192 -> N = 28672). A step is
+one BitLinear forward of the batch: per-token int8 quantization of the activations, the
+exact int32 contraction on the tcgen05 int8 tensor cores and the rescale to bf16. The
+weights are quantized once before the timed region (absmean gamma, ternary codes, 2-bit
+packing), as a deployed layer holds them; the weight quantization is timed on its own and
+reported in the same line, over every 70B-shaped layer matrix, together with the decode
+shapes (70B up/down, 700M up) and, where built, the 3B 26-layer FFN chain.
 
-The timed loop replays one CUDA graph per step (captured from the same library calls), so
-host launch overhead is not part of the number; `e2e` times the plain library calls with
-host buffers instead.
-
-Default workload: the 700M-class FFN up-projection (K=1536, N=4096, W ~ N(0, 0.02) fp32,
-bf16 activations ~ N(0, 1) with 1% outlier channels x20), M = 16 tokens. Inputs larger
-than L2: the step cycles through enough weight copies (8 x 25 MB) that every step reads
-its weights from HBM.
+The timed loops replay CUDA graphs captured from the library calls, so host launch
+overhead is not part of the kernel numbers; `e2e` times the plain library calls with host
+buffers (host->device copy of the batch, forward, device->host copy of the output).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload NAME] [--M M]
+                    [--workload NAME] [--M M] [--no-others] [--no-cpu-baseline] [--no-e2e]
 
 Multi-GPU (torchrun): every rank runs the same per-GPU workload on its own weights and
 batch (weak scaling, no data-path collective); timing is the max over ranks.
@@ -43,47 +43,58 @@ from ternary_weight_linear_03_b200 import synthetic as syn  # noqa: E402
 
 METRIC = "BitLinear tokens/s; decode HBM GB/s and prefill INT8 TOPS as % of roofline"
 L2_BYTES = 126 * 1024 * 1024
+HEADLINE = "70b_prefill_4096x8192x28672"
+EPS = 1e-5
 
 
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=200)
-    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--steps", type=int, default=100)
+    p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--workload", default="700m_up_1536x4096")
-    p.add_argument("--M", type=int, default=16)
+    p.add_argument("--workload", default=HEADLINE)
+    p.add_argument("--M", type=int, default=None, help="tokens (default: the workload's largest)")
+    p.add_argument("--no-others", action="store_true", help="skip the secondary figures")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
-    return p.parse_args()
+    a = p.parse_args()
+    if a.M is None:
+        a.M = max(syn.WORKLOADS[a.workload]["Ms"])
+    return a
 
 
 KERNEL_SOURCES = {"weight_quant_kernel": "weight_quant.cuh", "gemm_tc_kernel": "gemm_tc.cuh",
                   "gemm_skinny_kernel": "gemm_skinny.cuh", "gemv_kernel": "gemv.cuh"}
 
 
-def ncu_traffic(kernel: str, workload: str):
+def ncu_traffic(kernel: str, workload: str, M: int):
     """DRAM bytes per launch of `kernel` from the committed ncu capture, or None when the
     capture was of another workload or the kernel source changed since it was taken."""
     import hashlib
     path = os.path.join(ROOT, "profiles", "traffic.json")
     src = os.path.join(ROOT, "ternary_weight_linear_03_b200", "csrc", KERNEL_SOURCES[kernel])
     try:
-        rec = json.load(open(path))[kernel]
-        sha = hashlib.sha1(open(src, "rb").read()).hexdigest()
+        with open(path) as f:
+            rec = json.load(f)[kernel]
+        with open(src, "rb") as f:
+            sha = hashlib.sha1(f.read()).hexdigest()
     except (OSError, KeyError, ValueError):
         return None
-    if rec.get("workload") != workload or rec.get("source_sha1") != sha:
+    if rec.get("workload") != workload or rec.get("M") != M or rec.get("source_sha1") != sha:
         return None
     return rec["dram_bytes_per_launch"]
 
 
 def peaks():
+    """(HBM GB/s, bf16 burst TFLOP/s, bf16 sustained TFLOP/s, source)."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
-        d = json.load(open(path))
-        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
-    return 6650.0, 1590.0, "fallback"
+        with open(path) as f:
+            d = json.load(f)
+        return (float(d["hbm_gbs"]), float(d["bf16_tflops"]),
+                float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured")
+    return 6650.0, 1590.0, 1400.0, "fallback"
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -140,85 +151,205 @@ class ClockSampler:
                 "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
-# ----------------------------------------------------------------------------- workload
+# ----------------------------------------------------------------------------- oracle arm
 
 
-def make_inputs(name: str, M: int, device, copies: int, seed_offset: int = 0):
-    wl = syn.WORKLOADS[name]
-    N, K = wl["N"], wl["K"]
-    Ws = [syn.weights(N, K, wl["sigma"], seed=syn.w_seed(name, i) + seed_offset).to(device)
-          for i in range(copies)]
-    xs = [syn.activations(M, K, seed=syn.x_seed(name, M) + 97 * i + seed_offset,
-                          dtype=wl["x_dtype"], outlier_frac=wl["outlier_frac"]).to(device)
-          for i in range(copies)]
-    return N, K, Ws, xs
+class OracleSample:
+    """A bounded sample of one forward step for the oracle (plain single-threaded C++ on
+    the host): the first T tokens against the first R weight rows. The weights are
+    quantized once beforehand (gamma over those rows), as on the GPU side. The work of a
+    step is linear in tokens x rows (quantizing T activation rows is a small part), so a
+    full step takes (M * N) / (T * R) times as long and tokens/s = T * R / (N * step time)."""
+
+    def __init__(self, name: str, M: int):
+        from oracle import oracle as orc
+        self.orc = orc
+        wl = syn.WORKLOADS[name]
+        self.N, self.K, self.M = wl["N"], wl["K"], M
+        self.T = min(M, 16)
+        self.R = min(self.N, 256 if M > 64 else 512)
+        W = syn.weights(self.R, self.K, wl["sigma"], seed=syn.w_seed(name))
+        x = syn.activations(self.T, self.K, seed=syn.x_seed(name, M), dtype=wl["x_dtype"],
+                            outlier_frac=wl["outlier_frac"])
+        self.xin = syn.bf16_bits(x) if x.dtype == torch.bfloat16 else x.numpy()
+        self.packed, self.gamma = orc.quantize_weights(W.numpy(), EPS)
+        self.name = name
+
+    def step(self):
+        self.orc.forward(self.xin, self.packed, self.gamma, out="bf16")
+
+    def tokens_per_s(self, seconds_per_step: float) -> float:
+        return self.T * self.R / (self.N * seconds_per_step)
+
+    def describe(self, steps: int, elapsed: float) -> str:
+        return (f"{steps} steps of tokens 0..{self.T - 1} x weight rows 0..{self.R - 1} of the "
+                f"{self.name} forward (M={self.M}, N={self.N}, K={self.K}; act quant, int32 "
+                f"contraction, rescale to bf16), single-threaded C++ oracle, {elapsed:.1f} s; "
+                f"scaled by (M*N)/(T*R) = {self.M * self.N / (self.T * self.R):.0f} "
+                f"(work is linear in tokens x rows)")
 
 
 def cpu_baseline(name: str, M: int, budget_s: float = 12.0):
-    """The oracle, as it stands, on this host: quantize W and run the forward for M tokens,
-    repeated until budget_s has passed (the whole workload per step)."""
-    from oracle import oracle as orc
-    wl = syn.WORKLOADS[name]
-    N, K = wl["N"], wl["K"]
-    W = syn.weights(N, K, wl["sigma"], seed=syn.w_seed(name)).numpy()
-    x = syn.activations(M, K, seed=syn.x_seed(name, M), dtype=wl["x_dtype"],
-                        outlier_frac=wl["outlier_frac"])
-    xin = syn.bf16_bits(x) if x.dtype == torch.bfloat16 else x.numpy()
+    """The oracle, as it stands, on this host for about budget_s seconds."""
+    s = OracleSample(name, M)
     steps, t0 = 0, time.perf_counter()
     while True:
-        packed, gamma = orc.quantize_weights(W, 1e-5)
-        orc.forward(xin, packed, gamma, out="bf16")
+        s.step()
         steps += 1
         el = time.perf_counter() - t0
         if el >= budget_s:
             break
-    return {"value": M * steps / el, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"{steps} full steps ({name}, M={M}: quantize W {N}x{K} fp32 + forward),"
-                      f" single-threaded C++ oracle, {el:.1f} s"}
+    return {"value": s.tokens_per_s(el / steps), "unit": "tokens/s", "cores": 1,
+            "kind": "oracle", "sample": s.describe(steps, el)}
 
 
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    from oracle import oracle as orc
-    name, M = args.workload, args.M
-    wl = syn.WORKLOADS[name]
-    N, K = wl["N"], wl["K"]
-    W = syn.weights(N, K, wl["sigma"], seed=syn.w_seed(name)).numpy()
-    x = syn.activations(M, K, seed=syn.x_seed(name, M), dtype=wl["x_dtype"],
-                        outlier_frac=wl["outlier_frac"])
-    xin = syn.bf16_bits(x) if x.dtype == torch.bfloat16 else x.numpy()
-    # A bounded sample per step: the first R weight rows go through the whole path
-    # (absmean over those rows, ternarize, pack, forward for all M tokens). Every part of
-    # the work is linear in the number of rows, so tokens/s = M * R / (N * step time).
-    R = min(N, 512)
-    Wr = np.ascontiguousarray(W[:R])
-
-    def step():
-        packed, gamma = orc.quantize_weights(Wr, 1e-5)
-        orc.forward(xin, packed, gamma, out="bf16")
-
+    s = OracleSample(args.workload, args.M)
     for _ in range(args.warmup):
-        step()
+        s.step()
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        step()
+        s.step()
     el = time.perf_counter() - t0
-    value = M * args.steps * R / (N * el)
-    sample = (f"each step: rows 0..{R - 1} of the {N}x{K} weights through absmean, ternarize, "
-              f"pack and the forward of M={M} tokens; scaled by {R}/{N} (work is linear in rows)")
+    value = s.tokens_per_s(el / args.steps)
+    wl = syn.WORKLOADS[args.workload]
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": el * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "i8/i32 (fp32 quantization)", "data": "synthetic",
-        "config": {"workload": name, "M": M, "N": N, "K": K},
+        "vs_baseline": None, "dtype": "i8xternary->i32 (bf16 in/out)", "data": "synthetic",
+        "config": config_of(args.workload, args.M, wl, args.gpus),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                         "sample": sample},
+                         "sample": s.describe(args.steps, el)},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }))
+
+
+def config_of(name: str, M: int, wl: dict, world: int) -> dict:
+    return {"workload": name, "M": M, "N": wl["N"], "K": wl["K"], "w_dtype": "fp32",
+            "x_dtype": str(wl["x_dtype"]).replace("torch.", ""), "out": "bf16",
+            "weights": "quantized once before the timed region (2-bit packed, resident)",
+            "parallelism": f"replicas x{world}"}
+
+
+# ----------------------------------------------------------------------------- GPU helpers
+
+
+def time_in_graph(calls, reps: int = 3):
+    """Per-call device times (ms) of a list of library calls: one CUDA graph with an event
+    node before every call and after the last, replayed `reps` times; the times are those
+    of the last replay. Every call must have run eagerly once before (kernel set-up)."""
+    evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(calls) + 1)]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i, c in enumerate(calls):
+            evs[i].record()
+            c()
+        evs[-1].record()
+    for _ in range(reps):
+        g.replay()
+    torch.cuda.synchronize()
+    times = [evs[i].elapsed_time(evs[i + 1]) for i in range(len(calls))]
+    del g
+    return times
+
+
+def forward_launches(bl, M: int, N: int, K: int) -> int:
+    """Kernels one bitlinear_forward launches (the GEMV alone, or activation quantization
+    followed by a tensor-core kernel), from the library's own plan."""
+    path, _ = bl.debug_plan(M, N, K, sms=torch.cuda.get_device_properties(0).multi_processor_count)
+    return 1 if path == "gemv" else 2
+
+
+def packed_copies(bl, name: str, device, copies: int, seed_offset: int = 0):
+    """`copies` device copies of one quantized weight matrix of the workload (distinct
+    addresses, so rotating through them reads every step's weights from HBM)."""
+    wl = syn.WORKLOADS[name]
+    W = syn.weights(wl["N"], wl["K"], wl["sigma"], seed=syn.w_seed(name) + seed_offset,
+                    device=device)
+    packed, gamma = bl.quantize_weights(W, EPS)
+    del W
+    out = [(packed, gamma)] + [(packed.clone(), gamma.clone()) for _ in range(copies - 1)]
+    torch.cuda.synchronize()
+    return out
+
+
+def act_copies(name: str, M: int, device, copies: int, seed_offset: int = 0):
+    wl = syn.WORKLOADS[name]
+    return [syn.activations(M, wl["K"], seed=syn.x_seed(name, M) + 97 * i + seed_offset,
+                            dtype=wl["x_dtype"], outlier_frac=wl["outlier_frac"], device=device)
+            for i in range(copies)]
+
+
+def decode_figure(bl, name: str, M: int, device, hbm_peak: float, i8_peak: float):
+    """One forward shape timed alone: mean device time per launch over rotated copies of the
+    weights (more than twice L2 in total), GB/s of algorithmic bytes, int8 TOPS, fractions."""
+    wl = syn.WORKLOADS[name]
+    N, K = wl["N"], wl["K"]
+    w_bytes = N * K // 4
+    copies = max(2, math.ceil(2 * L2_BYTES / w_bytes))
+    ws = packed_copies(bl, name, device, copies)
+    xs = act_copies(name, M, device, min(copies, 8))
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+    work = bl.workspace(M, N, K, device)
+    calls = [(lambda i=i: bl.forward(xs[i % len(xs)], ws[i][0], ws[i][1], y=y, ws=work))
+             for i in range(copies)]
+    for c in calls[:2]:
+        c()
+    torch.cuda.synchronize()
+    ms = statistics.mean(time_in_graph(calls))
+    alg_bytes = w_bytes + M * K * 2 + M * N * 2
+    ops = 2.0 * M * N * K
+    gbs = alg_bytes / (ms * 1e-3) / 1e9
+    tops = ops / (ms * 1e-3) / 1e12
+    bound = "hbm" if alg_bytes / (hbm_peak * 1e9) >= ops / (i8_peak * 1e12) else "tensor"
+    path, splits = bl.debug_plan(M, N, K)
+    return {"workload": name, "M": M, "kernel": path, "k_splits": splits, "ms": ms,
+            "GBps": gbs, "frac_hbm": gbs / hbm_peak, "TOPS": tops, "frac_i8": tops / i8_peak,
+            "bound": bound, "tokens_per_s": M / (ms * 1e-3), "weight_copies": copies}
+
+
+# LLaMA-70B-style layer matrices (out x in) and how many of each one layer holds; 80 layers.
+WQ_70B_SHAPES = [(8192, 8192, 2), (1024, 8192, 2), (28672, 8192, 3)]
+WQ_70B_LAYERS = 80
+
+
+def weight_quant_figures(bl, device, hbm_peak: float):
+    """bitlinear_quantize_weights on every 70B-shaped layer matrix (fp32 W ~ N(0, 0.015)),
+    timed per shape over rotated copies, then totalled over 80 layers."""
+    rows, total_ms, total_bytes = [], 0.0, 0
+    for N, K, count in WQ_70B_SHAPES:
+        n_bytes = N * K * 4
+        copies = max(2, math.ceil(2 * L2_BYTES / n_bytes))
+        Ws = [syn.weights(N, K, 0.015, seed=5000 + N + i, device=device) for i in range(copies)]
+        packed = torch.empty((N, K // 4), dtype=torch.uint8, device=device)
+        gamma = torch.empty(1, dtype=torch.float32, device=device)
+        work = bl.workspace(1, N, K, device)
+        calls = [(lambda W=W: bl.quantize_weights(W, EPS, packed=packed, gamma=gamma, ws=work))
+                 for W in Ws]
+        calls[0]()
+        torch.cuda.synchronize()
+        ms = statistics.mean(time_in_graph(calls))
+        alg = n_bytes + N * K // 4
+        gbs = alg / (ms * 1e-3) / 1e9
+        rows.append({"shape": f"{N}x{K}", "per_layer": count, "ms": ms, "GBps": gbs,
+                     "frac_hbm": gbs / hbm_peak, "copies": copies})
+        total_ms += ms * count * WQ_70B_LAYERS
+        total_bytes += alg * count * WQ_70B_LAYERS
+        del Ws, calls
+        torch.cuda.empty_cache()
+    gbs = total_bytes / (total_ms * 1e-3) / 1e9
+    return {"shapes": rows, "all_layers": {"layers": WQ_70B_LAYERS, "ms": total_ms,
+                                           "algorithmic_GB": total_bytes / 1e9, "GBps": gbs,
+                                           "frac_hbm": gbs / hbm_peak,
+                                           "note": "sum over shapes of per-matrix time x count"}}
+
+
+# ----------------------------------------------------------------------------- main
 
 
 def main():
@@ -244,38 +375,39 @@ def main():
     name, M = args.workload, args.M
     wl = syn.WORKLOADS[name]
     N, K = wl["N"], wl["K"]
-    w_bytes = N * K * 4
-    copies = max(2, math.ceil(2 * L2_BYTES / w_bytes))
-    N, K, Ws, xs = make_inputs(name, M, device, copies, seed_offset=bldist.seed_offset(rank))
-    packed = torch.empty((N, K // 4), dtype=torch.uint8, device=device)
-    gamma = torch.empty(1, dtype=torch.float32, device=device)
+    hbm_peak, bf16_peak, _, peak_kind = peaks()
+    i8_peak = 2.0 * bf16_peak  # nominal int8:bf16 dense ratio of 2 on the measured bf16 burst
+
+    # Inputs of consecutive steps rotate over `copies` weight and activation copies, more
+    # than twice L2 in total, so every step reads its operands from HBM (no L2 flush).
+    step_bytes = N * K // 4 + M * K * (2 if wl["x_dtype"] == torch.bfloat16 else 4)
+    copies = max(2, math.ceil(2 * L2_BYTES / step_bytes))
+    off = bldist.seed_offset(rank)
+    ws_copies = packed_copies(bl, name, device, copies, seed_offset=off)
+    xs = act_copies(name, M, device, copies, seed_offset=off)
     y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
-    ws = bl.workspace(M, N, K, device)
+    work = bl.workspace(M, N, K, device)
     stream = torch.cuda.current_stream()
 
-    def step(i, ev=None):
-        if ev is not None:
-            ev[0].record()
-        bl.quantize_weights(Ws[i % copies], 1e-5, packed=packed, gamma=gamma, ws=ws)
-        if ev is not None:
-            ev[1].record()
-        bl.forward(xs[i % copies], packed, gamma, y=y, ws=ws)
-        if ev is not None:
-            ev[2].record()
+    def step(i):
+        packed, gamma = ws_copies[i % copies]
+        bl.forward(xs[i % copies], packed, gamma, y=y, ws=work)
 
-    for i in range(max(args.warmup, copies)):  # eager warm-up also configures every kernel
+    for i in range(max(args.warmup, 2)):  # eager warm-up also configures every kernel
         step(i)
     torch.cuda.synchronize()
     assert bl.get_device_status() == 0
 
-    # One CUDA graph per weight copy (the step's launches with timing-event nodes between
-    # the weight quantization and the forward); the timed loop replays them in turn.
+    # One CUDA graph per copy (event node, forward, event node); the timed loop replays
+    # them in turn, one graph per step.
     graphs, evs = [], []
     for i in range(copies):
-        ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)]
+        ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            step(i, ev)
+            ev[0].record()
+            step(i)
+            ev[1].record()
         graphs.append(g)
         evs.append(ev)
     for i in range(max(3, args.warmup)):
@@ -300,61 +432,28 @@ def main():
     status = bl.get_device_status()
     if status != 0:
         raise SystemExit(f"device status {bl.status_string(status)} after the timed region")
-
-    # per-launch times: the event nodes of each copy's graph as of its last replay
-    wq_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
-    fw_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
-    hbm_peak, bf16_peak, peak_kind = peaks()
-    wq_bytes = N * K * 4 + N * K // 4
-    fw_bytes = N * K // 4 + M * K * 2 + M * N * 2
-    fw_ops = 2.0 * M * N * K
-    others = {"quantize_weights_ms": wq_ms, "forward_ms": fw_ms,
-              "forward_GBps": fw_bytes / (fw_ms * 1e-3) / 1e9,
-              "forward_TOPS": fw_ops / (fw_ms * 1e-3) / 1e12}
-    if wq_ms >= fw_ms:
-        achieved = wq_bytes / (wq_ms * 1e-3) / 1e9
-        roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                    "frac": achieved / hbm_peak,
-                    "traffic": ncu_traffic("weight_quant_kernel", name),
-                    "peak_source": f"{peak_kind} HBM copy",
-                    "kernel": "bitlinear_quantize_weights (absmean + ternarize/pack)",
-                    "algorithmic_bytes": wq_bytes, "ms_per_launch": wq_ms}
-    elif M > 256:
-        # the tcgen05 int8 GEMM: a dense contraction, measured against the int8 tensor peak
-        # (the measured bf16 burst figure times the nominal int8:bf16 ratio of 2)
-        i8_peak = 2.0 * bf16_peak
-        achieved = fw_ops / (fw_ms * 1e-3) / 1e12
-        roofline = {"bound": "tensor", "achieved": achieved, "peak": i8_peak, "unit": "TFLOP/s",
-                    "frac": achieved / i8_peak, "traffic": ncu_traffic("gemm_tc_kernel", name),
-                    "peak_source": f"{peak_kind} bf16 burst x 2 (int8)",
-                    "kernel": "bitlinear_forward (activation quant + tcgen05 int8 GEMM)",
-                    "algorithmic_ops": fw_ops, "ms_per_launch": fw_ms}
-    else:
-        achieved = fw_bytes / (fw_ms * 1e-3) / 1e9
-        roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                    "frac": achieved / hbm_peak, "traffic": None,
-                    "peak_source": f"{peak_kind} HBM copy", "kernel": "bitlinear_forward",
-                    "algorithmic_bytes": fw_bytes, "ms_per_launch": fw_ms}
-    roofline["others"] = others
-
+    fw_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs[:min(copies, args.steps)])
+    del graphs
     tokens = M * args.steps * world
     value = tokens / (elapsed_ms * 1e-3)
 
-    # end to end through the public API with host buffers (pinned), H2D + D2H timed
+    # end to end through the public API with host buffers (pinned): the batch goes up, the
+    # forward runs on the resident packed weights, the output comes back, every step
     e2e = None
     if not args.no_e2e:
-        W_h = Ws[0].cpu().pin_memory()
         x_h = xs[0].cpu().pin_memory()
         y_h = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
-        W_d = torch.empty_like(Ws[0])
         x_d = torch.empty_like(xs[0])
-        e2e_steps = max(3, min(args.steps, 50))
-        for _ in range(2):
-            W_d.copy_(W_h, non_blocking=True)
+        packed, gamma = ws_copies[0]
+        e2e_steps = max(3, min(args.steps, 20))
+
+        def e2e_step():
             x_d.copy_(x_h, non_blocking=True)
-            bl.quantize_weights(W_d, 1e-5, packed=packed, gamma=gamma, ws=ws)
-            bl.forward(x_d, packed, gamma, y=y, ws=ws)
+            bl.forward(x_d, packed, gamma, y=y, ws=work)
             y_h.copy_(y, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
         torch.cuda.synchronize()
         if dist is not None:
             dist.barrier()
@@ -362,39 +461,72 @@ def main():
         e2 = torch.cuda.Event(enable_timing=True)
         s2.record(stream)
         for _ in range(e2e_steps):
-            W_d.copy_(W_h, non_blocking=True)
-            x_d.copy_(x_h, non_blocking=True)
-            bl.quantize_weights(W_d, 1e-5, packed=packed, gamma=gamma, ws=ws)
-            bl.forward(x_d, packed, gamma, y=y, ws=ws)
-            y_h.copy_(y, non_blocking=True)
+            e2e_step()
         e2.record(stream)
         torch.cuda.synchronize()
         e_ms = bldist.max_over_ranks(s2.elapsed_time(e2), dist, device)
         e2e = {"value": M * e2e_steps * world / (e_ms * 1e-3), "unit": "tokens/s",
-               "h2d_bytes_per_step": W_h.numel() * 4 + x_h.numel() * x_h.element_size(),
-               "d2h_bytes_per_step": y_h.numel() * 2, "steps": e2e_steps}
+               "h2d_bytes_per_step": x_h.numel() * x_h.element_size(),
+               "d2h_bytes_per_step": y_h.numel() * y_h.element_size(), "steps": e2e_steps}
 
-    del graphs
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
     if rank != 0:
         return
+
+    # ------------------------------------------------------------------ roofline
+    path, splits = bl.debug_plan(M, N, K)
+    fw_ops = 2.0 * M * N * K
+    fw_bytes = N * K // 4 + M * K * 2 + M * N * 2
+    if path == "prefill":
+        # the activation quantization of the same batch timed alone, for the GEMM's share
+        xq_calls = [(lambda i=i: bl.quantize_acts(xs[i])) for i in range(min(copies, 4))]
+        xq_calls[0]()
+        aq_ms = statistics.mean(time_in_graph(xq_calls))
+        achieved = fw_ops / (fw_ms * 1e-3) / 1e12
+        roofline = {"bound": "tensor", "achieved": achieved, "peak": i8_peak, "unit": "TFLOP/s",
+                    "frac": achieved / i8_peak,
+                    "traffic": ncu_traffic("gemm_tc_kernel", name, M),
+                    "peak_source": f"{peak_kind} bf16 burst x 2 (int8 ops, nominal ratio)",
+                    "kernel": "bitlinear_forward = act_quant_kernel + gemm_tc_kernel "
+                              "(tcgen05 kind::i8)",
+                    "algorithmic_ops_per_launch": fw_ops, "ms_per_launch": fw_ms,
+                    "act_quant_ms": aq_ms, "gemm_ms_est": fw_ms - aq_ms,
+                    "gemm_frac_est": fw_ops / ((fw_ms - aq_ms) * 1e-3) / 1e12 / i8_peak}
+    else:
+        achieved = fw_bytes / (fw_ms * 1e-3) / 1e9
+        kern = "gemv_kernel" if path == "gemv" else "gemm_skinny_kernel"
+        roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                    "frac": achieved / hbm_peak, "traffic": ncu_traffic(kern, name, M),
+                    "peak_source": f"{peak_kind} HBM copy", "kernel": f"bitlinear_forward ({path})",
+                    "algorithmic_bytes_per_launch": fw_bytes, "ms_per_launch": fw_ms}
+
+    others = {}
+    if not args.no_others:
+        others["decode"] = [decode_figure(bl, n, m, device, hbm_peak, i8_peak)
+                            for n, m in [("70b_up_8192x28672", 1), ("70b_up_8192x28672", 16),
+                                         ("70b_up_8192x28672", 176),
+                                         ("70b_down_28672x8192", 1), ("70b_down_28672x8192", 16),
+                                         ("70b_down_28672x8192", 176),
+                                         ("700m_up_1536x4096", 1), ("700m_up_1536x4096", 4),
+                                         ("700m_up_1536x4096", 16)]]
+        others["weight_quant_70b"] = weight_quant_figures(bl, device, hbm_peak)
+    roofline["others"] = others
+
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(name, M)
-    launches_per_step = 1 + (1 if M <= 4 else 2)  # weight quant + (GEMV | act quant + GEMM)
+    config = config_of(name, M, wl, world)
+    config["inputs_vs_l2"] = (f"{copies} copies of packed W + x rotated "
+                              f"({copies * step_bytes / 2**20:.0f} MiB > 2 x L2), no flush")
     out = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "i8xternary->i32 (fp32 quantization, bf16 out)", "data": "synthetic",
-        "config": {"workload": name, "M": M, "N": N, "K": K, "w_dtype": "fp32",
-                   "x_dtype": str(wl["x_dtype"]).replace("torch.", ""), "out": "bf16",
-                   "inputs_vs_l2": f"{copies} weight copies x {w_bytes / 2**20:.1f} MiB rotated "
-                                   f"(> L2), no flush", "parallelism": f"replicas x{world}"},
+        "dtype": "i8xternary->i32 (bf16 in/out)", "data": "synthetic", "config": config,
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk.result(),
-        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches": forward_launches(bl, M, N, K) * args.steps,
     }
     print(json.dumps(out))
 

@@ -2,11 +2,11 @@
  * bitlinear.h - C ABI of the B200 (sm_100a) BitLinear forward library.
  *
  * What it computes: the BitLinear layer of BitNet b1.58 ("The Era of 1-bit LLMs: All
- * Large Language Models are in 1.58 Bits"). In the words of the dmarx anthology record
- * LIT-380 (Key takeaways, bullet 1), nn.Linear is replaced by BitLinear, the weights are
- * constrained to {-1, 0, +1} by an absmean quantization function and the activations are
- * 8-bit; bullet 4 says the matrix product becomes integer addition. The searcharxiv.com
- * abstract page (Abstract) states that every weight is ternary. The pages give no formula;
+ * Large Language Models are in 1.58 Bits"). Per the dmarx anthology record LIT-380 (Key
+ * takeaways, bullet 1), BitLinear takes the place of nn.Linear, an absmean quantization
+ * function limits the weights to {-1, 0, +1} and activations are held in 8 bits; bullet 4
+ * notes that the matrix product then needs only integer additions. The searcharxiv.com
+ * abstract page (Abstract) has every weight ternary. The pages give no formula;
  * the library implements the plainest reading:
  *
  *   gamma    = mean |W|                                    (fp32; exact sum, rounded once)
@@ -18,7 +18,7 @@
  *
  * Shapes follow nn.Linear: W [N][K] (out x in), x [M][K], y [M][N], all row-major.
  *
- * Packed weight format ("1.58 bit ... 2 bits in practice", hackerpaper HN page,
+ * Packed weight format (a 1.58-bit weight stored in 2 bits, hackerpaper HN page,
  * thread 17): trit c is stored as the 2-bit code u = c + 1 (0, 1, 2; 3 is never
  * written). Row n occupies K/4 bytes at byte offset n*K/4. The little-endian 32-bit word
  * g of a row holds trits k = 16g .. 16g+15; trit k = 16g + 4j + i (i, j in 0..3) is in
@@ -84,7 +84,7 @@ bl_status bitlinear_quantize_weights(const void* W, int w_dtype, int N, int K, f
                                      uint8_t* packed, float* gamma, void* ws,
                                      size_t ws_bytes, void* stream);
 
-/* Per-token absmax int8 activation quantization ("activations are 8-bit", LIT-380
+/* Per-token absmax int8 activation quantization (8-bit activations, LIT-380
  * bullet 1): q = clip(rne(x * (127 / a_t)), -127, 127), scale_t = a_t / 127.
  *   x      device, [M][K], fp32 or bf16 (x_dtype); read only.
  *   xq     device, [M][K] int8, written.
@@ -94,7 +94,7 @@ bl_status bitlinear_quantize_acts(const void* x, int x_dtype, int M, int K, int8
                                   float* scale, void* stream);
 
 /* The BitLinear forward: quantize x per token, contract with the packed ternary weights
- * in exact int32 ("integer addition", LIT-380 bullet 4) and rescale by s_t * gamma.
+ * in exact int32 (additions only, LIT-380 bullet 4) and rescale by s_t * gamma.
  *   x       device, [M][K], fp32 or bf16 (x_dtype).
  *   packed  device, [N][K/4] packed codes from bitlinear_quantize_weights.
  *   gamma   device, one float.
@@ -127,6 +127,11 @@ bl_status bitlinear_contract_i32(const int8_t* xq, const uint8_t* packed, int32_
  *   until the process exits). Small M needs none; otherwise M*K + 8*M bytes (each part
  *   rounded up to 256) must fit in 16 MiB, else BL_ERR_WORKSPACE is returned before
  *   anything is queued.
+ *   Kernels: the same CUDA-core GEMV as bitlinear_forward for the smallest M; up to 256
+ *   tokens the skinny tensor-core kernel with K never split across CTAs (bitlinear_forward
+ *   splits K on shapes with few weight tiles, so those shapes run slower here, e.g. 16
+ *   tokens on a 3200 x 8640 matrix); above 256 tokens the prefill GEMM. Same bits either
+ *   way.
  *   The first call on a device looks up the array's device address (cudaGetSymbolAddress)
  *   and caches it; make that first call before any stream capture.
  *   Every call on a device shares the one array: calls whose work overlaps on the GPU

@@ -6,22 +6,22 @@
 // file; only the tests, the smoke check and the benchmark's CPU-baseline leg do.
 // It shares no code, header, table or helper with the CUDA library.
 //
-// Sources (page, section):
-//  - "every single parameter (or weight) of the LLM is ternary {-1, 0, 1}":
+// Sources (page, section), restated:
+//  - every weight of the model takes one of the three values -1, 0, +1:
 //    searcharxiv.com abstract page, Abstract.
-//  - "nn.Linear is replaced by BitLinear; weights are constrained to {-1, 0, +1} by an
-//    absmean quantization function, activations are 8-bit": dmarx anthology record
-//    LIT-380, Key takeaways, bullet 1.
-//  - "Matrix multiplication becomes integer addition, with no multiplication at all":
-//    LIT-380, Key takeaways, bullet 4.
-//  - "1.58 bit LLM (2 bits in practice)": hackerpaper HN page, thread 17.
+//  - BitLinear takes the place of nn.Linear; an absmean quantization function limits
+//    the weights to {-1, 0, +1} and the activations are held in 8 bits: dmarx anthology
+//    record LIT-380, Key takeaways, bullet 1.
+//  - with ternary weights the matrix product needs only integer additions (and
+//    subtractions), no multiplications: LIT-380, Key takeaways, bullet 4.
+//  - a 1.58-bit weight is stored in 2 bits in practice: hackerpaper HN page, thread 17.
 // The pages print no formula. The formulas below are the plainest reading of
-// "absmean" and "8-bit activations": gamma = mean|W|, W~ = RoundClip(W/(gamma+eps), -1, 1),
+// absmean weights and 8-bit activations: gamma = mean|W|, W~ = RoundClip(W/(gamma+eps), -1, 1),
 // per-token absmax int8 in [-127, 127], int32 accumulation, rescale by gamma*absmax/127,
 // round-half-to-even everywhere. Every arithmetic step is fp32 IEEE round-to-nearest-even
 // with no contraction (build with -ffp-contract=off, no fast-math).
 //
-// Packed weight format (the library's 2-bit storage, "2 bits in practice"):
+// Packed weight format (the library's 2-bit storage of each trit):
 //  - each trit c in {-1,0,+1} is stored as the 2-bit unsigned code u = c + 1 (0,1,2; 3 is
 //    never written);
 //  - row n of W[N][K] occupies K/4 bytes starting at byte n*K/4 (K a multiple of 16);
@@ -204,7 +204,7 @@ int oracle_unpack(const uint8_t* packed, int64_t N, int64_t K, int8_t* codes) {
   return 0;
 }
 
-// Steps X1+X2: per-token absmax int8 quantization ("activations are 8-bit", LIT-380
+// Steps X1+X2: per-token absmax int8 quantization (8-bit activations, LIT-380
 // bullet 1). a_t = max_k |x[t,k]|; r_t = 127 / a_t (fp32); q = clip(rne(x * r_t), -127, 127);
 // s_t = a_t / 127 (fp32). A zero row gives q = 0 and s_t = 0; an exactly-zero element
 // gives q = 0. Returns 0, 1 if x holds Inf or NaN, 3 if the rounding mode is not nearest.
@@ -249,8 +249,8 @@ int oracle_quantize_acts(const void* x, int dtype, int64_t M, int64_t K, int8_t*
 }
 
 // Step C1: acc[t,n] = sum over k with c = +1 of q[t,k] minus sum over k with c = -1 of
-// q[t,k] ("integer addition, with no multiplication at all", LIT-380 bullet 4). Zero codes
-// are skipped ("feature filtering", LIT-380 bullet 2). codes is the unpacked [N][K] array.
+// q[t,k]: additions and subtractions only, no multiplication (LIT-380 bullet 4). Zero codes
+// are skipped, the feature filtering of LIT-380 bullet 2. codes is the unpacked [N][K] array.
 void oracle_contract_i32(const int8_t* q, const int8_t* codes, int64_t M, int64_t N,
                          int64_t K, int32_t* acc) {
   for (int64_t t = 0; t < M; ++t) {

@@ -1,4 +1,4 @@
-// Per-token absmax int8 activation quantization ("activations are 8-bit", dmarx anthology
+// Per-token absmax int8 activation quantization (8-bit activations, dmarx anthology
 // record LIT-380, Key takeaways bullet 1):
 //   a_t = max_k |x[t,k]|,  r_t = fl(127 / a_t),  s_t = fl(a_t / 127),
 //   q[t,k] = clip(rne(fl(x[t,k] * r_t)), -127, 127)   (0 when a_t == 0 or x == 0).

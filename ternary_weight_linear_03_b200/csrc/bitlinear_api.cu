@@ -16,6 +16,7 @@
 #include "gemm_skinny.cuh"
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
+#include "per_device.h"
 #include "weight_quant.cuh"
 
 namespace {
@@ -38,15 +39,33 @@ bool shape_ok(long long M, long long N, long long K) {
   return M * K < lim && N * K < lim && M * N < lim;
 }
 
+int current_device() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  return dev;
+}
+
+// Multiprocessors of the current device (148 on B200 if the query fails).
 int num_sms() {
-  static int sms = 0;
-  if (sms == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (sms <= 0) sms = 148;
-  }
-  return sms;
+  static bl::PerDevice cache;
+  const int v = cache.get(current_device(), [](int dev) {
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    return sms;
+  });
+  return v > 0 ? v : 148;
+}
+
+// Raises `kern`'s dynamic shared-memory limit to `bytes` on the current device, once per
+// device (the attribute belongs to that device's context). False if the call failed.
+template <class Kernel>
+bool set_smem_limit_once(bl::PerDevice& cache, Kernel kern, int bytes) {
+  return cache.get(current_device(), [&](int) {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ==
+                   cudaSuccess
+               ? 1
+               : 0;
+  }) > 0;
 }
 
 // The CUDA-core GEMV for one or two tokens, and for up to kGemvMaxM tokens when the packed
@@ -184,14 +203,9 @@ bl_status launch_gemv_t(const void* x, const uint8_t* packed, const float* gamma
                         int N, int K, cudaStream_t s) {
   auto kern = bl::gemv_kernel<MT, XM, OM, XR, R>;
   const int smem = MT * K;
-  static int configured_smem = -1;
-  static int blocks_per_sm = 1;
-  if (configured_smem < smem) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemvMaxSmem) !=
-        cudaSuccess)
-      return BL_ERR_CUDA;
-    configured_smem = smem;
-  }
+  static bl::PerDevice configured;
+  if (!set_smem_limit_once(configured, kern, kGemvMaxSmem)) return BL_ERR_CUDA;
+  int blocks_per_sm = 1;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_per_sm, kern, bl::kGemvThreads,
                                                     smem) != cudaSuccess ||
       blocks_per_sm < 1)
@@ -261,13 +275,8 @@ bl_status launch_gemm_t(const int8_t* xq, const uint8_t* packed, const int* rows
   if (!make_map_u8(&map_b, packed, K / 4, N, K / 4, bl::tc::BK / 4, bl::tc::BN, false))
     return BL_ERR_CUDA;
   auto kern = bl::gemm_tc_kernel<OM>;
-  static bool configured = false;
-  if (!configured) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             bl::tc::SMEM_BYTES) != cudaSuccess)
-      return BL_ERR_CUDA;
-    configured = true;
-  }
+  static bl::PerDevice configured;
+  if (!set_smem_limit_once(configured, kern, bl::tc::SMEM_BYTES)) return BL_ERR_CUDA;
   const long long tiles = static_cast<long long>((M + bl::tc::BM - 1) / bl::tc::BM) *
                           ((N + bl::tc::BN - 1) / bl::tc::BN);
   const int grid = static_cast<int>(std::min<long long>(tiles, num_sms()));
@@ -297,15 +306,10 @@ bl_status launch_skinny_t(const int8_t* xq, const uint8_t* packed, const int* ro
                    true))
     return BL_ERR_CUDA;
   auto kern = bl::gemm_skinny_kernel<OM>;
-  static bool configured = false;
-  if (!configured) {
-    int most = 0;
-    for (int b = 16; b <= bl::sk::BW * 2; b += 16) most = std::max(most, bl::sk::smem_bytes(b));
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, most) !=
-        cudaSuccess)
-      return BL_ERR_CUDA;
-    configured = true;
-  }
+  static bl::PerDevice configured;
+  int most = 0;
+  for (int b = 16; b <= bl::sk::BW * 2; b += 16) most = std::max(most, bl::sk::smem_bytes(b));
+  if (!set_smem_limit_once(configured, kern, most)) return BL_ERR_CUDA;
   // Programmatic dependent launch: the kernel may start while the quantization kernel before
   // it (which also zeroed the split-K sums and counters) is still running; it loads W and
   // sets up TMEM meanwhile and waits for that grid before touching its outputs.
@@ -337,17 +341,34 @@ void skinny_zero_region(void* ws, int M, int N, int K, uint4** z, long long* n16
   *n16 = (p.splits > 1) ? static_cast<long long>((w.bytes - head) / 16) : 0;
 }
 
-bl_status launch_skinny(const int8_t* xq, const uint8_t* packed, const int* rowsum,
-                        const float* scale, const float* gamma, void* y, int y_dtype, int M,
-                        int N, int K, void* ws, cudaStream_t s) {
-  const SkinnyPlan p = skinny_plan(M, N, K);
-  const SkinnyWs w = skinny_ws_layout(ws, M, N, K, p);
+bl_status launch_skinny_plan(const int8_t* xq, const uint8_t* packed, const int* rowsum,
+                             const float* scale, const float* gamma, void* y, int y_dtype,
+                             int M, int N, int K, const SkinnyPlan& p, const SkinnyWs& w,
+                             cudaStream_t s) {
   switch (y_dtype) {
     case BL_F32: return launch_skinny_t<0>(xq, packed, rowsum, scale, gamma, y, M, N, K, p, w, s);
     case BL_BF16: return launch_skinny_t<1>(xq, packed, rowsum, scale, gamma, y, M, N, K, p, w, s);
     case BL_I32: return launch_skinny_t<2>(xq, packed, rowsum, scale, gamma, y, M, N, K, p, w, s);
     default: return BL_ERR_INVALID_ARG;
   }
+}
+
+bl_status launch_skinny(const int8_t* xq, const uint8_t* packed, const int* rowsum,
+                        const float* scale, const float* gamma, void* y, int y_dtype, int M,
+                        int N, int K, void* ws, cudaStream_t s) {
+  const SkinnyPlan p = skinny_plan(M, N, K);
+  const SkinnyWs w = skinny_ws_layout(ws, M, N, K, p);
+  return launch_skinny_plan(xq, packed, rowsum, scale, gamma, y, y_dtype, M, N, K, p, w, s);
+}
+
+// The skinny plan with K left unsplit: one CTA per weight tile, so the kernel needs no
+// split-K sums or counters (only the staged activations).
+SkinnyPlan skinny_plan_unsplit(int M, int N, int K) {
+  SkinnyPlan p = skinny_plan(M, N, K);
+  const int KB = (K + bl::sk::BK - 1) / bl::sk::BK;
+  p.splits = 1;
+  p.kbps = (KB + bl::sk::KPS - 1) / bl::sk::KPS * bl::sk::KPS;
+  return p;
 }
 
 // Workspace bytes the forward / contract paths need for (M, N, K).
@@ -379,15 +400,19 @@ bl_status launch_weight_quant_t(const void* W, long long n, float eps, void* ws,
                                 cudaStream_t s) {
   auto kern = bl::weight_quant_kernel<kBf16>;
   constexpr int kSmem = bl::kWqStages * bl::kWqStageBytes;
-  static int blocks_per_sm = 0;
-  if (blocks_per_sm == 0) {
+  // blocks of this kernel resident per SM, found once per device after raising its
+  // shared-memory limit (a cooperative launch needs every block resident)
+  static bl::PerDevice occupancy;
+  const int blocks_per_sm = occupancy.get(current_device(), [&](int) {
+    int b = 0;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) !=
             cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_per_sm, kern, bl::kWqThreads,
-                                                      kSmem) != cudaSuccess ||
-        blocks_per_sm < 1)
-      return BL_ERR_CUDA;
-  }
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kern, bl::kWqThreads, kSmem) !=
+            cudaSuccess)
+      return 0;
+    return b;
+  });
+  if (blocks_per_sm < 1) return BL_ERR_CUDA;
   // one block per 32 KB of weights at least, at most all resident blocks
   const long long want = (n * (kBf16 ? 2 : 4) + 32767) / 32768;
   const int grid = static_cast<int>(
@@ -551,8 +576,10 @@ bl_status bitlinear_get_device_status(void* stream) {
 }
 
 // Same computation as bitlinear_forward, for callers that cannot allocate device memory:
-// the staging buffers of the tensor-core path live in g_noalloc_scratch instead of a
-// caller-supplied workspace. Nothing in the scratch has to start at zero (each call
+// the staging buffers of the tensor-core paths live in g_noalloc_scratch instead of a
+// caller-supplied workspace. Kernel choice: the GEMV where bitlinear_forward uses it, the
+// skinny tensor-core kernel with K unsplit up to 256 tokens (bitlinear_forward may split K
+// there, which needs int32 sums this scratch does not hold), the prefill GEMM above. Nothing in the scratch has to start at zero (each call
 // writes every byte it later reads). No cudaMalloc, cudaFree or allocating library call
 // is made. Calls that overlap on the GPU (other streams, other host threads) race on the
 // shared scratch; callers serialize them.
@@ -578,6 +605,11 @@ bl_status bitlinear_forward_noalloc(const void* x, int x_dtype, const uint8_t* p
   FwdWs w = fwd_ws_layout(scratch, M, K);
   st = launch_act_quant(x, x_dtype, M, K, w.xq, w.scale, w.rowsum, s);
   if (st != BL_OK) return st;
+  if (M <= kSkinnyMaxM) {
+    SkinnyWs none{};
+    return launch_skinny_plan(w.xq, packed, w.rowsum, w.scale, gamma, y, y_dtype, M, N, K,
+                              skinny_plan_unsplit(M, N, K), none, s);
+  }
   return launch_gemm(w.xq, packed, w.rowsum, w.scale, gamma, y, y_dtype, M, N, K, s);
 }
 

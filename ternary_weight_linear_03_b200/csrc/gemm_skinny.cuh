@@ -3,7 +3,7 @@
 //   D[n][t] = sum_k u[n][k] * xq[t][k]     (A = 128 unpacked weight rows, B = the M tokens)
 // so the weights fill the MMA's 128-row slot and the few tokens its N slot (16..256), and
 // every weight tile is unpacked once no matter how many tokens there are. This is the
-// integer "addition" of BitNet b1.58 (dmarx anthology record LIT-380, Key takeaways
+// addition-only integer product of BitNet b1.58 (dmarx anthology record LIT-380, Key takeaways
 // bullet 4) in the same u = c + 1 form as the other kernels (acc = D - rowsum_t).
 //
 // Data path:

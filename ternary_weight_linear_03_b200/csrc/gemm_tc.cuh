@@ -4,7 +4,7 @@
 //   D[m][n] = sum_k xq[m][k] * u[n][k]          (tcgen05.mma kind::i8, int32 in TMEM)
 //   acc     = D - rowsum_m                       (u = c + 1, so sum_k u q = acc + sum_k q)
 //   y       = float(acc) * (scale_m * gamma)     (epilogue, fp32 or bf16)
-// which is exactly the integer "addition" of BitNet b1.58 (dmarx anthology record
+// which is exactly the addition-only integer product of BitNet b1.58 (dmarx anthology record
 // LIT-380, Key takeaways bullet 4) evaluated by the tensor core.
 //
 // One persistent CTA per SM, 10 warps, warp-specialized:

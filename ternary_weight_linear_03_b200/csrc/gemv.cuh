@@ -1,7 +1,7 @@
 // Decode BitLinear (small M): one CUDA-core kernel that quantizes the M tokens in its
 // prologue and then streams the packed ternary weights once from HBM.
 //
-// The contraction is the "integer addition" of BitNet b1.58 (dmarx anthology record
+// The contraction is the addition-only integer product of BitNet b1.58 (dmarx anthology record
 // LIT-380, Key takeaways bullet 4). Weights are stored as u = c + 1 in {0, 1, 2}, so
 //   acc[t,n] = sum_k c[n,k] q[t,k] = sum_k u[n,k] q[t,k] - rowsum_t,
 // and one packed 32-bit word (16 trits) unpacks to four int8x4 registers with one shift

@@ -18,24 +18,29 @@ import math
 import torch
 
 
-def gen(seed: int) -> torch.Generator:
-    g = torch.Generator(device="cpu")
+def gen(seed: int, device="cpu") -> torch.Generator:
+    g = torch.Generator(device=device)
     g.manual_seed(int(seed))
     return g
 
 
-def weights(N: int, K: int, sigma: float, seed: int, dtype=torch.float32) -> torch.Tensor:
-    w = torch.randn((N, K), generator=gen(seed), dtype=torch.float32) * sigma
+def weights(N: int, K: int, sigma: float, seed: int, dtype=torch.float32,
+            device="cpu") -> torch.Tensor:
+    """N x K weights ~ N(0, sigma^2). device="cpu" is the reference recipe (CPU generator,
+    what the parity tests use); a CUDA device draws the same distribution with that
+    device's seeded generator (other values, far faster for the large benchmark sets)."""
+    w = torch.randn((N, K), generator=gen(seed, device), dtype=torch.float32, device=device)
+    w.mul_(sigma)
     return w.to(dtype)
 
 
 def activations(M: int, K: int, seed: int, dtype=torch.bfloat16, outlier_frac: float = 0.0,
-                outlier_gain: float = 20.0) -> torch.Tensor:
-    g = gen(seed)
-    x = torch.randn((M, K), generator=g, dtype=torch.float32)
+                outlier_gain: float = 20.0, device="cpu") -> torch.Tensor:
+    g = gen(seed, device)
+    x = torch.randn((M, K), generator=g, dtype=torch.float32, device=device)
     if outlier_frac > 0.0:
         n_out = int(math.ceil(outlier_frac * K))
-        cols = torch.randperm(K, generator=g)[:n_out]
+        cols = torch.randperm(K, generator=g, device=device)[:n_out]
         x[:, cols] *= outlier_gain
     return x.to(dtype)
 

@@ -28,7 +28,7 @@ def test_reference_arm_prints_one_contract_line():
                 "cpu_baseline", "e2e"):
         assert key in d, key
     assert d["value"] > 0 and d["unit"] == "tokens/s" and d["higher_is_better"] is True
-    assert d["config"]["workload"] == "700m_up_1536x4096" and d["config"]["M"] == 16
+    assert d["config"]["workload"] == "70b_prefill_4096x8192x28672" and d["config"]["M"] == 4096
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}

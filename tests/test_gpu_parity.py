@@ -5,7 +5,9 @@ bit-exactly; fp32 outputs within 1e-6 relative error and bf16 outputs within 1 u
 practice both are bit-identical, because both sides fix the same fp32 operation order).
 """
 
+import json
 import math
+import os
 
 import numpy as np
 import pytest
@@ -59,6 +61,9 @@ def assert_bf16_within_1ulp(got_bits: np.ndarray, ref_bits: np.ndarray):
 @pytest.mark.parametrize("N,K,dtype", [
     (256, 256, torch.float32), (293, 192, torch.float32), (4096, 1536, torch.float32),
     (300, 8640, torch.bfloat16), (8, 64, torch.bfloat16), (1, 64, torch.float32),
+    # more than 64 KB of W per block (the ring of four 16 KB stages): the second pass
+    # streams the block's range again instead of reading it from shared memory
+    (1024, 8192, torch.float32), (2048, 8192, torch.bfloat16), (1111, 8256, torch.float32),
 ])
 def test_quantize_weights_bit_exact(N, K, dtype):
     W = syn.weights(N, K, 0.02, seed=N * 7 + K, dtype=dtype)
@@ -93,8 +98,8 @@ def test_quantize_weights_exact_sum_edge_cases(kind):
 
 
 def test_quantize_weights_rows_of_very_different_scale():
-    """Row blocks whose scale differs 100x: the per-block gamma guesses miss the final
-    threshold for many blocks, which then re-read their range. Codes stay exact."""
+    """Row blocks whose scale differs 100x, so the blocks' own shares of the sum of |w|
+    differ by as much: gamma still comes out exact and every code with it."""
     N, K = 2048, 1536
     W = syn.weights(N, K, 1.0, seed=77)
     scale = torch.where((torch.arange(N) // 64) % 2 == 0, 0.001, 0.1)
@@ -107,8 +112,9 @@ def test_quantize_weights_rows_of_very_different_scale():
 
 @pytest.mark.parametrize("ws_kind", ["full", "tiny"])
 def test_quantize_weights_many_ambiguous(ws_kind):
-    """Half of the weights sit within 1% of gamma/2: far more ambiguous entries than the
-    lists hold (always with the tiny workspace), so blocks fall back to a re-read."""
+    """Half of the weights sit within 1% of (gamma + eps)/2, right at the threshold between
+    0 and +-1, so a threshold off by one float would flip codes; also with the smallest
+    workspace the call accepts."""
     rng = np.random.default_rng(5)
     N, K = 512, 2048
     mag = np.where(rng.random(N * K) < 0.5, 0.5 * (1 + 0.01 * rng.uniform(-1, 1, N * K)), 1.5)
@@ -248,6 +254,21 @@ def test_forward_paths_agree_at_the_switch(m_small, m_big, N, K):
 # ----------------------------------------------------------------------------- full sizes
 
 
+def oracle_forward_parallel(x_in, packed: np.ndarray, gamma: float, out: str):
+    """The oracle's forward over every weight row, the rows cut into contiguous ranges run
+    on one host thread each (the oracle itself stays single-threaded; ctypes releases the
+    interpreter lock). Returns [M][N] and the thread count."""
+    from concurrent.futures import ThreadPoolExecutor
+    threads = max(1, min(os.cpu_count() or 1, 32))
+    edges = np.linspace(0, packed.shape[0], threads + 1).astype(int)
+    ranges = [(a, b) for a, b in zip(edges[:-1], edges[1:]) if b > a]
+    with ThreadPoolExecutor(len(ranges)) as ex:
+        parts = list(ex.map(
+            lambda r: orc.forward(x_in, np.ascontiguousarray(packed[r[0]:r[1]]), gamma, out=out),
+            ranges))
+    return np.concatenate(parts, axis=1), len(ranges)
+
+
 FULL = [
     ("700m_up_1536x4096", 16), ("3b_gate_up_3200x8640", 64), ("3b_down_8640x3200", 1),
     ("70b_up_8192x28672", 176), ("70b_down_28672x8192", 16),
@@ -255,24 +276,75 @@ FULL = [
 
 
 @pytest.mark.parametrize("name,M", FULL)
-def test_full_size_sampled_rows(name, M):
-    """Full-size matrices: gamma and every packed byte exactly, outputs on sampled rows."""
+def test_full_size_every_packed_byte(name, M):
+    """Full-size matrices: gamma and every packed byte against the oracle (the 3B and 70B
+    ones take the second pass's streaming branch), then the forward on sampled rows."""
     wl = syn.WORKLOADS[name]
     N, K = wl["N"], wl["K"]
     W = syn.weights(N, K, wl["sigma"], seed=syn.w_seed(name))
     x = syn.activations(M, K, seed=syn.x_seed(name, M), dtype=wl["x_dtype"],
                         outlier_frac=wl["outlier_frac"])
     packed, gamma = bl.quantize_weights(W.cuda())
-    assert gamma.item() == float(orc.absmean(W.numpy()))
-    rows = np.random.default_rng(0).choice(N, size=min(N, 96), replace=False)
-    rows.sort()
-    ref_packed_rows, _ = None, None
-    codes = orc.ternarize(np.ascontiguousarray(W.numpy()[rows]), gamma.item(), 1e-5)
-    np.testing.assert_array_equal(packed.cpu().numpy()[rows], orc.pack(codes))
+    ref_gamma = orc.absmean(W.numpy())
+    assert gamma.item() == float(ref_gamma)
+    ref_packed = orc.pack(orc.ternarize(W.numpy(), ref_gamma, 1e-5))
+    got_packed = packed.cpu().numpy()
+    np.testing.assert_array_equal(got_packed, ref_packed)
+    rows = np.sort(np.random.default_rng(0).choice(N, size=min(N, 96), replace=False))
     y = bl.forward(x.cuda(), packed, gamma, out_dtype=torch.bfloat16)
-    ref = orc.forward(_np_in(x), orc.pack(codes), gamma.item(), out="bf16")
+    ref = orc.forward(_np_in(x), np.ascontiguousarray(ref_packed[rows]), ref_gamma, out="bf16")
     got = y.cpu().view(torch.int16).numpy().view(np.uint16)[:, rows]
     np.testing.assert_array_equal(got, ref)
+
+
+@pytest.mark.parametrize("N,K", [(8192, 8192), (1024, 8192)])
+def test_70b_layer_shapes_every_packed_byte(N, K):
+    """The other 70B-shaped layer matrices the weight quantization serves (attention
+    projections): gamma and every packed byte."""
+    W = syn.weights(N, K, 0.015, seed=5000 + N)
+    packed, gamma = bl.quantize_weights(W.cuda())
+    ref_packed, ref_gamma = orc.quantize_weights(W.numpy(), 1e-5)
+    assert gamma.item() == float(ref_gamma)
+    np.testing.assert_array_equal(packed.cpu().numpy(), ref_packed)
+
+
+@pytest.mark.parametrize("name,M", [("70b_up_8192x28672", 16), ("70b_down_28672x8192", 16)])
+def test_70b_decode_forward_every_output(name, M):
+    """One 70B decode forward (M = 16, the skinny tensor-core kernel), every one of its
+    M x N bf16 outputs against the oracle, the oracle run over disjoint row ranges on the
+    host's cores."""
+    wl = syn.WORKLOADS[name]
+    N, K = wl["N"], wl["K"]
+    W = syn.weights(N, K, wl["sigma"], seed=syn.w_seed(name))
+    x = syn.activations(M, K, seed=syn.x_seed(name, M), dtype=wl["x_dtype"])
+    packed, gamma = bl.quantize_weights(W.cuda())
+    y = bl.forward(x.cuda(), packed, gamma, out_dtype=torch.bfloat16)
+    ref, threads = oracle_forward_parallel(_np_in(x), packed.cpu().numpy(), gamma.item(), "bf16")
+    got = y.cpu().view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(got, ref)
+    assert threads >= 1
+
+
+@pytest.mark.parametrize("fixture", ["hand_worked_2x16.json", "hand_worked_eps_scale_2x16.json"])
+def test_hand_worked_examples_on_device(fixture):
+    """The hand-worked examples (tests/golden/) through the library: gamma, packed bytes
+    and the fp32 outputs, bit for bit."""
+    with open(os.path.join(os.path.dirname(__file__), "golden", fixture)) as f:
+        d = json.load(f)
+    W = torch.tensor(d["W"], dtype=torch.float32)
+    # The library needs K % 64 == 0: the 16 columns are padded to 64 with weights equal to
+    # gamma (so the mean of |W| over all 128 entries is still exactly gamma, the codes of
+    # the real weights unchanged) facing zero activations (absmax and acc unchanged).
+    K0 = W.shape[1]
+    Wp = torch.full((W.shape[0], 64), d["gamma"], dtype=torch.float32)
+    Wp[:, :K0] = W
+    x = torch.zeros((1, 64))
+    x[:, :K0] = torch.tensor(d["x"], dtype=torch.float32)
+    packed, gamma = bl.quantize_weights(Wp.cuda(), eps=d["eps"])
+    assert gamma.item() == d["gamma"]
+    np.testing.assert_array_equal(packed.cpu().numpy()[:, :K0 // 4], np.array(d["packed"], np.uint8))
+    y = bl.forward(x.cuda(), packed, gamma, out_dtype=torch.float32)
+    np.testing.assert_array_equal(y.cpu().numpy(), np.array(d["y"], np.float32))
 
 
 def test_prefill_shape_sampled_rows():

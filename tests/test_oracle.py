@@ -24,9 +24,12 @@ def _fsum_gamma(w: np.ndarray) -> np.float32:
 # ----------------------------------------------------------------------------- golden
 
 
-def test_hand_worked_example():
-    """Every stage of the hand-worked 2x16 example (tests/golden/hand_worked_2x16.json)."""
-    with open(os.path.join(GOLDEN, "hand_worked_2x16.json")) as f:
+@pytest.mark.parametrize("fixture", ["hand_worked_2x16.json", "hand_worked_eps_scale_2x16.json"])
+def test_hand_worked_example(fixture):
+    """Every stage of a hand-worked 2x16 example (tests/golden/): the first with eps = 0
+    and unit scale, the second with eps > 0 and a scale that is not a power of two, where
+    the rescale's operation order and its use of gamma (not gamma + eps) show in the bits."""
+    with open(os.path.join(GOLDEN, fixture)) as f:
         d = json.load(f)
     W = np.array(d["W"], np.float32)
     x = np.array(d["x"], np.float32)
@@ -43,6 +46,9 @@ def test_hand_worked_example():
     np.testing.assert_array_equal(acc, np.array(d["acc"], np.int32))
     y = orc.forward(x, packed, gamma)
     np.testing.assert_array_equal(y, np.array(d["y"], np.float32))
+    for wrong in ("y_wrong_order", "y_rescaled_by_gamma_plus_eps"):
+        if wrong in d:  # the fixture's alternatives really differ from the answer
+            assert np.all(np.array(d[wrong], np.float32) != y), wrong
 
 
 # ----------------------------------------------------------------------------- absmean

@@ -42,8 +42,10 @@ def _call_forward(lib, x, packed, gamma, y, ws, M, N, K):
 
 def test_noalloc_matches_forward_on_two_calls_in_a_row():
     lib = bl.load_library()
-    cases = [(200, 1000, 1536, torch.bfloat16, torch.float32),   # tensor-core path
-             (64, 4096, 3200, torch.float32, torch.bfloat16)]    # second call, other shape
+    cases = [(200, 1000, 1536, torch.bfloat16, torch.float32),   # skinny tensor-core kernel
+             (64, 4096, 3200, torch.float32, torch.bfloat16),    # second call, other shape
+             (16, 8640, 3200, torch.bfloat16, torch.bfloat16),   # bitlinear_forward splits K
+             (300, 520, 1536, torch.bfloat16, torch.float32)]    # prefill GEMM
     for i, (M, N, K, xdt, ydt) in enumerate(cases):
         W = syn.weights(N, K, 0.02, seed=300 + i).cuda()
         x = syn.activations(M, K, seed=400 + i, dtype=xdt, outlier_frac=0.01).cuda()
