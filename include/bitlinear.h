@@ -84,6 +84,38 @@ bl_status bitlinear_quantize_weights(const void* W, int w_dtype, int N, int K, f
                                      uint8_t* packed, float* gamma, void* ws,
                                      size_t ws_bytes, void* stream);
 
+/* Words of the exact sum of |w| that bitlinear_weight_abssum writes. */
+#define BL_ABSSUM_WORDS 14
+
+/* Tensor parallelism, step 1 of 2 of the absmean weight quantization of a matrix split
+ * over several GPUs (rows for a column-parallel layer, columns for a row-parallel one):
+ * gamma is the mean of |w| over the WHOLE matrix (LIT-380 bullet 1; one scale per weight
+ * tensor), so each GPU first forms the exact sum of |w| over its own shard.
+ *   W     device, the shard [N][K] row-major (its own contiguous copy), fp32 or bf16.
+ *   sums  device, BL_ABSSUM_WORDS uint64, written: the exact sum S of |w| over the shard
+ *         as S * 2^149 = sum_j sums[j] * 2^(32 j) (columns not carried, each below 2^57).
+ *         The words of several shards add up exactly (plain uint64 addition, e.g. an
+ *         NCCL sum all-reduce) to the words of their union.
+ *   ws    device workspace of at least bitlinear_workspace_size(1, N, K) bytes.
+ * Inf/NaN in W sets BL_ERR_NONFINITE in the device status word. */
+bl_status bitlinear_weight_abssum(const void* W, int w_dtype, int N, int K, uint64_t* sums,
+                                  void* ws, size_t ws_bytes, void* stream);
+
+/* Tensor parallelism, step 2 of 2: gamma = (S rounded once to double) / n_total rounded to
+ * float, from the added words of every shard, then the codes of THIS shard's weights,
+ * RoundClip(w / (gamma + eps), -1, 1), 2-bit packed as bitlinear_quantize_weights does.
+ * With every shard's words added, gamma and the codes are bit for bit those of
+ * bitlinear_quantize_weights on the whole matrix.
+ *   W        device, the shard [N][K] (the one given to step 1).
+ *   n_total  number of weights of the whole matrix (>= N * K).
+ *   sums     device, BL_ABSSUM_WORDS uint64: the words of all shards, added.
+ *   packed   device, N*K/4 bytes; gamma device, one float; both written.
+ * Non-finite weights are reported by step 1, not here. */
+bl_status bitlinear_quantize_weights_from_abssum(const void* W, int w_dtype, int N, int K,
+                                                 long long n_total, const uint64_t* sums,
+                                                 float eps, uint8_t* packed, float* gamma,
+                                                 void* stream);
+
 /* Per-token absmax int8 activation quantization (8-bit activations, LIT-380
  * bullet 1): q = clip(rne(x * (127 / a_t)), -127, 127), scale_t = a_t / 127.
  *   x      device, [M][K], fp32 or bf16 (x_dtype); read only.
@@ -92,6 +124,33 @@ bl_status bitlinear_quantize_weights(const void* W, int w_dtype, int N, int K, f
  * Inf/NaN in x sets BL_ERR_NONFINITE in the device status word. */
 bl_status bitlinear_quantize_acts(const void* x, int x_dtype, int M, int K, int8_t* xq,
                                   float* scale, void* stream);
+
+/* Per-token absolute maximum a_t = max_k |x[t,k]| (the first half of the activation
+ * quantization). Under tensor parallelism with K split, each GPU holds a K-shard of every
+ * token row; the MAX all-reduce of these per-shard values is the row's a_t.
+ *   x     device, [M][K] fp32 or bf16.   amax  device, [M] fp32, written.
+ * Inf/NaN in x sets BL_ERR_NONFINITE in the device status word. */
+bl_status bitlinear_act_absmax(const void* x, int x_dtype, int M, int K, float* amax,
+                               void* stream);
+
+/* The activation quantization with a_t given: q = clip(rne(x * fl(127 / a_t)), -127, 127),
+ * scale_t = fl(a_t / 127), exactly as bitlinear_quantize_acts computes them when a_t is
+ * the row's own absmax. For a K-shard of the rows, pass the absmax of the whole rows.
+ *   x      device, [M][K].   amax   device, [M] fp32 (a_t >= 0; values of x above a_t
+ *   clip to +-127).   xq     device, [M][K] int8, written.   scale  device, [M], written. */
+bl_status bitlinear_quantize_acts_absmax(const void* x, int x_dtype, int M, int K,
+                                         const float* amax, int8_t* xq, float* scale,
+                                         void* stream);
+
+/* The rescale on its own: y[t,n] = fl(float(acc[t,n]) * fl(scale_t * gamma)) (fp32, or the
+ * bf16 RNE of that value), for an int32 product formed elsewhere, e.g. the SUM
+ * all-reduce of per-GPU partial products of bitlinear_contract_i32 under a K split (an
+ * exact integer sum, so the result equals the single-GPU forward bit for bit).
+ *   acc    device, [M][N] int32.   scale  device, [M].   gamma  device, one float.
+ *   y      device, [M][N], y_dtype BL_F32 or BL_BF16, written.
+ * M, N >= 1 and M*N below 2^31, else BL_ERR_UNSUPPORTED_SHAPE. */
+bl_status bitlinear_rescale(const int32_t* acc, const float* scale, const float* gamma,
+                            void* y, int y_dtype, int M, int N, void* stream);
 
 /* The BitLinear forward: quantize x per token, contract with the packed ternary weights
  * in exact int32 (additions only, LIT-380 bullet 4) and rescale by s_t * gamma.

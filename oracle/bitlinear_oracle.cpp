@@ -35,6 +35,7 @@
 #include <cstring>
 #include <cfenv>
 #include <cmath>
+#include <vector>
 
 namespace {
 
@@ -72,9 +73,13 @@ extern "C" {
 // m < 2^24. Bucket B[e] accumulates the integer mantissas of exponent e (uint64 is enough
 // for n <= 2^31). The exact sum S * 2^149 = sum_e B[e] * 2^(max(e,1) - 1) is built in a
 // multi-word integer, rounded once to double (round half to even), divided by n in double
-// and rounded to float. Returns 0 on success, 1 if any |w| is Inf or NaN.
-int oracle_absmean(const void* W, int dtype, int64_t n, float* gamma_out) {
-  uint64_t bucket[256];
+// and rounded to float. The two halves are separate functions so that the buckets of the
+// parts of a matrix split over several devices can be added (integers) before gamma is
+// formed once for the whole matrix.
+
+// First half: the 256 exponent buckets of the n values (bucket[0] stays 0; subnormals go
+// to bucket[1]). Returns 0, or 1 if any |w| is Inf or NaN.
+int oracle_abs_buckets(const void* W, int dtype, int64_t n, uint64_t* bucket) {
   for (int e = 0; e < 256; ++e) bucket[e] = 0;
   for (int64_t i = 0; i < n; ++i) {
     uint32_t bits = float_bits(load_value(W, dtype, i)) & 0x7fffffffu;
@@ -84,6 +89,11 @@ int oracle_absmean(const void* W, int dtype, int64_t n, float* gamma_out) {
     if (e != 0u) m |= 0x800000u;
     bucket[e == 0u ? 1u : e] += m;  // subnormals share the unit 2^-149 with e = 1
   }
+  return 0;
+}
+
+// Second half: gamma from the buckets of n values in all.
+void oracle_absmean_from_buckets(const uint64_t* bucket, int64_t n, float* gamma_out) {
 
   // Exact integer S * 2^149 as little-endian 32-bit words (512 bits is plenty:
   // the largest term is < 2^55 * 2^253).
@@ -141,6 +151,13 @@ int oracle_absmean(const void* W, int dtype, int64_t n, float* gamma_out) {
   }
   double mean = sum / static_cast<double>(n);
   *gamma_out = static_cast<float>(mean);
+}
+
+// gamma = mean |W| over the n values: both halves. Returns 0, or 1 for Inf/NaN.
+int oracle_absmean(const void* W, int dtype, int64_t n, float* gamma_out) {
+  uint64_t bucket[256];
+  if (oracle_abs_buckets(W, dtype, n, bucket) != 0) return 1;
+  oracle_absmean_from_buckets(bucket, n, gamma_out);
   return 0;
 }
 
@@ -208,9 +225,12 @@ int oracle_unpack(const uint8_t* packed, int64_t N, int64_t K, int8_t* codes) {
 // bullet 1). a_t = max_k |x[t,k]|; r_t = 127 / a_t (fp32); q = clip(rne(x * r_t), -127, 127);
 // s_t = a_t / 127 (fp32). A zero row gives q = 0 and s_t = 0; an exactly-zero element
 // gives q = 0. Returns 0, 1 if x holds Inf or NaN, 3 if the rounding mode is not nearest.
-int oracle_quantize_acts(const void* x, int dtype, int64_t M, int64_t K, int8_t* q,
-                         float* scale) {
-  if (!rounding_mode_is_nearest()) return 3;
+//
+// Split in two steps (X1, then X2 given a_t) so that a row held in K-shards on several
+// devices can form a_t as the maximum of the shards' maxima first.
+
+// X1 alone: amax[t] = max_k |x[t,k]|. Returns 0, or 1 if x holds Inf or NaN.
+int oracle_act_absmax(const void* x, int dtype, int64_t M, int64_t K, float* amax) {
   for (int64_t t = 0; t < M; ++t) {
     float a = 0.0f;
     for (int64_t k = 0; k < K; ++k) {
@@ -218,6 +238,18 @@ int oracle_quantize_acts(const void* x, int dtype, int64_t M, int64_t K, int8_t*
       if (!(v <= 3.4028234663852886e38f)) return 1;  // Inf or NaN
       if (v > a) a = v;
     }
+    amax[t] = a;
+  }
+  return 0;
+}
+
+// X2 with a_t given (a_t >= 0 and finite; values above a_t clip to +-127).
+// Returns 0, or 3 if the rounding mode is not nearest.
+int oracle_quantize_acts_absmax(const void* x, int dtype, int64_t M, int64_t K,
+                                const float* amax, int8_t* q, float* scale) {
+  if (!rounding_mode_is_nearest()) return 3;
+  for (int64_t t = 0; t < M; ++t) {
+    const float a = amax[t];
     if (a == 0.0f) {
       for (int64_t k = 0; k < K; ++k) q[t * K + k] = 0;
       scale[t] = 0.0f;
@@ -246,6 +278,15 @@ int oracle_quantize_acts(const void* x, int dtype, int64_t M, int64_t K, int8_t*
     }
   }
   return 0;
+}
+
+// X1 then X2 on whole rows. Returns 0, 1 if x holds Inf or NaN, 3 if the rounding mode is
+// not nearest.
+int oracle_quantize_acts(const void* x, int dtype, int64_t M, int64_t K, int8_t* q,
+                         float* scale) {
+  std::vector<float> amax(static_cast<size_t>(M));
+  if (oracle_act_absmax(x, dtype, M, K, amax.data()) != 0) return 1;
+  return oracle_quantize_acts_absmax(x, dtype, M, K, amax.data(), q, scale);
 }
 
 // Step C1: acc[t,n] = sum over k with c = +1 of q[t,k] minus sum over k with c = -1 of

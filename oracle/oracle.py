@@ -53,6 +53,14 @@ def lib() -> ctypes.CDLL:
         _lib.oracle_unpack.restype = i32
         _lib.oracle_quantize_acts.argtypes = [p, i32, i64, i64, p, p]
         _lib.oracle_quantize_acts.restype = i32
+        _lib.oracle_abs_buckets.argtypes = [p, i32, i64, p]
+        _lib.oracle_abs_buckets.restype = i32
+        _lib.oracle_absmean_from_buckets.argtypes = [p, i64, p]
+        _lib.oracle_absmean_from_buckets.restype = None
+        _lib.oracle_act_absmax.argtypes = [p, i32, i64, i64, p]
+        _lib.oracle_act_absmax.restype = i32
+        _lib.oracle_quantize_acts_absmax.argtypes = [p, i32, i64, i64, p, p, p]
+        _lib.oracle_quantize_acts_absmax.restype = i32
         _lib.oracle_contract_i32.argtypes = [p, p, i64, i64, i64, p]
         _lib.oracle_contract_i32.restype = None
         _lib.oracle_rescale.argtypes = [p, p, f32, i64, i64, p]
@@ -85,6 +93,48 @@ def absmean(W: np.ndarray) -> np.float32:
     if rc != 0:
         raise ValueError("non-finite weight")
     return out[0]
+
+
+def abs_buckets(W: np.ndarray) -> np.ndarray:
+    """The 256 exponent buckets (uint64) of the exact sum of |W|; the buckets of the parts
+    of a matrix add up (as integers) to those of the whole."""
+    W, dt = _as_input(W)
+    out = np.zeros(256, np.uint64)
+    if lib().oracle_abs_buckets(_ptr(W), dt, W.size, _ptr(out)) != 0:
+        raise ValueError("non-finite weight")
+    return out
+
+
+def absmean_from_buckets(buckets: np.ndarray, n: int) -> np.float32:
+    """gamma from the buckets of n values in all (the second half of absmean)."""
+    b = np.ascontiguousarray(buckets, dtype=np.uint64)
+    assert b.shape == (256,)
+    out = np.zeros(1, np.float32)
+    lib().oracle_absmean_from_buckets(_ptr(b), int(n), _ptr(out))
+    return out[0]
+
+
+def act_absmax(x: np.ndarray) -> np.ndarray:
+    """a_t = max_k |x[t,k]| (fp32 [M])."""
+    x, dt = _as_input(x)
+    M, K = x.shape
+    a = np.zeros(M, np.float32)
+    if lib().oracle_act_absmax(_ptr(x), dt, M, K, _ptr(a)) != 0:
+        raise ValueError("non-finite activation")
+    return a
+
+
+def quantize_acts_absmax(x: np.ndarray, amax: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """Per-token int8 quantization with a_t given (the absmax of the whole rows when x is a
+    K-shard of them)."""
+    x, dt = _as_input(x)
+    M, K = x.shape
+    a = np.ascontiguousarray(amax, dtype=np.float32)
+    q = np.zeros((M, K), np.int8)
+    s = np.zeros(M, np.float32)
+    if lib().oracle_quantize_acts_absmax(_ptr(x), dt, M, K, _ptr(a), _ptr(q), _ptr(s)) != 0:
+        raise RuntimeError("FPU rounding mode is not round-to-nearest")
+    return q, s
 
 
 def ternarize(W: np.ndarray, gamma: float, eps: float) -> np.ndarray:

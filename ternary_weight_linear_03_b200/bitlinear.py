@@ -24,6 +24,8 @@ STATUS = {
 # Every symbol declared in include/bitlinear.h.
 EXPORTS = (
     "bitlinear_workspace_size", "bitlinear_quantize_weights", "bitlinear_quantize_acts",
+    "bitlinear_weight_abssum", "bitlinear_quantize_weights_from_abssum", "bitlinear_act_absmax",
+    "bitlinear_quantize_acts_absmax", "bitlinear_rescale",
     "bitlinear_forward", "bitlinear_forward_noalloc", "bitlinear_contract_i32",
     "bitlinear_get_device_status",
     "bitlinear_debug_timeout_probe", "bitlinear_debug_plan", "bitlinear_status_string",
@@ -56,6 +58,17 @@ def load_library() -> ctypes.CDLL:
     lib.bitlinear_quantize_weights.restype = i
     lib.bitlinear_quantize_acts.argtypes = [p, i, i, i, p, p, p]
     lib.bitlinear_quantize_acts.restype = i
+    i64 = ctypes.c_longlong
+    lib.bitlinear_weight_abssum.argtypes = [p, i, i, i, p, p, sz, p]
+    lib.bitlinear_weight_abssum.restype = i
+    lib.bitlinear_quantize_weights_from_abssum.argtypes = [p, i, i, i, i64, p, f, p, p, p]
+    lib.bitlinear_quantize_weights_from_abssum.restype = i
+    lib.bitlinear_act_absmax.argtypes = [p, i, i, i, p, p]
+    lib.bitlinear_act_absmax.restype = i
+    lib.bitlinear_quantize_acts_absmax.argtypes = [p, i, i, i, p, p, p, p]
+    lib.bitlinear_quantize_acts_absmax.restype = i
+    lib.bitlinear_rescale.argtypes = [p, p, p, p, i, i, i, p]
+    lib.bitlinear_rescale.restype = i
     lib.bitlinear_forward.argtypes = [p, i, p, p, p, i, i, i, i, p, sz, p]
     lib.bitlinear_forward.restype = i
     lib.bitlinear_forward_noalloc.argtypes = [p, i, p, p, p, i, i, i, i, p]
@@ -141,6 +154,83 @@ def quantize_acts(x: torch.Tensor, stream=None) -> tuple[torch.Tensor, torch.Ten
                                        _dev(scale, "scale"), _stream(stream)),
            "bitlinear_quantize_acts")
     return xq, scale
+
+
+ABSSUM_WORDS = 14
+
+
+def weight_abssum(W: torch.Tensor, sums: torch.Tensor | None = None,
+                  ws: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Exact sum of |w| over W (a shard of a matrix) as ABSSUM_WORDS int64 words (uint64
+    bit patterns): the words of several shards add up exactly to those of their union."""
+    lib = load_library()
+    N, K = W.shape
+    if sums is None:
+        sums = torch.empty(ABSSUM_WORDS, dtype=torch.int64, device=W.device)
+    if ws is None:
+        ws = workspace(1, N, K, W.device)
+    _check(lib.bitlinear_weight_abssum(_dev(W, "W"), _dtype_code(W), N, K, _dev(sums, "sums"),
+                                       _dev(ws, "ws"), ws.numel(), _stream(stream)),
+           "bitlinear_weight_abssum")
+    return sums
+
+
+def quantize_weights_from_abssum(W: torch.Tensor, n_total: int, sums: torch.Tensor,
+                                 eps: float = 1e-5, packed: torch.Tensor | None = None,
+                                 gamma: torch.Tensor | None = None,
+                                 stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """gamma from the added words of every shard (over n_total weights), then this shard's
+    packed codes."""
+    lib = load_library()
+    N, K = W.shape
+    if packed is None:
+        packed = torch.empty((N, K // 4), dtype=torch.uint8, device=W.device)
+    if gamma is None:
+        gamma = torch.empty(1, dtype=torch.float32, device=W.device)
+    _check(lib.bitlinear_quantize_weights_from_abssum(
+        _dev(W, "W"), _dtype_code(W), N, K, int(n_total), _dev(sums, "sums"), float(eps),
+        _dev(packed, "packed"), _dev(gamma, "gamma"), _stream(stream)),
+        "bitlinear_quantize_weights_from_abssum")
+    return packed, gamma
+
+
+def act_absmax(x: torch.Tensor, amax: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Per-token max |x| (fp32 [M])."""
+    lib = load_library()
+    M, K = x.shape
+    if amax is None:
+        amax = torch.empty(M, dtype=torch.float32, device=x.device)
+    _check(lib.bitlinear_act_absmax(_dev(x, "x"), _dtype_code(x), M, K, _dev(amax, "amax"),
+                                    _stream(stream)), "bitlinear_act_absmax")
+    return amax
+
+
+def quantize_acts_absmax(x: torch.Tensor, amax: torch.Tensor,
+                         stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """Per-token int8 quantization with the absmax given (of the whole rows)."""
+    lib = load_library()
+    M, K = x.shape
+    xq = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    scale = torch.empty(M, dtype=torch.float32, device=x.device)
+    _check(lib.bitlinear_quantize_acts_absmax(_dev(x, "x"), _dtype_code(x), M, K,
+                                              _dev(amax, "amax"), _dev(xq, "xq"),
+                                              _dev(scale, "scale"), _stream(stream)),
+           "bitlinear_quantize_acts_absmax")
+    return xq, scale
+
+
+def rescale(acc: torch.Tensor, scale: torch.Tensor, gamma: torch.Tensor,
+            out_dtype: torch.dtype = torch.bfloat16, y: torch.Tensor | None = None,
+            stream=None) -> torch.Tensor:
+    """y = float(acc) * (scale_t * gamma) for an int32 product [M][N]."""
+    lib = load_library()
+    M, N = acc.shape
+    if y is None:
+        y = torch.empty((M, N), dtype=out_dtype, device=acc.device)
+    _check(lib.bitlinear_rescale(_dev(acc, "acc"), _dev(scale, "scale"), _dev(gamma, "gamma"),
+                                 _dev(y, "y"), _dtype_code(y), M, N, _stream(stream)),
+           "bitlinear_rescale")
+    return y
 
 
 def forward(x: torch.Tensor, packed: torch.Tensor, gamma: torch.Tensor,

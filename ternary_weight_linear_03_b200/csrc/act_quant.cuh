@@ -72,13 +72,22 @@ __device__ __forceinline__ void grid_zero(uint4* __restrict__ z, long long n16) 
     z[i] = make_uint4(0u, 0u, 0u, 0u);
 }
 
+// Where a token's absmax a_t comes from.
+enum AqMode : int {
+  kAqRow = 0,     // from the row itself (the whole row is in x)
+  kAqGiven = 1,   // from amax[t], computed elsewhere: over the whole row when x holds only
+                  // a K-shard of it (tensor parallelism), or by the kernel that produced x
+  kAqAbsmax = 2,  // only compute a_t = max_k |x[t,k]| into amax[t]; no codes
+};
+
 // grid = M blocks, K % 8 == 0. rowsum may be null; zero/zero_n16 name an extra region to
 // clear (may be null/0). Lets the dependent kernel launch at once (it waits for this
 // grid's completion before reading any of these outputs).
-template <bool kBf16>
+template <bool kBf16, int AMODE = kAqRow>
 __global__ void __launch_bounds__(kAqThreads) act_quant_kernel(
     const void* __restrict__ x, int K, int8_t* __restrict__ xq, float* __restrict__ scale,
-    int* __restrict__ rowsum, uint4* __restrict__ zero, long long zero_n16) {
+    int* __restrict__ rowsum, uint4* __restrict__ zero, long long zero_n16,
+    float* __restrict__ amax = nullptr) {
   __shared__ float redf[32];
   __shared__ int redi[32];
   allow_dependent_launch();
@@ -87,19 +96,28 @@ __global__ void __launch_bounds__(kAqThreads) act_quant_kernel(
   const char* row = static_cast<const char*>(x) + static_cast<size_t>(t) * K * (kBf16 ? 2 : 4);
   const int nc = K / 8;
   float a = 0.0f;
-  bool bad = false;
-  for (int c = threadIdx.x; c < nc; c += blockDim.x) {
-    float v[8];
-    load8<kBf16>(row, c, v);
+  if (AMODE == kAqGiven) {
+    a = amax[t];
+    if (!(a <= 3.4028234663852886e38f)) record_status(kStatusNonfinite);
+  } else {
+    bool bad = false;
+    for (int c = threadIdx.x; c < nc; c += blockDim.x) {
+      float v[8];
+      load8<kBf16>(row, c, v);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float m = abs_bits(v[i]);
-      bad |= !(m <= 3.4028234663852886e38f);
-      a = fmaxf(a, m);
+      for (int i = 0; i < 8; ++i) {
+        const float m = abs_bits(v[i]);
+        bad |= !(m <= 3.4028234663852886e38f);
+        a = fmaxf(a, m);
+      }
+    }
+    if (bad) record_status(kStatusNonfinite);
+    a = block_max(a, redf);
+    if (AMODE == kAqAbsmax) {
+      if (threadIdx.x == 0) amax[t] = a;
+      return;
     }
   }
-  if (bad) record_status(kStatusNonfinite);
-  a = block_max(a, redf);
   const float r = (a > 0.0f) ? __fdiv_rn(127.0f, a) : 0.0f;
   int8_t* qrow = xq + static_cast<size_t>(t) * K;
   int sum = 0;

@@ -17,6 +17,7 @@
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
 #include "per_device.h"
+#include "rescale.cuh"
 #include "weight_quant.cuh"
 
 namespace {
@@ -394,11 +395,11 @@ bl_status launch_act_quant(const void* x, int x_dtype, int M, int K, int8_t* xq,
 // Workspace of bitlinear_quantize_weights: the exact-sum columns and the barrier counters.
 size_t wq_ws_bytes(long long) { return align_up(sizeof(WqWorkspace), 256); }
 
-template <bool kBf16>
-bl_status launch_weight_quant_t(const void* W, long long n, float eps, void* ws,
-                                size_t ws_bytes, float* gamma, uint32_t* packed,
-                                cudaStream_t s) {
-  auto kern = bl::weight_quant_kernel<kBf16>;
+template <bool kBf16, int MODE>
+bl_status launch_weight_quant_t(const void* W, long long n, long long n_total, float eps,
+                                void* ws, unsigned long long* sums, float* gamma,
+                                uint32_t* packed, cudaStream_t s) {
+  auto kern = bl::weight_quant_kernel<kBf16, MODE>;
   constexpr int kSmem = bl::kWqStages * bl::kWqStageBytes;
   // blocks of this kernel resident per SM, found once per device after raising its
   // shared-memory limit (a cooperative launch needs every block resident)
@@ -418,20 +419,25 @@ bl_status launch_weight_quant_t(const void* W, long long n, float eps, void* ws,
   const int grid = static_cast<int>(
       std::max<long long>(1, std::min<long long>(want, 1ll * blocks_per_sm * num_sms())));
   WqWorkspace* hdr = static_cast<WqWorkspace*>(ws);
-  (void)ws_bytes;
-  if (cudaMemsetAsync(hdr, 0, sizeof(WqWorkspace), s) != cudaSuccess) return BL_ERR_CUDA;
+  if (MODE != bl::kWqFinish &&
+      cudaMemsetAsync(hdr, 0, sizeof(WqWorkspace), s) != cudaSuccess)
+    return BL_ERR_CUDA;
   unsigned long long limit = kWaitLimitNs;
-  void* args[] = {const_cast<void**>(&W), &n, &eps, &hdr, &gamma, &packed, &limit};
+  void* args[] = {const_cast<void**>(&W), &n, &n_total, &eps, &hdr, &sums, &gamma, &packed,
+                  &limit};
   if (cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kern), dim3(grid),
                                   dim3(bl::kWqThreads), args, kSmem, s) != cudaSuccess)
     return BL_ERR_CUDA;
   return launch_status();
 }
 
-bl_status launch_weight_quant(const void* W, bool bf16, long long n, float eps, void* ws,
-                              size_t ws_bytes, float* gamma, uint32_t* packed, cudaStream_t s) {
-  return bf16 ? launch_weight_quant_t<true>(W, n, eps, ws, ws_bytes, gamma, packed, s)
-              : launch_weight_quant_t<false>(W, n, eps, ws, ws_bytes, gamma, packed, s);
+template <int MODE>
+bl_status launch_weight_quant(const void* W, bool bf16, long long n, long long n_total,
+                              float eps, void* ws, unsigned long long* sums, float* gamma,
+                              uint32_t* packed, cudaStream_t s) {
+  return bf16 ? launch_weight_quant_t<true, MODE>(W, n, n_total, eps, ws, sums, gamma, packed, s)
+              : launch_weight_quant_t<false, MODE>(W, n, n_total, eps, ws, sums, gamma, packed,
+                                                   s);
 }
 
 // ------------------------------------------------------------------ debug probe
@@ -500,8 +506,39 @@ bl_status bitlinear_quantize_weights(const void* W, int w_dtype, int N, int K, f
     return BL_ERR_MISALIGNED;
   if (ws_bytes < sizeof(WqWorkspace)) return BL_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return launch_weight_quant(W, w_dtype == BL_BF16, static_cast<long long>(N) * K, eps, ws,
-                             ws_bytes, gamma, reinterpret_cast<uint32_t*>(packed), s);
+  const long long n = static_cast<long long>(N) * K;
+  return launch_weight_quant<bl::kWqFull>(W, w_dtype == BL_BF16, n, n, eps, ws, nullptr, gamma,
+                                          reinterpret_cast<uint32_t*>(packed), s);
+}
+
+bl_status bitlinear_weight_abssum(const void* W, int w_dtype, int N, int K, uint64_t* sums,
+                                  void* ws, size_t ws_bytes, void* stream) {
+  if (!W || !sums || !ws) return BL_ERR_INVALID_ARG;
+  if (w_dtype != BL_F32 && w_dtype != BL_BF16) return BL_ERR_INVALID_ARG;
+  if (!shape_ok(1, N, K)) return BL_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(W) || !aligned16(sums) || !aligned16(ws)) return BL_ERR_MISALIGNED;
+  if (ws_bytes < sizeof(WqWorkspace)) return BL_ERR_WORKSPACE;
+  const long long n = static_cast<long long>(N) * K;
+  return launch_weight_quant<bl::kWqPartial>(
+      W, w_dtype == BL_BF16, n, n, 0.0f, ws, reinterpret_cast<unsigned long long*>(sums),
+      nullptr, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+bl_status bitlinear_quantize_weights_from_abssum(const void* W, int w_dtype, int N, int K,
+                                                 long long n_total, const uint64_t* sums,
+                                                 float eps, uint8_t* packed, float* gamma,
+                                                 void* stream) {
+  if (!W || !sums || !packed || !gamma) return BL_ERR_INVALID_ARG;
+  if (w_dtype != BL_F32 && w_dtype != BL_BF16) return BL_ERR_INVALID_ARG;
+  if (!(eps >= 0.0f) || !std::isfinite(eps)) return BL_ERR_INVALID_ARG;
+  if (!shape_ok(1, N, K)) return BL_ERR_UNSUPPORTED_SHAPE;
+  if (n_total < static_cast<long long>(N) * K) return BL_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(sums) || !aligned16(packed) || !aligned16(gamma))
+    return BL_ERR_MISALIGNED;
+  return launch_weight_quant<bl::kWqFinish>(
+      W, w_dtype == BL_BF16, static_cast<long long>(N) * K, n_total, eps, nullptr,
+      const_cast<unsigned long long*>(reinterpret_cast<const unsigned long long*>(sums)), gamma,
+      reinterpret_cast<uint32_t*>(packed), static_cast<cudaStream_t>(stream));
 }
 
 bl_status bitlinear_quantize_acts(const void* x, int x_dtype, int M, int K, int8_t* xq,
@@ -511,6 +548,65 @@ bl_status bitlinear_quantize_acts(const void* x, int x_dtype, int M, int K, int8
   if (!shape_ok(M, 1, K)) return BL_ERR_UNSUPPORTED_SHAPE;
   if (!aligned16(x) || !aligned16(xq) || !aligned16(scale)) return BL_ERR_MISALIGNED;
   return launch_act_quant(x, x_dtype, M, K, xq, scale, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+bl_status bitlinear_act_absmax(const void* x, int x_dtype, int M, int K, float* amax,
+                               void* stream) {
+  if (!x || !amax) return BL_ERR_INVALID_ARG;
+  if (x_dtype != BL_F32 && x_dtype != BL_BF16) return BL_ERR_INVALID_ARG;
+  if (!shape_ok(M, 1, K)) return BL_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(x) || !aligned16(amax)) return BL_ERR_MISALIGNED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (x_dtype == BL_BF16)
+    bl::act_quant_kernel<true, bl::kAqAbsmax><<<M, bl::kAqThreads, 0, s>>>(
+        x, K, nullptr, nullptr, nullptr, nullptr, 0, amax);
+  else
+    bl::act_quant_kernel<false, bl::kAqAbsmax><<<M, bl::kAqThreads, 0, s>>>(
+        x, K, nullptr, nullptr, nullptr, nullptr, 0, amax);
+  return launch_status();
+}
+
+bl_status bitlinear_quantize_acts_absmax(const void* x, int x_dtype, int M, int K,
+                                         const float* amax, int8_t* xq, float* scale,
+                                         void* stream) {
+  if (!x || !amax || !xq || !scale) return BL_ERR_INVALID_ARG;
+  if (x_dtype != BL_F32 && x_dtype != BL_BF16) return BL_ERR_INVALID_ARG;
+  if (!shape_ok(M, 1, K)) return BL_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(x) || !aligned16(amax) || !aligned16(xq) || !aligned16(scale))
+    return BL_ERR_MISALIGNED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float* a = const_cast<float*>(amax);
+  if (x_dtype == BL_BF16)
+    bl::act_quant_kernel<true, bl::kAqGiven><<<M, bl::kAqThreads, 0, s>>>(
+        x, K, xq, scale, nullptr, nullptr, 0, a);
+  else
+    bl::act_quant_kernel<false, bl::kAqGiven><<<M, bl::kAqThreads, 0, s>>>(
+        x, K, xq, scale, nullptr, nullptr, 0, a);
+  return launch_status();
+}
+
+bl_status bitlinear_rescale(const int32_t* acc, const float* scale, const float* gamma,
+                            void* y, int y_dtype, int M, int N, void* stream) {
+  if (!acc || !scale || !gamma || !y) return BL_ERR_INVALID_ARG;
+  if (y_dtype != BL_F32 && y_dtype != BL_BF16) return BL_ERR_INVALID_ARG;
+  if (M < 1 || N < 1 || static_cast<long long>(M) * N >= (1ll << 31))
+    return BL_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(acc) || !aligned16(scale) || !aligned16(gamma) || !aligned16(y))
+    return BL_ERR_MISALIGNED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const long long work = static_cast<long long>(M) * N / ((N % 4 == 0) ? 4 : 1);
+  const int grid = static_cast<int>(std::max<long long>(
+      1, std::min<long long>((work + bl::kRsThreads - 1) / bl::kRsThreads, 8ll * num_sms())));
+  if (N % 4 == 0) {
+    if (y_dtype == BL_F32) bl::rescale_kernel<0><<<grid, bl::kRsThreads, 0, s>>>(acc, scale, gamma, y, M, N);
+    else bl::rescale_kernel<1><<<grid, bl::kRsThreads, 0, s>>>(acc, scale, gamma, y, M, N);
+  } else {
+    if (y_dtype == BL_F32)
+      bl::rescale_scalar_kernel<0><<<grid, bl::kRsThreads, 0, s>>>(acc, scale, gamma, y, M, N);
+    else
+      bl::rescale_scalar_kernel<1><<<grid, bl::kRsThreads, 0, s>>>(acc, scale, gamma, y, M, N);
+  }
+  return launch_status();
 }
 
 bl_status bitlinear_forward(const void* x, int x_dtype, const uint8_t* packed,

@@ -199,12 +199,34 @@ __device__ __forceinline__ void wq_issue(const WqRing& r, int st, int g) {
   bulk_load(r.stage + slot * kWqStageBytes, r.src + 1ll * st * kWqStageBytes, nb, &r.full[slot]);
 }
 
+// What one launch does. A matrix split over several GPUs (tensor parallelism) still has
+// one gamma, the mean over the whole matrix: every shard computes its part of the exact
+// sum (kWqPartial), the parts are added across the GPUs (the kWqLimbs 64-bit column sums
+// add exactly, like any integers below 2^64), and every shard then codes its weights
+// against that total (kWqFinish).
+enum WqMode : int {
+  kWqFull = 0,     // exact sum, gamma, codes: the whole matrix in one launch
+  kWqPartial = 1,  // exact sum only: writes the kWqLimbs column sums to sums_io
+  kWqFinish = 2,   // gamma and codes from the column sums in sums_io, over n_total values
+};
+
+// The kWqLimbs column sums of the block copies in the workspace, added (below 2^64: each
+// is below 2^39 times the grid size).
+__device__ __forceinline__ unsigned long long wq_column_total(const WqWorkspace* ws, int j) {
+  unsigned long long t = 0ull;
+#pragma unroll
+  for (int c = 0; c < kWqCopies; ++c) t += __ldcg(&ws->cols[c][j]);
+  return t;
+}
+
 // W holds n values (fp32, or bf16 if kBf16), n % 16 == 0, 16-byte aligned. Launched
 // cooperatively (all blocks resident) with kWqStages * kWqStageBytes of dynamic shared
-// memory. ws is zeroed by the host.
-template <bool kBf16>
+// memory. ws is zeroed by the host (kWqFull, kWqPartial). gamma is the exact sum over
+// n_total values (n_total = n except for kWqFinish on a shard).
+template <bool kBf16, int MODE>
 __global__ void __launch_bounds__(kWqThreads) weight_quant_kernel(
-    const void* __restrict__ W, long long n, float eps, WqWorkspace* __restrict__ ws,
+    const void* __restrict__ W, long long n, long long n_total, float eps,
+    WqWorkspace* __restrict__ ws, unsigned long long* __restrict__ sums_io,
     float* __restrict__ gamma_out, uint32_t* __restrict__ packed, unsigned long long limit_ns) {
   extern __shared__ __align__(128) unsigned char wq_stage[];  // kWqStages x 16 KB
   __shared__ unsigned long long sb[kWqBuckets];
@@ -238,6 +260,8 @@ __global__ void __launch_bounds__(kWqThreads) weight_quant_kernel(
   __syncthreads();
 
   // ---------------------------------------------------------------- pass A: exact sum
+  bool resident = false;  // pass B reads pass A's stages from shared memory
+  if (MODE != kWqFinish) {
   double acc0 = 0.0, acc1 = 0.0;
   bool nonfinite = false;
   int base = 1;
@@ -320,8 +344,8 @@ __global__ void __launch_bounds__(kWqThreads) weight_quant_kernel(
   // When the block's whole range fits the ring, pass A left every stage in its slot
   // (stage st in slot st) and pass B reads them there; otherwise pass B streams the range
   // again, starting now (its stages do not depend on gamma).
-  const bool resident = ring.nst <= kWqStages;
-  if (tid == 0 && !resident)
+  resident = ring.nst <= kWqStages;
+  if (MODE == kWqFull && tid == 0 && !resident)
     for (int st = 0; st < kWqStages; ++st) wq_issue(ring, st, ring.nst + st);
 
   // ---------------------------------------------------------------- grid barrier
@@ -344,26 +368,29 @@ __global__ void __launch_bounds__(kWqThreads) weight_quant_kernel(
     }
   }
   __syncthreads();
+  if (MODE == kWqPartial) {  // this shard's column sums are the result
+    if (blockIdx.x == 0 && tid < kWqLimbs) sums_io[tid] = wq_column_total(ws, tid);
+    return;
+  }
+  if (tid < kWqLimbs) col[tid] = wq_column_total(ws, tid);
+  }  // pass A
+  if (MODE == kWqFinish && tid < kWqLimbs) col[tid] = sums_io[tid];  // added over all shards
 
   // ---------------------------------------------------------------- gamma and T
-  if (tid < kWqLimbs) {
-    unsigned long long t = 0ull;  // below 2^39 times the grid size: far from 2^64
-#pragma unroll
-    for (int c = 0; c < kWqCopies; ++c) t += __ldcg(&ws->cols[c][tid]);
-    col[tid] = t;
-  }
   __syncthreads();
   if (tid == 0) {
     uint32_t L[kWqLimbs];
     unsigned long long carry = 0ull;
 #pragma unroll
     for (int j = 0; j < kWqLimbs; ++j) {
-      const unsigned long long t = col[j] + carry;  // no overflow (see above)
+      // no overflow: a column is below 2^39 per block (2^57 for 2^18 blocks over all
+      // shards) and a carry below 2^32
+      const unsigned long long t = col[j] + carry;
       L[j] = static_cast<uint32_t>(t);
       carry = t >> 32;
     }
     const double S = wq_limbs_to_double(L);
-    const float gamma = __double2float_rn(__ddiv_rn(S, static_cast<double>(n)));
+    const float gamma = __double2float_rn(__ddiv_rn(S, static_cast<double>(n_total)));
     if (blockIdx.x == 0) *gamma_out = gamma;
     s_T = wq_threshold(__fadd_rn(gamma, eps));
   }
@@ -375,8 +402,9 @@ __global__ void __launch_bounds__(kWqThreads) weight_quant_kernel(
   uint32_t mul[E];                     // 1 << bit position of element e of this part
 #pragma unroll
   for (int e = 0; e < E; ++e) mul[e] = 1u << wq_shift(wq_k<kBf16>(part, e));
+  const int g0 = (MODE == kWqFinish) ? 0 : ring.nst;  // stages pass A consumed
   for (int st = 0; st < ring.nst; ++st) {
-    const int g = ring.nst + st;  // stages consumed by this block so far
+    const int g = g0 + st;  // stages consumed by this block so far
     const int slot = resident ? st : g % kWqStages;
     if (!resident && !mbar_wait(&full[slot], static_cast<uint32_t>((g / kWqStages) & 1), limit_ns))
       s_ok = 0;
@@ -401,7 +429,7 @@ __global__ void __launch_bounds__(kWqThreads) weight_quant_kernel(
     if (resident) continue;
     __syncthreads();
     if (tid == 0 && st + kWqStages < ring.nst)
-      wq_issue(ring, st + kWqStages, ring.nst + st + kWqStages);
+      wq_issue(ring, st + kWqStages, g0 + st + kWqStages);
   }
   (void)s_ok;
 }

@@ -75,3 +75,26 @@ def test_argument_errors_are_synchronous(lib):
     assert q(FAKE, 0, 1, 63, FAKE, FAKE, None) == 2
     assert q(FAKE, 3, 1, 64, FAKE, FAKE, None) == 1
     assert lib.bitlinear_debug_timeout_probe(10, None) == 1                      # < 1 us
+
+
+def test_tensor_parallel_entry_points_check_arguments(lib):
+    a = lib.bitlinear_weight_abssum
+    assert a(None, 0, 16, 64, FAKE, FAKE, 1 << 20, None) == 1
+    assert a(FAKE, 0, 16, 96, FAKE, FAKE, 1 << 20, None) == 2
+    assert a(FAKE, 0, 16, 64, FAKE + 8, FAKE, 1 << 20, None) == 3
+    assert a(FAKE, 0, 16, 64, FAKE, FAKE, 16, None) == 7
+    f = lib.bitlinear_quantize_weights_from_abssum
+    assert f(FAKE, 0, 16, 64, 16 * 64, None, 1e-5, FAKE, FAKE, None) == 1
+    assert f(FAKE, 0, 16, 64, 16 * 64 - 1, FAKE, 1e-5, FAKE, FAKE, None) == 1  # n_total < N*K
+    assert f(FAKE, 0, 16, 64, 16 * 64, FAKE, -1.0, FAKE, FAKE, None) == 1
+    assert f(FAKE, 0, 16, 64, 16 * 64, FAKE, 1e-5, FAKE + 4, FAKE, None) == 3
+    m = lib.bitlinear_act_absmax
+    assert m(FAKE, 2, 1, 64, FAKE, None) == 1
+    assert m(FAKE, 0, 1, 65, FAKE, None) == 2
+    q = lib.bitlinear_quantize_acts_absmax
+    assert q(FAKE, 0, 1, 64, None, FAKE, FAKE, None) == 1
+    assert q(FAKE, 0, 1, 64, FAKE, FAKE + 1, FAKE, None) == 3
+    r = lib.bitlinear_rescale
+    assert r(FAKE, FAKE, FAKE, FAKE, 2, 1, 16, None) == 1   # int32 out is not a rescale
+    assert r(FAKE, FAKE, FAKE, FAKE, 0, 0, 16, None) == 2
+    assert r(FAKE, FAKE, FAKE, FAKE + 2, 0, 1, 16, None) == 3

@@ -34,7 +34,7 @@ def _worker(rank, world, port, results):
 
 def test_two_rank_gloo_logic():
     world = 2
-    manager = mp.Manager()
+    manager = mp.get_context("spawn").Manager()
     results = manager.dict()
     mp.spawn(_worker, args=(world, _free_port(), results), nprocs=world, join=True)
     assert set(results.keys()) == {0, 1}

@@ -292,3 +292,53 @@ def test_forward_quantization_error_bound():
     s = np.abs(x).max(axis=1) / 127.0
     bound = float(gamma) * (s[:, None] / 2) * np.abs(codes).sum(axis=1)[None, :] * (1 + 1e-5)
     assert np.all(np.abs(y - exact) <= bound + 1e-5 * np.abs(exact))
+
+
+# ----------------------------------------------------------------------------- shards
+
+
+@pytest.mark.parametrize("split", ["rows", "cols"])
+def test_abs_buckets_of_shards_add_to_the_whole(split):
+    """The two halves of absmean: the bucket arrays of the parts of a matrix add up to the
+    whole's, and gamma formed from the added buckets is the correctly rounded mean of the
+    whole (math.fsum), also when the parts differ in scale by 10^6."""
+    rng = np.random.default_rng(11)
+    W = (rng.standard_normal((64, 320)) * 0.02).astype(np.float32)
+    W[:32] *= 1e-6 if split == "rows" else 1.0
+    W[:, :128] *= 1e3 if split == "cols" else 1.0
+    parts = [W[:32], W[32:]] if split == "rows" else [W[:, :128], W[:, 128:]]
+    b = sum(orc.abs_buckets(np.ascontiguousarray(p)) for p in parts)
+    np.testing.assert_array_equal(b, orc.abs_buckets(W))
+    assert orc.absmean_from_buckets(b, W.size) == _fsum_gamma(W)
+    assert orc.absmean_from_buckets(b, W.size) == orc.absmean(W)
+
+
+def test_act_absmax_is_numpy_max():
+    rng = np.random.default_rng(12)
+    x = (rng.standard_normal((7, 192)) * 3).astype(np.float32)
+    x[2] = 0.0
+    np.testing.assert_array_equal(orc.act_absmax(x), np.max(np.abs(x), axis=1))
+
+
+def test_quantize_acts_absmax_on_k_shards_matches_whole_rows():
+    """A row held in K-shards: each shard quantized with the absmax of the whole row gives
+    exactly the whole row's codes and scale."""
+    rng = np.random.default_rng(13)
+    x = (rng.standard_normal((5, 512)) * 2).astype(np.float32)
+    x[1, 300] = 40.0  # the row's maximum lies in the second shard
+    q, s = orc.quantize_acts(x)
+    a = np.max(np.abs(x), axis=1)
+    for k0, k1 in [(0, 192), (192, 512)]:
+        qs, ss = orc.quantize_acts_absmax(np.ascontiguousarray(x[:, k0:k1]), a)
+        np.testing.assert_array_equal(qs, q[:, k0:k1])
+        np.testing.assert_array_equal(ss, s)
+
+
+def test_quantize_acts_absmax_closed_form():
+    """With a_t = 2 * 127 / 127 = 2 and x = 1 the code is rne(1 * fl(127/2)) = rne(63.5) =
+    64 (ties to even); x = a_t gives 127; x above a_t clips to 127."""
+    x = np.array([[1.0, 2.0, 3.0, -5.0, 0.0, 0.5, -1.0, 1.5]], np.float32)
+    x = np.tile(x, (1, 8))
+    q, s = orc.quantize_acts_absmax(x, np.array([2.0], np.float32))
+    np.testing.assert_array_equal(q[0, :8], [64, 127, 127, -127, 0, 32, -64, 95])
+    assert s[0] == np.float32(2.0) / np.float32(127.0)
