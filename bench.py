@@ -313,6 +313,60 @@ def decode_figure(bl, name: str, M: int, device, hbm_peak: float, i8_peak: float
             "bound": bound, "tokens_per_s": M / (ms * 1e-3), "weight_copies": copies}
 
 
+def sweep_3b_figures(bl, device, hbm_peak: float, Ms=(1, 16, 64), blocks: int = 26):
+    """The 3B-class feed-forward sweep: 26 blocks of gate and up (3200 -> 8640, one shared
+    input) and down (8640 -> 3200, reading up; the elementwise activation between them is
+    not part of BitLinear), 78 matrices and 539 MB of packed weights, as one
+    bitlinear_chain_forward captured in a CUDA graph; next to it the same 78 forwards as
+    separate bitlinear_forward calls (each quantizing its own input) in one graph."""
+    d, h = 3200, 8640
+    layers, src = [], -1
+    for b in range(blocks):
+        for i, (N, K) in enumerate([(h, d), (h, d), (d, h)]):
+            W = syn.weights(N, K, 0.02, seed=9000 + 3 * b + i, device=device)
+            packed, gamma = bl.quantize_weights(W, EPS)
+            del W
+            layers.append([packed, gamma, src if i < 2 else len(layers) - 1])
+        src = len(layers) - 1
+    torch.cuda.synchronize()
+    w_bytes = sum(ly[0].numel() for ly in layers)
+    rows = []
+    for M in Ms:
+        gate = torch.empty((M, h), dtype=torch.bfloat16, device=device)
+        chain = [(p_, g_, s_, gate) if i % 3 == 0 else (p_, g_, s_)
+                 for i, (p_, g_, s_) in enumerate(layers)]
+        x = syn.activations(M, d, seed=77 + M, device=device)
+        y = torch.empty((M, d), dtype=torch.bfloat16, device=device)
+        ws = bl.chain_workspace(M, chain, device)
+        bl.chain_forward(x, chain, y=y, ws=ws)
+        torch.cuda.synchronize()
+        ms_chain = statistics.mean(time_in_graph(
+            [lambda: bl.chain_forward(x, chain, y=y, ws=ws)] * 4))
+        # unchained: separate forwards, each quantizing its input itself
+        bufs = {-1: x}
+        outs = [torch.empty((M, ly[0].shape[0]), dtype=torch.bfloat16, device=device)
+                for ly in layers]
+        fws = torch.empty(max(bl.workspace_size(M, h, d), bl.workspace_size(M, d, h)),
+                          dtype=torch.uint8, device=device)
+
+        def separate():
+            for i, (p_, g_, s_) in enumerate(layers):
+                bl.forward(bufs[s_] if s_ < 0 else outs[s_], p_, g_, y=outs[i], ws=fws)
+
+        separate()
+        torch.cuda.synchronize()
+        ms_sep = statistics.mean(time_in_graph([separate] * 2))
+        gbs = w_bytes / (ms_chain * 1e-3) / 1e9
+        rows.append({"M": M, "ms_per_sweep": ms_chain, "tokens_per_s": M / (ms_chain * 1e-3),
+                     "GBps": gbs, "frac_hbm": gbs / hbm_peak,
+                     "ms_per_sweep_separate_forwards": ms_sep,
+                     "ideal_ms_at_peak": w_bytes / (hbm_peak * 1e9) * 1e3})
+        del ws, bufs, outs
+    return {"matrices": len(layers), "packed_MB": w_bytes / 1e6, "rows": rows,
+            "launches_per_sweep": {"chain": "1 memset + per matrix 1 kernel (GEMV) or "
+                                            "act quant once per input + 1 tensor-core kernel"}}
+
+
 # LLaMA-70B-style layer matrices (out x in) and how many of each one layer holds; 80 layers.
 WQ_70B_SHAPES = [(8192, 8192, 2), (1024, 8192, 2), (28672, 8192, 3)]
 WQ_70B_LAYERS = 80
@@ -512,6 +566,7 @@ def main():
                                          ("700m_up_1536x4096", 1), ("700m_up_1536x4096", 4),
                                          ("700m_up_1536x4096", 16)]]
         others["weight_quant_70b"] = weight_quant_figures(bl, device, hbm_peak)
+        others["sweep_3b_26_layers"] = sweep_3b_figures(bl, device, hbm_peak)
     roofline["others"] = others
 
     cpu = None

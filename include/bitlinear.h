@@ -63,6 +63,16 @@ typedef enum {
 
 typedef enum { BL_F32 = 0, BL_BF16 = 1, BL_I32 = 2 } bl_dtype;
 
+/* One BitLinear layer of a chain (bitlinear_chain_forward). */
+typedef struct {
+  const uint8_t* packed; /* device [N][K/4], from bitlinear_quantize_weights */
+  const float* gamma;    /* device, one float */
+  int N, K;              /* out x in */
+  int src;               /* its input: -1 = the chain input x, j = the output of layer j < this */
+  void* out;             /* device [M][N] bf16 to receive its output, or NULL (then kept in
+                            the workspace); ignored for the last layer, which writes y */
+} bl_layer;
+
 /* Device bytes of workspace that bitlinear_quantize_weights (for N x K) and
  * bitlinear_forward / bitlinear_contract_i32 (for M x N x K) need; the largest of the
  * three. Pure host function. Returns 0 for shapes the library rejects. */
@@ -165,6 +175,31 @@ bl_status bitlinear_rescale(const int32_t* acc, const float* scale, const float*
 bl_status bitlinear_forward(const void* x, int x_dtype, const uint8_t* packed,
                             const float* gamma, void* y, int y_dtype, int M, int N, int K,
                             void* ws, size_t ws_bytes, void* stream);
+
+/* Workspace bytes of bitlinear_chain_forward for these layers and M tokens; 0 if the
+ * chain is invalid. Pure host function. */
+size_t bitlinear_chain_workspace_size(int M, const bl_layer* layers, int L);
+
+/* A chain of BitLinear layers over one batch of M tokens, every layer as in
+ * bitlinear_forward: layer l reads x (src = -1) or the output of an earlier layer, every
+ * output but the last is kept in bf16 (the activation type of the model), the last
+ * layer writes y. Several layers may read the same input (the gate and up projections of
+ * a feed-forward block); the input is then quantized once.
+ * Fused across layers: the kernel that writes a layer's output also forms the per-token
+ * absmax of it (atomic max in its epilogue), so the next layer's activation quantization
+ * is a single pass (or part of the GEMV's prologue); every kernel is launched with
+ * programmatic dependent launch, so it sets up, and prefetches its packed weights (TMA
+ * into shared memory, or into L2), while the kernel before it still runs. Capture the call
+ * in a CUDA graph to take the host out of the loop. Results equal layer-by-layer
+ * bitlinear_forward calls with bf16 intermediates, bit for bit.
+ *   x       device [M][K of the layers with src = -1], fp32 or bf16.
+ *   layers  host array of L layers; K of a layer with src = j equals N of layer j.
+ *   y       device [M][N of the last layer], BL_F32 or BL_BF16.
+ *   ws      device, at least bitlinear_chain_workspace_size bytes (contents ignored).
+ * Errors as bitlinear_forward; BL_ERR_INVALID_ARG for a bad src, null pointers or L < 1. */
+bl_status bitlinear_chain_forward(const void* x, int x_dtype, int M, const bl_layer* layers,
+                                  int L, void* y, int y_dtype, void* ws, size_t ws_bytes,
+                                  void* stream);
 
 /* The integer stage alone (test hook, same kernels as bitlinear_forward):
  * acc[t,n] = sum_k c[n,k] * xq[t,k].

@@ -25,11 +25,18 @@ STATUS = {
 EXPORTS = (
     "bitlinear_workspace_size", "bitlinear_quantize_weights", "bitlinear_quantize_acts",
     "bitlinear_weight_abssum", "bitlinear_quantize_weights_from_abssum", "bitlinear_act_absmax",
-    "bitlinear_quantize_acts_absmax", "bitlinear_rescale",
+    "bitlinear_quantize_acts_absmax", "bitlinear_rescale", "bitlinear_chain_workspace_size",
+    "bitlinear_chain_forward",
     "bitlinear_forward", "bitlinear_forward_noalloc", "bitlinear_contract_i32",
     "bitlinear_get_device_status",
     "bitlinear_debug_timeout_probe", "bitlinear_debug_plan", "bitlinear_status_string",
 )
+
+
+class Layer(ctypes.Structure):
+    """bl_layer of include/bitlinear.h: one layer of a chain."""
+    _fields_ = [("packed", ctypes.c_void_p), ("gamma", ctypes.c_void_p), ("N", ctypes.c_int),
+                ("K", ctypes.c_int), ("src", ctypes.c_int), ("out", ctypes.c_void_p)]
 
 
 class BitLinearError(RuntimeError):
@@ -69,6 +76,10 @@ def load_library() -> ctypes.CDLL:
     lib.bitlinear_quantize_acts_absmax.restype = i
     lib.bitlinear_rescale.argtypes = [p, p, p, p, i, i, i, p]
     lib.bitlinear_rescale.restype = i
+    lib.bitlinear_chain_workspace_size.argtypes = [i, ctypes.POINTER(Layer), i]
+    lib.bitlinear_chain_workspace_size.restype = sz
+    lib.bitlinear_chain_forward.argtypes = [p, i, i, ctypes.POINTER(Layer), i, p, i, p, sz, p]
+    lib.bitlinear_chain_forward.restype = i
     lib.bitlinear_forward.argtypes = [p, i, p, p, p, i, i, i, i, p, sz, p]
     lib.bitlinear_forward.restype = i
     lib.bitlinear_forward_noalloc.argtypes = [p, i, p, p, p, i, i, i, i, p]
@@ -230,6 +241,44 @@ def rescale(acc: torch.Tensor, scale: torch.Tensor, gamma: torch.Tensor,
     _check(lib.bitlinear_rescale(_dev(acc, "acc"), _dev(scale, "scale"), _dev(gamma, "gamma"),
                                  _dev(y, "y"), _dtype_code(y), M, N, _stream(stream)),
            "bitlinear_rescale")
+    return y
+
+
+def chain_layers(layers) -> ctypes.Array:
+    """ctypes array of bl_layer from (packed, gamma, src[, out]) tuples (device tensors;
+    out a bf16 [M][N] tensor or None)."""
+    arr = (Layer * len(layers))()
+    for i, ly in enumerate(layers):
+        packed, gamma, src = ly[0], ly[1], ly[2]
+        out = ly[3] if len(ly) > 3 else None
+        arr[i] = Layer(_dev(packed, "packed"), _dev(gamma, "gamma"), packed.shape[0],
+                       packed.shape[1] * 4, int(src), _dev(out, "out") if out is not None else None)
+    return arr
+
+
+def chain_workspace(M: int, layers, device="cuda") -> torch.Tensor:
+    arr = chain_layers(layers)
+    n = int(load_library().bitlinear_chain_workspace_size(M, arr, len(layers)))
+    if n == 0:
+        raise BitLinearError(1, "bitlinear_chain_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def chain_forward(x: torch.Tensor, layers, out_dtype: torch.dtype = torch.bfloat16,
+                  y: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+                  stream=None) -> torch.Tensor:
+    """A chain of BitLinear layers (bitlinear_chain_forward): layers are (packed, gamma,
+    src[, out]) with src = -1 for x or the index of the layer whose output is the input."""
+    lib = load_library()
+    M = x.shape[0]
+    arr = chain_layers(layers)
+    if y is None:
+        y = torch.empty((M, layers[-1][0].shape[0]), dtype=out_dtype, device=x.device)
+    if ws is None:
+        ws = chain_workspace(M, layers, x.device)
+    _check(lib.bitlinear_chain_forward(_dev(x, "x"), _dtype_code(x), M, arr, len(layers),
+                                       _dev(y, "y"), _dtype_code(y), _dev(ws, "ws"), ws.numel(),
+                                       _stream(stream)), "bitlinear_chain_forward")
     return y
 
 

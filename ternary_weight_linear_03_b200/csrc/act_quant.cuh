@@ -91,6 +91,7 @@ __global__ void __launch_bounds__(kAqThreads) act_quant_kernel(
   __shared__ float redf[32];
   __shared__ int redi[32];
   allow_dependent_launch();
+  grid_dependency_wait();  // x (and amax) may come from the kernel before; no-op otherwise
   grid_zero(zero, zero_n16);
   const int t = blockIdx.x;
   const char* row = static_cast<const char*>(x) + static_cast<size_t>(t) * K * (kBf16 ? 2 : 4);

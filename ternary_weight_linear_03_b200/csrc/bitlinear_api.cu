@@ -9,6 +9,8 @@
 #include <cmath>
 #include <cstdint>
 #include <mutex>
+#include <utility>
+#include <vector>
 
 #include "../../include/bitlinear.h"
 #include "act_quant.cuh"
@@ -151,6 +153,33 @@ bl_status launch_status() {
   return (cudaGetLastError() == cudaSuccess) ? BL_OK : BL_ERR_CUDA;
 }
 
+// Options of a launch inside a layer chain (bitlinear_chain_forward); all off for the
+// single-layer entry points.
+struct ChainOpts {
+  const float* amax_in = nullptr;  // absmax of the input rows, from the kernel that wrote them
+  float* amax_out = nullptr;       // receives the absmax of this launch's output rows
+  bool pdl = false;                // programmatic dependent launch on the kernel before
+};
+
+// Launches kern with or without programmatic stream serialization.
+template <typename... KArgs, typename... Args>
+bl_status launch_ex(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                    bool pdl, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = pdl ? attr : nullptr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  if (cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...) != cudaSuccess)
+    return BL_ERR_CUDA;
+  return launch_status();
+}
+
 // ------------------------------------------------------------------ TMA descriptors
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -201,7 +230,7 @@ int choose_lpr_log2(int cpr) {
 
 template <int MT, int XM, int OM, bool XR, int R>
 bl_status launch_gemv_t(const void* x, const uint8_t* packed, const float* gamma, void* y,
-                        int N, int K, cudaStream_t s) {
+                        int N, int K, cudaStream_t s, const ChainOpts& o) {
   auto kern = bl::gemv_kernel<MT, XM, OM, XR, R>;
   const int smem = MT * K;
   static bl::PerDevice configured;
@@ -215,8 +244,9 @@ bl_status launch_gemv_t(const void* x, const uint8_t* packed, const float* gamma
   const long long rows_per_block = static_cast<long long>(bl::kGemvWarps) * (32 >> lpr_log2) * R;
   const long long need = (N + rows_per_block - 1) / rows_per_block;
   const int grid = static_cast<int>(std::min<long long>(need, 1ll * blocks_per_sm * num_sms()));
-  kern<<<grid, bl::kGemvThreads, smem, s>>>(x, packed, gamma, y, N, K, lpr_log2);
-  return launch_status();
+  const int chain = o.pdl ? 1 : 0;
+  return launch_ex(kern, dim3(grid), dim3(bl::kGemvThreads), smem, s, o.pdl, x, packed, gamma,
+                   y, N, K, lpr_log2, o.amax_in, o.amax_out, chain);
 }
 
 // Activations stay in registers for one token when a lane owns at most kGemvRegChunks
@@ -235,33 +265,35 @@ bool gemv_two_rows(int N, int K) {
 
 template <int MT, int XM, int OM>
 bl_status launch_gemv_r(const void* x, const uint8_t* packed, const float* gamma, void* y,
-                        int N, int K, cudaStream_t s) {
-  return gemv_two_rows(N, K) ? launch_gemv_t<MT, XM, OM, false, 2>(x, packed, gamma, y, N, K, s)
-                             : launch_gemv_t<MT, XM, OM, false, 1>(x, packed, gamma, y, N, K, s);
+                        int N, int K, cudaStream_t s, const ChainOpts& o) {
+  return gemv_two_rows(N, K)
+             ? launch_gemv_t<MT, XM, OM, false, 2>(x, packed, gamma, y, N, K, s, o)
+             : launch_gemv_t<MT, XM, OM, false, 1>(x, packed, gamma, y, N, K, s, o);
 }
 
 template <int XM, int OM>
 bl_status launch_gemv_m(const void* x, const uint8_t* packed, const float* gamma, void* y,
-                        int M, int N, int K, cudaStream_t s) {
+                        int M, int N, int K, cudaStream_t s, const ChainOpts& o) {
   switch (M) {
     case 1:
       return gemv_x_in_registers(M, K)
-                 ? launch_gemv_t<1, XM, OM, true, 1>(x, packed, gamma, y, N, K, s)
-                 : launch_gemv_r<1, XM, OM>(x, packed, gamma, y, N, K, s);
-    case 2: return launch_gemv_r<2, XM, OM>(x, packed, gamma, y, N, K, s);
-    case 3: return launch_gemv_r<3, XM, OM>(x, packed, gamma, y, N, K, s);
-    case 4: return launch_gemv_r<4, XM, OM>(x, packed, gamma, y, N, K, s);
+                 ? launch_gemv_t<1, XM, OM, true, 1>(x, packed, gamma, y, N, K, s, o)
+                 : launch_gemv_r<1, XM, OM>(x, packed, gamma, y, N, K, s, o);
+    case 2: return launch_gemv_r<2, XM, OM>(x, packed, gamma, y, N, K, s, o);
+    case 3: return launch_gemv_r<3, XM, OM>(x, packed, gamma, y, N, K, s, o);
+    case 4: return launch_gemv_r<4, XM, OM>(x, packed, gamma, y, N, K, s, o);
     default: return BL_ERR_UNSUPPORTED_SHAPE;
   }
 }
 
 template <int XM>
 bl_status launch_gemv_x(const void* x, const uint8_t* packed, const float* gamma, void* y,
-                        int y_dtype, int M, int N, int K, cudaStream_t s) {
+                        int y_dtype, int M, int N, int K, cudaStream_t s,
+                        const ChainOpts& o = {}) {
   switch (y_dtype) {
-    case BL_F32: return launch_gemv_m<XM, bl::kOf32>(x, packed, gamma, y, M, N, K, s);
-    case BL_BF16: return launch_gemv_m<XM, bl::kObf16>(x, packed, gamma, y, M, N, K, s);
-    case BL_I32: return launch_gemv_m<XM, bl::kOi32>(x, packed, gamma, y, M, N, K, s);
+    case BL_F32: return launch_gemv_m<XM, bl::kOf32>(x, packed, gamma, y, M, N, K, s, o);
+    case BL_BF16: return launch_gemv_m<XM, bl::kObf16>(x, packed, gamma, y, M, N, K, s, o);
+    case BL_I32: return launch_gemv_m<XM, bl::kOi32>(x, packed, gamma, y, M, N, K, s, o);
     default: return BL_ERR_INVALID_ARG;
   }
 }
@@ -270,7 +302,7 @@ bl_status launch_gemv_x(const void* x, const uint8_t* packed, const float* gamma
 template <int OM>
 bl_status launch_gemm_t(const int8_t* xq, const uint8_t* packed, const int* rowsum,
                         const float* scale, const float* gamma, void* y, int M, int N, int K,
-                        cudaStream_t s) {
+                        cudaStream_t s, const ChainOpts& o) {
   CUtensorMap map_a, map_b;
   if (!make_map_u8(&map_a, xq, K, M, K, bl::tc::BK, bl::tc::BM, true)) return BL_ERR_CUDA;
   if (!make_map_u8(&map_b, packed, K / 4, N, K / 4, bl::tc::BK / 4, bl::tc::BN, false))
@@ -281,18 +313,17 @@ bl_status launch_gemm_t(const int8_t* xq, const uint8_t* packed, const int* rows
   const long long tiles = static_cast<long long>((M + bl::tc::BM - 1) / bl::tc::BM) *
                           ((N + bl::tc::BN - 1) / bl::tc::BN);
   const int grid = static_cast<int>(std::min<long long>(tiles, num_sms()));
-  kern<<<grid, bl::tc::THREADS, bl::tc::SMEM_BYTES, s>>>(map_a, map_b, rowsum, scale, gamma, y,
-                                                         M, N, K, kWaitLimitNs);
-  return launch_status();
+  return launch_ex(kern, dim3(grid), dim3(bl::tc::THREADS), bl::tc::SMEM_BYTES, s, o.pdl,
+                   map_a, map_b, rowsum, scale, gamma, y, M, N, K, kWaitLimitNs, o.amax_out);
 }
 
 bl_status launch_gemm(const int8_t* xq, const uint8_t* packed, const int* rowsum,
                       const float* scale, const float* gamma, void* y, int y_dtype, int M, int N,
-                      int K, cudaStream_t s) {
+                      int K, cudaStream_t s, const ChainOpts& o = {}) {
   switch (y_dtype) {
-    case BL_F32: return launch_gemm_t<0>(xq, packed, rowsum, scale, gamma, y, M, N, K, s);
-    case BL_BF16: return launch_gemm_t<1>(xq, packed, rowsum, scale, gamma, y, M, N, K, s);
-    case BL_I32: return launch_gemm_t<2>(xq, packed, rowsum, scale, gamma, y, M, N, K, s);
+    case BL_F32: return launch_gemm_t<0>(xq, packed, rowsum, scale, gamma, y, M, N, K, s, o);
+    case BL_BF16: return launch_gemm_t<1>(xq, packed, rowsum, scale, gamma, y, M, N, K, s, o);
+    case BL_I32: return launch_gemm_t<2>(xq, packed, rowsum, scale, gamma, y, M, N, K, s, o);
     default: return BL_ERR_INVALID_ARG;
   }
 }
@@ -300,7 +331,8 @@ bl_status launch_gemm(const int8_t* xq, const uint8_t* packed, const int* rowsum
 template <int OM>
 bl_status launch_skinny_t(const int8_t* xq, const uint8_t* packed, const int* rowsum,
                           const float* scale, const float* gamma, void* y, int M, int N, int K,
-                          const SkinnyPlan& p, const SkinnyWs& w, cudaStream_t s) {
+                          const SkinnyPlan& p, const SkinnyWs& w, cudaStream_t s,
+                          float* amax_out) {
   CUtensorMap map_x, map_w;
   if (!make_map_u8(&map_x, xq, K, M, K, bl::sk::BK, p.bnt, true)) return BL_ERR_CUDA;
   if (!make_map_u8(&map_w, packed, K / 4, N, K / 4, bl::sk::BK * bl::sk::KPS / 4, bl::sk::BW,
@@ -314,21 +346,10 @@ bl_status launch_skinny_t(const int8_t* xq, const uint8_t* packed, const int* ro
   // Programmatic dependent launch: the kernel may start while the quantization kernel before
   // it (which also zeroed the split-K sums and counters) is still running; it loads W and
   // sets up TMEM meanwhile and waits for that grid before touching its outputs.
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(p.tiles * p.splits));
-  cfg.blockDim = dim3(bl::sk::THREADS);
-  cfg.dynamicSmemBytes = static_cast<size_t>(bl::sk::smem_bytes(p.bnt));
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, map_x, map_w, rowsum, scale, gamma, y, w.partial,
-                         w.counters, M, N, K, p.bnt, p.splits, p.kbps, kWaitLimitNs) !=
-      cudaSuccess)
-    return BL_ERR_CUDA;
-  return launch_status();
+  return launch_ex(kern, dim3(static_cast<unsigned>(p.tiles * p.splits)),
+                   dim3(bl::sk::THREADS), static_cast<size_t>(bl::sk::smem_bytes(p.bnt)), s,
+                   true, map_x, map_w, rowsum, scale, gamma, y, w.partial, w.counters, M, N, K,
+                   p.bnt, p.splits, p.kbps, kWaitLimitNs, amax_out);
 }
 
 // The part of the workspace the skinny kernel needs zeroed (split-K sums and counters; a
@@ -345,11 +366,14 @@ void skinny_zero_region(void* ws, int M, int N, int K, uint4** z, long long* n16
 bl_status launch_skinny_plan(const int8_t* xq, const uint8_t* packed, const int* rowsum,
                              const float* scale, const float* gamma, void* y, int y_dtype,
                              int M, int N, int K, const SkinnyPlan& p, const SkinnyWs& w,
-                             cudaStream_t s) {
+                             cudaStream_t s, float* amax_out = nullptr) {
   switch (y_dtype) {
-    case BL_F32: return launch_skinny_t<0>(xq, packed, rowsum, scale, gamma, y, M, N, K, p, w, s);
-    case BL_BF16: return launch_skinny_t<1>(xq, packed, rowsum, scale, gamma, y, M, N, K, p, w, s);
-    case BL_I32: return launch_skinny_t<2>(xq, packed, rowsum, scale, gamma, y, M, N, K, p, w, s);
+    case BL_F32:
+      return launch_skinny_t<0>(xq, packed, rowsum, scale, gamma, y, M, N, K, p, w, s, amax_out);
+    case BL_BF16:
+      return launch_skinny_t<1>(xq, packed, rowsum, scale, gamma, y, M, N, K, p, w, s, amax_out);
+    case BL_I32:
+      return launch_skinny_t<2>(xq, packed, rowsum, scale, gamma, y, M, N, K, p, w, s, amax_out);
     default: return BL_ERR_INVALID_ARG;
   }
 }
@@ -389,6 +413,27 @@ bl_status launch_act_quant(const void* x, int x_dtype, int M, int K, int8_t* xq,
     bl::act_quant_kernel<false><<<M, bl::kAqThreads, 0, s>>>(x, K, xq, scale, rowsum, zero,
                                                              zero_n16);
   return launch_status();
+}
+
+// The activation quantization inside a chain: absmax given (from the kernel that wrote x)
+// or not (the chain's input), launched with programmatic dependent launch.
+bl_status launch_act_quant_chain(const void* x, int x_dtype, int M, int K, int8_t* xq,
+                                 float* scale, int* rowsum, cudaStream_t s,
+                                 const float* amax_in) {
+  float* a = const_cast<float*>(amax_in);
+  if (x_dtype == BL_BF16)
+    return amax_in ? launch_ex(bl::act_quant_kernel<true, bl::kAqGiven>, dim3(M),
+                               dim3(bl::kAqThreads), 0, s, true, x, K, xq, scale, rowsum,
+                               static_cast<uint4*>(nullptr), 0ll, a)
+                   : launch_ex(bl::act_quant_kernel<true, bl::kAqRow>, dim3(M),
+                               dim3(bl::kAqThreads), 0, s, true, x, K, xq, scale, rowsum,
+                               static_cast<uint4*>(nullptr), 0ll, a);
+  return amax_in ? launch_ex(bl::act_quant_kernel<false, bl::kAqGiven>, dim3(M),
+                             dim3(bl::kAqThreads), 0, s, true, x, K, xq, scale, rowsum,
+                             static_cast<uint4*>(nullptr), 0ll, a)
+                 : launch_ex(bl::act_quant_kernel<false, bl::kAqRow>, dim3(M),
+                             dim3(bl::kAqThreads), 0, s, true, x, K, xq, scale, rowsum,
+                             static_cast<uint4*>(nullptr), 0ll, a);
 }
 
 // ------------------------------------------------------------------ weight quantization
@@ -636,6 +681,161 @@ bl_status bitlinear_forward(const void* x, int x_dtype, const uint8_t* packed,
   if (M <= kSkinnyMaxM)
     return launch_skinny(w.xq, packed, w.rowsum, w.scale, gamma, y, y_dtype, M, N, K, ws, s);
   return launch_gemm(w.xq, packed, w.rowsum, w.scale, gamma, y, y_dtype, M, N, K, s);
+}
+
+}  // extern "C"
+
+namespace {
+
+// Workspace plan of a layer chain (see bitlinear_chain_forward). Activation buffer j = 0 is
+// the chain input x, j = l + 1 the output of layer l.
+struct ChainPlan {
+  int L = 0, M = 0, K0 = 0;
+  size_t bytes = 0;
+  // offsets into the workspace (bytes)
+  size_t amax_off = 0;      // (L + 1) x M floats: absmax of every activation buffer
+  size_t partial_off = 0;   // shared int32 split-K sums (self-cleaning), then counters
+  size_t zero_bytes = 0;    // bytes from amax_off cleared once per call
+  size_t counters_off = 0;
+  std::vector<size_t> act_off;   // per layer: its output in the workspace (or SIZE_MAX)
+  std::vector<size_t> xq_off;    // per buffer j: int8 codes + scale + rowsum (or SIZE_MAX)
+  std::vector<char> consumed;    // per buffer j: read by a later layer
+};
+
+constexpr size_t kNone = static_cast<size_t>(-1);
+
+bl_status chain_plan(int M, const bl_layer* layers, int L, ChainPlan* plan) {
+  if (!layers || L < 1 || L > 4096 || M < 1) return BL_ERR_INVALID_ARG;
+  ChainPlan p;
+  p.L = L;
+  p.M = M;
+  p.consumed.assign(L + 1, 0);
+  p.act_off.assign(L, kNone);
+  p.xq_off.assign(L + 1, kNone);
+  int K0 = -1;
+  for (int l = 0; l < L; ++l) {
+    const bl_layer& ly = layers[l];
+    if (!ly.packed || !ly.gamma) return BL_ERR_INVALID_ARG;
+    if (ly.src < -1 || ly.src >= l) return BL_ERR_INVALID_ARG;
+    if (!shape_ok(M, ly.N, ly.K)) return BL_ERR_UNSUPPORTED_SHAPE;
+    if (ly.src == -1) {
+      if (K0 >= 0 && K0 != ly.K) return BL_ERR_UNSUPPORTED_SHAPE;
+      K0 = ly.K;
+    } else if (layers[ly.src].N != ly.K) {
+      return BL_ERR_UNSUPPORTED_SHAPE;
+    }
+    if (!aligned16(ly.packed) || !aligned16(ly.gamma) || (ly.out && !aligned16(ly.out)))
+      return BL_ERR_MISALIGNED;
+    p.consumed[ly.src + 1] = 1;
+  }
+  if (K0 < 0) return BL_ERR_INVALID_ARG;  // nothing reads x
+  p.K0 = K0;
+  size_t off = 0;
+  p.amax_off = off;
+  off += align_up(static_cast<size_t>(L + 1) * M * 4, 256);
+  size_t part = 0, tiles = 0;
+  for (int l = 0; l < L; ++l) {
+    const bl_layer& ly = layers[l];
+    if (!use_gemv(M, ly.N, ly.K) && M <= kSkinnyMaxM) {
+      const SkinnyPlan sp = skinny_plan(M, ly.N, ly.K);
+      if (sp.splits > 1) part = std::max(part, static_cast<size_t>(M) * ly.N * 4);
+      tiles = std::max(tiles, static_cast<size_t>(sp.tiles));
+    }
+  }
+  p.partial_off = off;
+  off += align_up(part, 256);
+  p.counters_off = off;
+  off += align_up(tiles * 4, 256);
+  p.zero_bytes = off - p.amax_off;
+  for (int l = 0; l < L; ++l) {
+    const bl_layer& ly = layers[l];
+    const bool last = (l == L - 1);
+    if (!last && ly.out == nullptr) {
+      p.act_off[l] = off;
+      off += align_up(static_cast<size_t>(M) * ly.N * 2, 256);
+    }
+    const int j = ly.src + 1;
+    if (!use_gemv(M, ly.N, ly.K) && p.xq_off[j] == kNone) {
+      p.xq_off[j] = off;
+      off += fwd_ws_layout(nullptr, M, ly.K).bytes;
+    }
+  }
+  p.bytes = align_up(std::max<size_t>(off, 256), 256);
+  *plan = std::move(p);
+  return BL_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t bitlinear_chain_workspace_size(int M, const bl_layer* layers, int L) {
+  ChainPlan p;
+  if (chain_plan(M, layers, L, &p) != BL_OK) return 0;
+  return p.bytes;
+}
+
+bl_status bitlinear_chain_forward(const void* x, int x_dtype, int M, const bl_layer* layers,
+                                  int L, void* y, int y_dtype, void* ws, size_t ws_bytes,
+                                  void* stream) {
+  if (!x || !y || !ws) return BL_ERR_INVALID_ARG;
+  if (x_dtype != BL_F32 && x_dtype != BL_BF16) return BL_ERR_INVALID_ARG;
+  if (y_dtype != BL_F32 && y_dtype != BL_BF16) return BL_ERR_INVALID_ARG;
+  ChainPlan p;
+  bl_status st = chain_plan(M, layers, L, &p);
+  if (st != BL_OK) return st;
+  if (!aligned16(x) || !aligned16(y) || !aligned16(ws)) return BL_ERR_MISALIGNED;
+  if (ws_bytes < p.bytes) return BL_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  char* base = static_cast<char*>(ws);
+  float* amax = reinterpret_cast<float*>(base + p.amax_off);
+  if (cudaMemsetAsync(base + p.amax_off, 0, p.zero_bytes, s) != cudaSuccess) return BL_ERR_CUDA;
+  std::vector<char> quantized(L + 1, 0);
+  for (int l = 0; l < L; ++l) {
+    const bl_layer& ly = layers[l];
+    const int j = ly.src + 1;  // input buffer
+    const void* in = (j == 0) ? x : (layers[ly.src].out ? layers[ly.src].out
+                                                          : base + p.act_off[ly.src]);
+    const int in_dtype = (j == 0) ? x_dtype : BL_BF16;
+    const float* amax_in = (j == 0) ? nullptr : amax + static_cast<size_t>(j) * M;
+    const bool last = (l == L - 1);
+    void* out = last ? y : (ly.out ? ly.out : base + p.act_off[l]);
+    const int out_dtype = last ? y_dtype : BL_BF16;
+    float* amax_out = (!last && p.consumed[l + 1]) ? amax + static_cast<size_t>(l + 1) * M : nullptr;
+    if (use_gemv(M, ly.N, ly.K)) {
+      ChainOpts o;
+      o.amax_in = amax_in;
+      o.amax_out = amax_out;
+      o.pdl = true;
+      st = (in_dtype == BL_BF16)
+               ? launch_gemv_x<bl::kXbf16>(in, ly.packed, ly.gamma, out, out_dtype, M, ly.N, ly.K, s, o)
+               : launch_gemv_x<bl::kXf32>(in, ly.packed, ly.gamma, out, out_dtype, M, ly.N, ly.K, s, o);
+      if (st != BL_OK) return st;
+      continue;
+    }
+    FwdWs w = fwd_ws_layout(base + p.xq_off[j], M, ly.K);
+    if (!quantized[j]) {  // once per input buffer, whatever number of layers read it
+      st = launch_act_quant_chain(in, in_dtype, M, ly.K, w.xq, w.scale, w.rowsum, s, amax_in);
+      if (st != BL_OK) return st;
+      quantized[j] = 1;
+    }
+    if (M <= kSkinnyMaxM) {
+      const SkinnyPlan sp = skinny_plan(M, ly.N, ly.K);
+      SkinnyWs sw{};
+      sw.partial = reinterpret_cast<int*>(base + p.partial_off);
+      sw.counters = reinterpret_cast<unsigned int*>(base + p.counters_off);
+      st = launch_skinny_plan(w.xq, ly.packed, w.rowsum, w.scale, ly.gamma, out, out_dtype, M,
+                              ly.N, ly.K, sp, sw, s, amax_out);
+    } else {
+      ChainOpts o;
+      o.amax_out = amax_out;
+      o.pdl = true;
+      st = launch_gemm(w.xq, ly.packed, w.rowsum, w.scale, ly.gamma, out, out_dtype, M, ly.N,
+                       ly.K, s, o);
+    }
+    if (st != BL_OK) return st;
+  }
+  return BL_OK;
 }
 
 bl_status bitlinear_contract_i32(const int8_t* xq, const uint8_t* packed, int32_t* acc, int M,

@@ -191,16 +191,36 @@ __device__ __forceinline__ bool epi_bar_or(bool v) { return bar_or<1, 128>(v); }
 __device__ __forceinline__ bool group_bar_or(bool v) { return bar_or<2, 160>(v); }
 
 // Rescales one accumulator and stores it. OM: 0 fp32, 1 bf16, 2 int32 (acc only).
+// Returns the bit pattern of |stored value| (0 for int32 output), for the absmax of a
+// chain's next layer: non-negative floats order like their bits.
 template <int OM>
-__device__ __forceinline__ void store_out(void* y, long long o, int a, float scale_t,
-                                          float gamma) {
+__device__ __forceinline__ unsigned store_out(void* y, long long o, int a, float scale_t,
+                                              float gamma) {
   if (OM == 2) {
     static_cast<int*>(y)[o] = a;
+    return 0u;
   } else {
     const float val = __fmul_rn(__int2float_rn(a), __fmul_rn(scale_t, gamma));
-    if (OM == 0) static_cast<float*>(y)[o] = val;
-    else static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(val);
+    if (OM == 0) {
+      static_cast<float*>(y)[o] = val;
+      return __float_as_uint(val) & 0x7fffffffu;
+    }
+    const __nv_bfloat16 h = __float2bfloat16_rn(val);
+    static_cast<__nv_bfloat16*>(y)[o] = h;
+    return __float_as_uint(__bfloat162float(h)) & 0x7fffffffu;
   }
+}
+
+// Atomic max of a non-negative float given by its bits (fire and forget).
+__device__ __forceinline__ void red_max_u32(float* p, unsigned bits) {
+  asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" ::"l"(p), "r"(bits) : "memory");
+}
+
+// The warp's largest |y| for token t (all 32 lanes call it with their own value) added
+// into amax_out[t] by lane 0.
+__device__ __forceinline__ void warp_amax_out(float* amax_out, int t, unsigned bits) {
+  const unsigned m = __reduce_max_sync(0xffffffffu, bits);
+  if ((threadIdx.x & 31) == 0 && m != 0u) red_max_u32(amax_out + t, m);
 }
 
 // bnt = token tile (multiple of 16, >= M). grid = n_tiles * splits; CTA u handles weight
@@ -213,8 +233,9 @@ __global__ void __launch_bounds__(sk::THREADS, 1) gemm_skinny_kernel(
     const int* __restrict__ rowsum, const float* __restrict__ scale,
     const float* __restrict__ gamma_ptr, void* __restrict__ y, int* __restrict__ partial,
     unsigned int* __restrict__ counters, int M, int N, int K, int bnt, int splits,
-    int kb_per_split, unsigned long long limit_ns) {
+    int kb_per_split, unsigned long long limit_ns, float* __restrict__ amax_out) {
   using namespace sk;
+  allow_dependent_launch();  // the next kernel may set up (it waits before using y)
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -445,10 +466,12 @@ __global__ void __launch_bounds__(sk::THREADS, 1) gemm_skinny_kernel(
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int t = c0 + j;
+            unsigned mag = 0u;
             if (t < M && nvalid)
-              store_out<OM>(y, static_cast<long long>(t) * N + n,
-                            static_cast<int>(v[j]) - rowsum[t], OM == 2 ? 0.0f : scale[t],
-                            gamma);
+              mag = store_out<OM>(y, static_cast<long long>(t) * N + n,
+                                  static_cast<int>(v[j]) - rowsum[t],
+                                  OM == 2 ? 0.0f : scale[t], gamma);
+            if (amax_out != nullptr && t < M) warp_amax_out(amax_out, t, mag);
           }
         }
       } else {
@@ -470,21 +493,28 @@ __global__ void __launch_bounds__(sk::THREADS, 1) gemm_skinny_kernel(
           bar->last = (prev == static_cast<unsigned int>(splits - 1)) ? 1 : 0;
         }
         epi_bar_sync();
-        if (bar->last && nvalid) {
+        if (bar->last) {  // the same for the whole CTA
           __threadfence();
           for (int t0 = 0; t0 < M; t0 += 16) {
             int a[16];
 #pragma unroll
-            for (int j = 0; j < 16; ++j)
-              a[j] = (t0 + j < M) ? __ldcg(partial + static_cast<long long>(t0 + j) * N + n) : 0;
+            for (int j = 0; j < 16; ++j) {
+              int* pp = partial + static_cast<long long>(t0 + j) * N + n;
+              a[j] = (t0 + j < M && nvalid) ? __ldcg(pp) : 0;
+              // leave the sums zeroed for the next launch that shares them (layer chains)
+              if (t0 + j < M && nvalid) __stcg(pp, 0);
+            }
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
               const int t = t0 + j;
-              if (t < M)
-                store_out<OM>(y, static_cast<long long>(t) * N + n, a[j] - rowsum[t],
-                              OM == 2 ? 0.0f : scale[t], gamma);
+              unsigned mag = 0u;
+              if (t < M && nvalid)
+                mag = store_out<OM>(y, static_cast<long long>(t) * N + n, a[j] - rowsum[t],
+                                    OM == 2 ? 0.0f : scale[t], gamma);
+              if (amax_out != nullptr && t < M) warp_amax_out(amax_out, t, mag);
             }
           }
+          if (threadIdx.x == 0) counters[tile] = 0u;  // every split has arrived
         }
       }
     }

@@ -79,8 +79,9 @@ __global__ void __launch_bounds__(tc::THREADS, 1) gemm_tc_kernel(
     const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
     const int* __restrict__ rowsum, const float* __restrict__ scale,
     const float* __restrict__ gamma_ptr, void* __restrict__ y, int M, int N, int K,
-    unsigned long long limit_ns) {
+    unsigned long long limit_ns, float* __restrict__ amax_out) {
   using namespace tc;
+  allow_dependent_launch();  // the next kernel may set up (it waits before using y)
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -121,6 +122,9 @@ __global__ void __launch_bounds__(tc::THREADS, 1) gemm_tc_kernel(
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = bar->tmem_base;
+  // Set-up done; the operands come from the kernel before (programmatic dependent launch:
+  // returns at once when launched without it).
+  grid_dependency_wait();
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
@@ -214,6 +218,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1) gemm_tc_kernel(
       const float f = (OM != 2 && valid) ? __fmul_rn(scale[m], gamma) : 0.0f;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                              static_cast<uint32_t>(ab * BN);
+      float ymax = 0.0f;  // largest |y| of this row in the tile (layer chains)
 #pragma unroll 1
       for (int cb = 0; cb < BN / 32; ++cb) {
         uint32_t v[32];
@@ -239,6 +244,13 @@ __global__ void __launch_bounds__(tc::THREADS, 1) gemm_tc_kernel(
 #pragma unroll
           for (int j = 0; j < 32; ++j)
             r[j] = __fmul_rn(__int2float_rn(static_cast<int>(v[j]) - rs), f);
+          if (amax_out != nullptr) {
+            // the bf16 rounding is monotone: the largest stored magnitude is the rounding
+            // of the largest fp32 one
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (n + j < N) ymax = fmaxf(ymax, fabsf(r[j]));
+          }
           if (OM == 0) {
             float* out = static_cast<float*>(y) + o;
             if (vec) {
@@ -269,6 +281,10 @@ __global__ void __launch_bounds__(tc::THREADS, 1) gemm_tc_kernel(
             }
           }
         }
+      }
+      if (OM != 2 && amax_out != nullptr && valid && ymax > 0.0f) {
+        const float m = (OM == 1) ? __bfloat162float(__float2bfloat16_rn(ymax)) : ymax;
+        atomicMax(reinterpret_cast<unsigned*>(amax_out) + m0 + row, __float_as_uint(m));
       }
       tc_fence_before();
       __syncwarp();

@@ -64,7 +64,37 @@ struct GemvShared {
   int red_i[MT][32];
   float f[MT];      // s_t * gamma
   int rowsum[MT];
+  float ymax[MT][32];  // per-warp max |y| of each token (layer chains)
 };
+
+// Largest |y| of the outputs this thread stored, per token, merged over the block and added
+// into amax_out[t] with one atomic max per block and token: the absmax the next layer of a
+// chain quantizes its input (this layer's output) with. Non-negative floats order like
+// their bit patterns, so the maximum is taken on the bits. Called by every thread.
+template <int MT>
+__device__ __forceinline__ void block_amax_out(const float (&ymax)[MT], GemvShared<MT>& sh,
+                                               float* __restrict__ amax_out) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int t = 0; t < MT; ++t) {
+    const unsigned m = __reduce_max_sync(0xffffffffu, __float_as_uint(ymax[t]));
+    if (lane == 0) sh.ymax[t][warp] = __uint_as_float(m);
+  }
+  __syncthreads();
+  if (threadIdx.x < MT) {
+    float m = 0.0f;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) m = fmaxf(m, sh.ymax[threadIdx.x][w]);
+    if (m > 0.0f) atomicMax(reinterpret_cast<unsigned*>(amax_out) + threadIdx.x, __float_as_uint(m));
+  }
+}
+
+// |value| of an output as stored (the bf16 rounding is monotone, so the largest stored
+// magnitude is the rounding of the largest fp32 one; taken per value here for clarity).
+template <int OM>
+__device__ __forceinline__ float stored_mag(float v) {
+  if (OM == 1) return fabsf(__bfloat162float(__float2bfloat16_rn(v)));
+  return fabsf(v);
+}
 
 // Loads 16 consecutive x values of row t starting at element k (k % 16 == 0).
 template <int XM>
@@ -90,15 +120,38 @@ __device__ __forceinline__ void load16(const void* x, long long off, float (&v)[
 
 // XR: activations in registers (one token). R: rows a warp sums at once on the shared-
 // memory path (2 lets every activation load feed two rows; worth it only with many rows).
+// Layer chains (optional, null when unused): amax_in[t] is the absmax of token t's row of
+// x, formed by the kernel that wrote x, so the prologue skips its max pass; amax_out
+// receives the absmax of this kernel's outputs per token (atomic max; zeroed beforehand).
+// Launched with programmatic dependent launch, the kernel first lets the next kernel of
+// the stream launch, and starts the L2 prefetch of its own weights, before it waits for
+// the kernel that wrote x.
 template <int MT, int XM, int OM, bool XR, int R>
 __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(
     const void* __restrict__ x, const uint8_t* __restrict__ packed,
-    const float* __restrict__ gamma_ptr, void* __restrict__ y, int N, int K, int lpr_log2) {
+    const float* __restrict__ gamma_ptr, void* __restrict__ y, int N, int K, int lpr_log2,
+    const float* __restrict__ amax_in = nullptr, float* __restrict__ amax_out = nullptr,
+    int chain = 0) {
   extern __shared__ __align__(16) unsigned char xs_raw[];  // [MT][K] int8, permuted
   __shared__ GemvShared<MT> sh;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int CPR = K >> 6;   // 16-byte packed chunks per weight row
   const int KB = K >> 4;    // 16-element groups per token row
+  allow_dependent_launch();
+  if (chain) {
+    // L2 prefetch of this block's share of the packed weights (it does not depend on the
+    // kernel before), in 4 KB pieces, then wait for that kernel's outputs
+    const long long wbytes = static_cast<long long>(N) * (K >> 2);
+    const long long per = (wbytes + gridDim.x - 1) / gridDim.x;
+    const long long b0 = min(wbytes, per * blockIdx.x), b1 = min(wbytes, b0 + per);
+    for (long long o = (b0 & ~4095ll) + 4096ll * tid; o < b1; o += 4096ll * kGemvThreads) {
+      const long long len = min(4096ll, wbytes - o);
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(packed + o),
+                   "r"(static_cast<unsigned>(len & ~15ll))
+                   : "memory");
+    }
+  }
+  grid_dependency_wait();
 
   // ---------------------------------------------------------------- prologue: x -> int8
   if (XM == kXi8) {
@@ -137,18 +190,23 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(
     bool bad = false;
 #pragma unroll
     for (int t = 0; t < MT; ++t) amax[t] = 0.0f;
-    for (int kb = tid; kb < KB; kb += kGemvThreads) {
+    if (amax_in == nullptr) {
+      for (int kb = tid; kb < KB; kb += kGemvThreads) {
 #pragma unroll
-      for (int t = 0; t < MT; ++t) {
-        float v[16];
-        load16<XM>(x, static_cast<long long>(t) * K + 16 * kb, v);
+        for (int t = 0; t < MT; ++t) {
+          float v[16];
+          load16<XM>(x, static_cast<long long>(t) * K + 16 * kb, v);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float m = abs_bits(v[i]);
-          bad |= !(m <= 3.4028234663852886e38f);
-          amax[t] = fmaxf(amax[t], m);
+          for (int i = 0; i < 16; ++i) {
+            const float m = abs_bits(v[i]);
+            bad |= !(m <= 3.4028234663852886e38f);
+            amax[t] = fmaxf(amax[t], m);
+          }
         }
       }
+    } else if (tid == 0) {
+#pragma unroll
+      for (int t = 0; t < MT; ++t) amax[t] = amax_in[t];  // reduced below like the others
     }
     if (bad) record_status(kStatusNonfinite);
 #pragma unroll
@@ -205,6 +263,9 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(
   __syncthreads();
 
   // ---------------------------------------------------------------- stream the weights
+  float ymax[MT];  // largest |y| this thread stored, per token
+#pragma unroll
+  for (int t = 0; t < MT; ++t) ymax[t] = 0.0f;
   const int LPR = 1 << lpr_log2;
   const int RPW = 32 >> lpr_log2;
   const int sub = lane & (LPR - 1);
@@ -270,6 +331,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(
             static_cast<int*>(y)[o] = a;
           } else {
             const float v = __fmul_rn(__int2float_rn(a), sh.f[t]);
+            ymax[t] = fmaxf(ymax[t], stored_mag<OM>(v));
             if (OM == kOf32) static_cast<float*>(y)[o] = v;
             else static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(v);
           }
@@ -346,6 +408,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(
               static_cast<int*>(y)[o] = a;
             } else {
               const float v = __fmul_rn(__int2float_rn(a), sh.f[t]);
+              ymax[t] = fmaxf(ymax[t], stored_mag<OM>(v));
               if (OM == kOf32) static_cast<float*>(y)[o] = v;
               else static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(v);
             }
@@ -354,6 +417,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(
       }
     }
   }
+  if (OM != kOi32 && amax_out != nullptr) block_amax_out<MT>(ymax, sh, amax_out);
 }
 
 }  // namespace bl
