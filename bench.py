@@ -367,6 +367,30 @@ def sweep_3b_figures(bl, device, hbm_peak: float, Ms=(1, 16, 64), blocks: int = 
                                             "act quant once per input + 1 tensor-core kernel"}}
 
 
+def decode3_figure(bl, name: str, M: int, device, hbm_peak: float):
+    """bitlinear_forward_base3 (5 trits per byte) on one decode shape, timed like
+    decode_figure over rotated copies of the base-3 weights."""
+    wl = syn.WORKLOADS[name]
+    N, K = wl["N"], wl["K"]
+    w3_bytes = N * bl.base3_row_bytes(K)
+    copies = max(2, math.ceil(2 * L2_BYTES / w3_bytes))
+    packed, gamma = packed_copies(bl, name, device, 1)[0]
+    p3 = bl.pack_base3(packed)
+    ws = [p3] + [p3.clone() for _ in range(copies - 1)]
+    xs = act_copies(name, M, device, min(copies, 8))
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+    calls = [(lambda i=i: bl.forward_base3(xs[i % len(xs)], ws[i], gamma, y=y))
+             for i in range(copies)]
+    calls[0]()
+    torch.cuda.synchronize()
+    ms = statistics.mean(time_in_graph(calls))
+    alg = w3_bytes + M * K * 2 + M * N * 2
+    gbs = alg / (ms * 1e-3) / 1e9
+    return {"workload": name, "M": M, "kernel": "gemv3 (base-3)", "ms": ms, "GBps": gbs,
+            "frac_hbm": gbs / hbm_peak, "weight_bytes": w3_bytes,
+            "weight_bytes_2bit": N * K // 4, "weight_copies": copies}
+
+
 # LLaMA-70B-style layer matrices (out x in) and how many of each one layer holds; 80 layers.
 WQ_70B_SHAPES = [(8192, 8192, 2), (1024, 8192, 2), (28672, 8192, 3)]
 WQ_70B_LAYERS = 80
@@ -565,6 +589,11 @@ def main():
                                          ("70b_down_28672x8192", 176),
                                          ("700m_up_1536x4096", 1), ("700m_up_1536x4096", 4),
                                          ("700m_up_1536x4096", 16)]]
+        others["decode_base3"] = [decode3_figure(bl, n, m, device, hbm_peak)
+                                  for n, m in [("70b_up_8192x28672", 1),
+                                               ("70b_down_28672x8192", 1),
+                                               ("70b_up_8192x28672", 4),
+                                               ("700m_up_1536x4096", 1)]]
         others["weight_quant_70b"] = weight_quant_figures(bl, device, hbm_peak)
         others["sweep_3b_26_layers"] = sweep_3b_figures(bl, device, hbm_peak)
     roofline["others"] = others

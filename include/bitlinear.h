@@ -201,6 +201,29 @@ bl_status bitlinear_chain_forward(const void* x, int x_dtype, int M, const bl_la
                                   int L, void* y, int y_dtype, void* ws, size_t ws_bytes,
                                   void* stream);
 
+/* Base-3 weight format (hackerpaper HN page, thread 3: five ternary digits fit a byte,
+ * 3^5 = 243 <= 256): 1.6 bits per weight, 0.8 of the 2-bit format's bytes, for the
+ * bandwidth-bound decode path. Row n occupies bitlinear_base3_row_bytes(K) =
+ * ceil(K/80)*16 bytes at n times that; in each 16-byte chunk j of a row, byte i holds the
+ * trits k = 80 j + 16 p + i (p = 0..4; past K they are 0) as B = ceil(256 v / 243), where
+ * v = sum_p (c_p + 1) 3^(4-p). The digits come back as floor(B 3^(p+1) / 256) mod 3.
+ * Pure host function; 0 for K that the library rejects. */
+size_t bitlinear_base3_row_bytes(int K);
+
+/* Converts packed weights from the 2-bit format (bitlinear_quantize_weights) to the base-3
+ * format: the same codes, bit for bit.
+ *   packed   device [N][K/4].   packed3  device [N][bitlinear_base3_row_bytes(K)], written. */
+bl_status bitlinear_pack_base3(const uint8_t* packed, int N, int K, uint8_t* packed3,
+                               void* stream);
+
+/* bitlinear_forward on base-3 weights, for decode batches of M <= 4 tokens (a CUDA-core
+ * GEMV that quantizes x in its prologue and decodes five trits per byte with multiplies
+ * by 3). Same arguments and bits as bitlinear_forward; no workspace.
+ * BL_ERR_UNSUPPORTED_SHAPE for M > 4 or M * ceil(K/80) * 80 above 200 KB. */
+bl_status bitlinear_forward_base3(const void* x, int x_dtype, const uint8_t* packed3,
+                                  const float* gamma, void* y, int y_dtype, int M, int N, int K,
+                                  void* stream);
+
 /* The integer stage alone (test hook, same kernels as bitlinear_forward):
  * acc[t,n] = sum_k c[n,k] * xq[t,k].
  *   xq      device, [M][K] int8 (values in [-127, 127]).

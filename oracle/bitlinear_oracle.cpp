@@ -221,6 +221,62 @@ int oracle_unpack(const uint8_t* packed, int64_t N, int64_t K, int8_t* codes) {
   return 0;
 }
 
+// ---------------------------------------------------------------------------------------
+// Base-3 packing, 5 trits per byte (hackerpaper HN page, thread 3: 3^5 = 243 <= 256, so
+// five ternary digits fit a byte, 1.6 bits per weight instead of 2).
+//
+// Layout (the library's base-3 format): row n of W[N][K] occupies R = ceil(K / 80) * 16
+// bytes at byte offset n * R, in 16-byte chunks of 80 trits. Byte i (0..15) of chunk j
+// holds the five trits k = 80 j + 16 p + i, p = 0..4 (trits past K are 0). With
+// u_p = c_p + 1 in {0, 1, 2}, the byte stores the base-3 number v = sum_p u_p 3^(4 - p)
+// (u_0 the leading digit) as the fixed-point value B = ceil(256 v / 243), in 0..255.
+// Decoding: u_p = floor(B 3^(p+1) / 256) mod 3, exactly, for every v in 0..242.
+
+// Bytes per row of the base-3 format.
+int64_t oracle_base3_row_bytes(int64_t K) { return (K + 79) / 80 * 16; }
+
+// codes [N][K] int8 in {-1,0,1} -> packed3 [N][R] (R = oracle_base3_row_bytes(K)).
+void oracle_pack_base3(const int8_t* codes, int64_t N, int64_t K, uint8_t* packed3) {
+  const int64_t R = oracle_base3_row_bytes(K);
+  for (int64_t n = 0; n < N; ++n) {
+    for (int64_t j = 0; j < R / 16; ++j) {
+      for (int i = 0; i < 16; ++i) {
+        int64_t v = 0;
+        for (int p = 0; p < 5; ++p) {
+          const int64_t k = 80 * j + 16 * p + i;
+          const int u = (k < K) ? codes[n * K + k] + 1 : 1;
+          v = 3 * v + u;  // u_0 ends up as the leading digit
+        }
+        packed3[n * R + 16 * j + i] = static_cast<uint8_t>((256 * v + 242) / 243);
+      }
+    }
+  }
+}
+
+// packed3 [N][R] -> codes [N][K]. Returns 0, or 1 if a decoded byte is not the encoding of
+// any v (the byte is not ceil(256 v / 243) of its decoded v) or a trit past K is non-zero.
+int oracle_unpack_base3(const uint8_t* packed3, int64_t N, int64_t K, int8_t* codes) {
+  const int64_t R = oracle_base3_row_bytes(K);
+  for (int64_t n = 0; n < N; ++n) {
+    for (int64_t j = 0; j < R / 16; ++j) {
+      for (int i = 0; i < 16; ++i) {
+        const int64_t B = packed3[n * R + 16 * j + i];
+        int64_t v = 0;
+        int64_t pow3 = 3;
+        for (int p = 0; p < 5; ++p, pow3 *= 3) {
+          const int u = static_cast<int>((B * pow3 / 256) % 3);
+          v = 3 * v + u;
+          const int64_t k = 80 * j + 16 * p + i;
+          if (k < K) codes[n * K + k] = static_cast<int8_t>(u - 1);
+          else if (u != 1) return 1;
+        }
+        if ((256 * v + 242) / 243 != B) return 1;
+      }
+    }
+  }
+  return 0;
+}
+
 // Steps X1+X2: per-token absmax int8 quantization (8-bit activations, LIT-380
 // bullet 1). a_t = max_k |x[t,k]|; r_t = 127 / a_t (fp32); q = clip(rne(x * r_t), -127, 127);
 // s_t = a_t / 127 (fp32). A zero row gives q = 0 and s_t = 0; an exactly-zero element

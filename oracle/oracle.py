@@ -53,6 +53,12 @@ def lib() -> ctypes.CDLL:
         _lib.oracle_unpack.restype = i32
         _lib.oracle_quantize_acts.argtypes = [p, i32, i64, i64, p, p]
         _lib.oracle_quantize_acts.restype = i32
+        _lib.oracle_base3_row_bytes.argtypes = [i64]
+        _lib.oracle_base3_row_bytes.restype = i64
+        _lib.oracle_pack_base3.argtypes = [p, i64, i64, p]
+        _lib.oracle_pack_base3.restype = None
+        _lib.oracle_unpack_base3.argtypes = [p, i64, i64, p]
+        _lib.oracle_unpack_base3.restype = i32
         _lib.oracle_abs_buckets.argtypes = [p, i32, i64, p]
         _lib.oracle_abs_buckets.restype = i32
         _lib.oracle_absmean_from_buckets.argtypes = [p, i64, p]
@@ -93,6 +99,30 @@ def absmean(W: np.ndarray) -> np.float32:
     if rc != 0:
         raise ValueError("non-finite weight")
     return out[0]
+
+
+def base3_row_bytes(K: int) -> int:
+    """Bytes per row of the base-3 (5 trits per byte) format: ceil(K / 80) * 16."""
+    return int(lib().oracle_base3_row_bytes(int(K)))
+
+
+def pack_base3(codes: np.ndarray) -> np.ndarray:
+    """int8 codes [N][K] -> base-3 bytes [N][ceil(K/80)*16] (5 trits per byte)."""
+    codes = np.ascontiguousarray(codes, dtype=np.int8)
+    N, K = codes.shape
+    out = np.zeros((N, base3_row_bytes(K)), np.uint8)
+    lib().oracle_pack_base3(_ptr(codes), N, K, _ptr(out))
+    return out
+
+
+def unpack_base3(packed3: np.ndarray, K: int) -> np.ndarray:
+    packed3 = np.ascontiguousarray(packed3, dtype=np.uint8)
+    N = packed3.shape[0]
+    assert packed3.shape[1] == base3_row_bytes(K)
+    codes = np.zeros((N, K), np.int8)
+    if lib().oracle_unpack_base3(_ptr(packed3), N, K, codes.ctypes.data) != 0:
+        raise ValueError("bytes that no trit group encodes")
+    return codes
 
 
 def abs_buckets(W: np.ndarray) -> np.ndarray:

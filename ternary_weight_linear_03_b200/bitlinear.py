@@ -26,7 +26,8 @@ EXPORTS = (
     "bitlinear_workspace_size", "bitlinear_quantize_weights", "bitlinear_quantize_acts",
     "bitlinear_weight_abssum", "bitlinear_quantize_weights_from_abssum", "bitlinear_act_absmax",
     "bitlinear_quantize_acts_absmax", "bitlinear_rescale", "bitlinear_chain_workspace_size",
-    "bitlinear_chain_forward",
+    "bitlinear_chain_forward", "bitlinear_base3_row_bytes", "bitlinear_pack_base3",
+    "bitlinear_forward_base3",
     "bitlinear_forward", "bitlinear_forward_noalloc", "bitlinear_contract_i32",
     "bitlinear_get_device_status",
     "bitlinear_debug_timeout_probe", "bitlinear_debug_plan", "bitlinear_status_string",
@@ -80,6 +81,12 @@ def load_library() -> ctypes.CDLL:
     lib.bitlinear_chain_workspace_size.restype = sz
     lib.bitlinear_chain_forward.argtypes = [p, i, i, ctypes.POINTER(Layer), i, p, i, p, sz, p]
     lib.bitlinear_chain_forward.restype = i
+    lib.bitlinear_base3_row_bytes.argtypes = [i]
+    lib.bitlinear_base3_row_bytes.restype = sz
+    lib.bitlinear_pack_base3.argtypes = [p, i, i, p, p]
+    lib.bitlinear_pack_base3.restype = i
+    lib.bitlinear_forward_base3.argtypes = [p, i, p, p, p, i, i, i, i, p]
+    lib.bitlinear_forward_base3.restype = i
     lib.bitlinear_forward.argtypes = [p, i, p, p, p, i, i, i, i, p, sz, p]
     lib.bitlinear_forward.restype = i
     lib.bitlinear_forward_noalloc.argtypes = [p, i, p, p, p, i, i, i, i, p]
@@ -279,6 +286,37 @@ def chain_forward(x: torch.Tensor, layers, out_dtype: torch.dtype = torch.bfloat
     _check(lib.bitlinear_chain_forward(_dev(x, "x"), _dtype_code(x), M, arr, len(layers),
                                        _dev(y, "y"), _dtype_code(y), _dev(ws, "ws"), ws.numel(),
                                        _stream(stream)), "bitlinear_chain_forward")
+    return y
+
+
+def base3_row_bytes(K: int) -> int:
+    return int(load_library().bitlinear_base3_row_bytes(K))
+
+
+def pack_base3(packed: torch.Tensor, stream=None) -> torch.Tensor:
+    """2-bit packed weights [N][K/4] -> base-3 [N][ceil(K/80)*16] (same codes)."""
+    lib = load_library()
+    N, K = packed.shape[0], packed.shape[1] * 4
+    out = torch.empty((N, base3_row_bytes(K)), dtype=torch.uint8, device=packed.device)
+    _check(lib.bitlinear_pack_base3(_dev(packed, "packed"), N, K, _dev(out, "packed3"),
+                                    _stream(stream)), "bitlinear_pack_base3")
+    return out
+
+
+def forward_base3(x: torch.Tensor, packed3: torch.Tensor, gamma: torch.Tensor,
+                  out_dtype: torch.dtype = torch.bfloat16, y: torch.Tensor | None = None,
+                  stream=None) -> torch.Tensor:
+    """BitLinear forward on base-3 weights (M <= 4 tokens)."""
+    lib = load_library()
+    M, K = x.shape
+    N = packed3.shape[0]
+    if packed3.shape[1] != base3_row_bytes(K):
+        raise ValueError("packed3 must be [N][ceil(K/80)*16]")
+    if y is None:
+        y = torch.empty((M, N), dtype=out_dtype, device=x.device)
+    _check(lib.bitlinear_forward_base3(
+        _dev(x, "x"), _dtype_code(x), _dev(packed3, "packed3"), _dev(gamma, "gamma"),
+        _dev(y, "y"), _dtype_code(y), M, N, K, _stream(stream)), "bitlinear_forward_base3")
     return y
 
 

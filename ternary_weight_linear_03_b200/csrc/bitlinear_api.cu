@@ -18,6 +18,7 @@
 #include "gemm_skinny.cuh"
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
+#include "gemv3.cuh"
 #include "per_device.h"
 #include "rescale.cuh"
 #include "weight_quant.cuh"
@@ -295,6 +296,42 @@ bl_status launch_gemv_x(const void* x, const uint8_t* packed, const float* gamma
     case BL_BF16: return launch_gemv_m<XM, bl::kObf16>(x, packed, gamma, y, M, N, K, s, o);
     case BL_I32: return launch_gemv_m<XM, bl::kOi32>(x, packed, gamma, y, M, N, K, s, o);
     default: return BL_ERR_INVALID_ARG;
+  }
+}
+
+// ------------------------------------------------------------------ base-3 GEMV launch
+constexpr int kGemv3MaxM = 4;
+
+template <int MT, int XM, int OM>
+bl_status launch_gemv3_t(const void* x, const uint8_t* packed3, const float* gamma, void* y,
+                         int N, int K, cudaStream_t s) {
+  auto kern = bl::gemv3_kernel<MT, XM, OM>;
+  const int CH = (K + 79) / 80;
+  const int smem = MT * 80 * CH;
+  static bl::PerDevice configured;
+  if (!set_smem_limit_once(configured, kern, kGemvMaxSmem)) return BL_ERR_CUDA;
+  int blocks_per_sm = 1;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_per_sm, kern, bl::kGemv3Threads,
+                                                    smem) != cudaSuccess ||
+      blocks_per_sm < 1)
+    blocks_per_sm = 1;
+  const int lpr_log2 = choose_lpr_log2(CH);
+  const long long rows_per_block = static_cast<long long>(bl::kGemv3Warps) * (32 >> lpr_log2);
+  const long long need = (N + rows_per_block - 1) / rows_per_block;
+  const int grid = static_cast<int>(std::min<long long>(need, 1ll * blocks_per_sm * num_sms()));
+  kern<<<grid, bl::kGemv3Threads, smem, s>>>(x, packed3, gamma, y, N, K, lpr_log2);
+  return launch_status();
+}
+
+template <int XM, int OM>
+bl_status launch_gemv3_m(const void* x, const uint8_t* packed3, const float* gamma, void* y,
+                         int M, int N, int K, cudaStream_t s) {
+  switch (M) {
+    case 1: return launch_gemv3_t<1, XM, OM>(x, packed3, gamma, y, N, K, s);
+    case 2: return launch_gemv3_t<2, XM, OM>(x, packed3, gamma, y, N, K, s);
+    case 3: return launch_gemv3_t<3, XM, OM>(x, packed3, gamma, y, N, K, s);
+    case 4: return launch_gemv3_t<4, XM, OM>(x, packed3, gamma, y, N, K, s);
+    default: return BL_ERR_UNSUPPORTED_SHAPE;
   }
 }
 
@@ -857,6 +894,43 @@ bl_status bitlinear_contract_i32(const int8_t* xq, const uint8_t* packed, int32_
   if (M <= kSkinnyMaxM)
     return launch_skinny(xq, packed, w.rowsum, nullptr, nullptr, acc, BL_I32, M, N, K, ws, s);
   return launch_gemm(xq, packed, w.rowsum, nullptr, nullptr, acc, BL_I32, M, N, K, s);
+}
+
+size_t bitlinear_base3_row_bytes(int K) {
+  if (K < 64 || K % 64 != 0) return 0;
+  return static_cast<size_t>((K + 79) / 80) * 16;
+}
+
+bl_status bitlinear_pack_base3(const uint8_t* packed, int N, int K, uint8_t* packed3,
+                               void* stream) {
+  if (!packed || !packed3) return BL_ERR_INVALID_ARG;
+  if (!shape_ok(1, N, K)) return BL_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(packed) || !aligned16(packed3)) return BL_ERR_MISALIGNED;
+  const long long chunks = static_cast<long long>(N) * ((K + 79) / 80);
+  const int grid = static_cast<int>(
+      std::max<long long>(1, std::min<long long>((chunks + 255) / 256, 16ll * num_sms())));
+  bl::pack_base3_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const uint32_t*>(packed), reinterpret_cast<uint4*>(packed3), N, K);
+  return launch_status();
+}
+
+bl_status bitlinear_forward_base3(const void* x, int x_dtype, const uint8_t* packed3,
+                                  const float* gamma, void* y, int y_dtype, int M, int N, int K,
+                                  void* stream) {
+  if (!x || !packed3 || !gamma || !y) return BL_ERR_INVALID_ARG;
+  if (x_dtype != BL_F32 && x_dtype != BL_BF16) return BL_ERR_INVALID_ARG;
+  if (y_dtype != BL_F32 && y_dtype != BL_BF16) return BL_ERR_INVALID_ARG;
+  if (!shape_ok(M, N, K) || M > kGemv3MaxM ||
+      static_cast<long long>(M) * 80 * ((K + 79) / 80) > kGemvMaxSmem)
+    return BL_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(x) || !aligned16(packed3) || !aligned16(gamma) || !aligned16(y))
+    return BL_ERR_MISALIGNED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (x_dtype == BL_BF16)
+    return (y_dtype == BL_F32) ? launch_gemv3_m<bl::kXbf16, bl::kOf32>(x, packed3, gamma, y, M, N, K, s)
+                               : launch_gemv3_m<bl::kXbf16, bl::kObf16>(x, packed3, gamma, y, M, N, K, s);
+  return (y_dtype == BL_F32) ? launch_gemv3_m<bl::kXf32, bl::kOf32>(x, packed3, gamma, y, M, N, K, s)
+                             : launch_gemv3_m<bl::kXf32, bl::kObf16>(x, packed3, gamma, y, M, N, K, s);
 }
 
 bl_status bitlinear_get_device_status(void* stream) {

@@ -342,3 +342,61 @@ def test_quantize_acts_absmax_closed_form():
     q, s = orc.quantize_acts_absmax(x, np.array([2.0], np.float32))
     np.testing.assert_array_equal(q[0, :8], [64, 127, 127, -127, 0, 32, -64, 95])
     assert s[0] == np.float32(2.0) / np.float32(127.0)
+
+
+# ----------------------------------------------------------------------------- base 3
+
+
+def test_base3_every_trit_group_encodes_to_its_fixed_point_byte():
+    """All 3^5 groups of five trits: the byte is ceil(256 v / 243) of the group's base-3
+    value v (u_0 leading, u = c + 1), computed here with Python integers; the 243 bytes
+    are distinct and rise with v (so the encoding is injective), and unpacking restores
+    every group."""
+    import itertools
+    groups = list(itertools.product((-1, 0, 1), repeat=5))
+    codes = np.zeros((len(groups), 80), np.int8)
+    for r, g in enumerate(groups):
+        for p, c in enumerate(g):
+            codes[r, 16 * p] = c  # byte 0 of the chunk holds trits 0, 16, 32, 48, 64
+    packed = orc.pack_base3(codes)
+    assert packed.shape == (243, 16)
+    vs = [sum((c + 1) * 3 ** (4 - p) for p, c in enumerate(g)) for g in groups]
+    want = [-(-256 * v // 243) for v in vs]
+    np.testing.assert_array_equal(packed[:, 0], want)
+    order = np.argsort(vs)
+    assert np.all(np.diff(packed[order, 0].astype(int)) > 0)
+    np.testing.assert_array_equal(orc.unpack_base3(packed, 80), codes)
+
+
+def test_base3_closed_form_bytes_and_positions():
+    """All +1 -> 255, all 0 -> 128, all -1 -> 0 (v = 242, 121, 0); one +1 among zeros at
+    digit p gives v = 121 + 3^(4-p) = 202, 148, 130, 124, 122: bytes ceil(256 v / 243) =
+    213, 156, 137, 131, 129 for p = 0..4 (e.g. 256 * 148 / 243 = 155.9), in byte
+    i of chunk j for trit k = 80 j + 16 p + i."""
+    K = 160
+    for c, b in ((1, 255), (0, 128), (-1, 0)):
+        np.testing.assert_array_equal(orc.pack_base3(np.full((1, K), c, np.int8)), b)
+    for p, b in enumerate((213, 156, 137, 131, 129)):
+        for j, i in ((0, 0), (1, 7), (1, 15)):
+            codes = np.zeros((1, K), np.int8)
+            codes[0, 80 * j + 16 * p + i] = 1
+            packed = orc.pack_base3(codes)
+            expect = np.full(32, 128, np.uint8)
+            expect[16 * j + i] = b
+            np.testing.assert_array_equal(packed[0], expect)
+
+
+def test_base3_ragged_rows_pad_with_zero_trits():
+    """K not a multiple of 80: the last chunk's missing trits are zeros (u = 1), the row
+    size is ceil(K / 80) * 16 bytes (1648 for K = 8192, 0.805 of the 2-bit 2048), and
+    non-zero padding is rejected on unpacking."""
+    assert orc.base3_row_bytes(8192) == 1648 and orc.base3_row_bytes(80) == 16
+    assert orc.base3_row_bytes(64) == 16 and orc.base3_row_bytes(28672) == 5744
+    rng = np.random.default_rng(21)
+    codes = rng.integers(-1, 2, size=(9, 192)).astype(np.int8)
+    packed = orc.pack_base3(codes)
+    np.testing.assert_array_equal(orc.unpack_base3(packed, 192), codes)
+    bad = packed.copy()
+    bad[0, 16 * 2 + 0] = 255  # chunk 2 byte 0 holds trits 160, 176 (real) and 192.. (padding)
+    with pytest.raises(ValueError):
+        orc.unpack_base3(bad, 192)
