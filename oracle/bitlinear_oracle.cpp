@@ -277,6 +277,61 @@ int oracle_unpack_base3(const uint8_t* packed3, int64_t N, int64_t K, int8_t* co
   return 0;
 }
 
+// ---------------------------------------------------------------------------------------
+// BitLinear backward for quantization-aware training with the straight-through estimator
+// (hackerpaper HN page, thread 21: the rounding steps are passed straight through in the
+// backward pass; LIT-380 bullet 1: the model is trained with these quantizers in place).
+// The forward is y = X~ W~^T with the dequantized operands X~[t,k] = q[t,k] s_t and
+// W~[n,k] = gamma c[n,k]; the estimator treats both quantizers as the identity, so for an
+// upstream gradient G = dL/dy [M][N]:
+//   dL/dx = G W~       -> grad_x[t,k] = gamma * sum_n G[t,n] c[n,k]
+//   dL/dW = G^T X~     -> grad_w[n,k] = sum_t G[t,n] X~[t,k]
+// G is bf16 (dtype 1) or fp32 (dtype 0). X~ is taken as the library holds it, in bf16:
+// X~[t,k] = bf16(fl32(q[t,k] * s_t)) (round half to even). Sums are formed in double
+// (every product is exact there), the results are doubles.
+
+// dequantized activations X~ [M][K] as bf16 bit patterns
+void oracle_dequant_acts_bf16(const int8_t* q, const float* scale, int64_t M, int64_t K,
+                              uint16_t* out) {
+  for (int64_t t = 0; t < M; ++t) {
+    for (int64_t k = 0; k < K; ++k) {
+      const float v = static_cast<float>(q[t * K + k]) * scale[t];
+      uint32_t b = float_bits(v);
+      uint32_t lower = b & 0xffffu, upper = b >> 16;
+      if (lower > 0x8000u || (lower == 0x8000u && (upper & 1u))) upper += 1;
+      out[t * K + k] = static_cast<uint16_t>(upper);
+    }
+  }
+}
+
+void oracle_ste_grad_x(const void* G, int dtype, const int8_t* codes, float gamma, int64_t M,
+                       int64_t N, int64_t K, double* grad_x) {
+  for (int64_t t = 0; t < M; ++t) {
+    for (int64_t k = 0; k < K; ++k) {
+      double s = 0.0;
+      for (int64_t n = 0; n < N; ++n) {
+        const int8_t c = codes[n * K + k];
+        if (c == 1) s += static_cast<double>(load_value(G, dtype, t * N + n));
+        else if (c == -1) s -= static_cast<double>(load_value(G, dtype, t * N + n));
+      }
+      grad_x[t * K + k] = static_cast<double>(gamma) * s;
+    }
+  }
+}
+
+void oracle_ste_grad_w(const void* G, int dtype, const uint16_t* xt_bf16, int64_t M, int64_t N,
+                       int64_t K, double* grad_w) {
+  for (int64_t n = 0; n < N; ++n) {
+    for (int64_t k = 0; k < K; ++k) {
+      double s = 0.0;
+      for (int64_t t = 0; t < M; ++t)
+        s += static_cast<double>(load_value(G, dtype, t * N + n)) *
+             static_cast<double>(load_value(xt_bf16, 1, t * K + k));
+      grad_w[n * K + k] = s;
+    }
+  }
+}
+
 // Steps X1+X2: per-token absmax int8 quantization (8-bit activations, LIT-380
 // bullet 1). a_t = max_k |x[t,k]|; r_t = 127 / a_t (fp32); q = clip(rne(x * r_t), -127, 127);
 // s_t = a_t / 127 (fp32). A zero row gives q = 0 and s_t = 0; an exactly-zero element

@@ -59,6 +59,12 @@ def lib() -> ctypes.CDLL:
         _lib.oracle_pack_base3.restype = None
         _lib.oracle_unpack_base3.argtypes = [p, i64, i64, p]
         _lib.oracle_unpack_base3.restype = i32
+        _lib.oracle_dequant_acts_bf16.argtypes = [p, p, i64, i64, p]
+        _lib.oracle_dequant_acts_bf16.restype = None
+        _lib.oracle_ste_grad_x.argtypes = [p, i32, p, f32, i64, i64, i64, p]
+        _lib.oracle_ste_grad_x.restype = None
+        _lib.oracle_ste_grad_w.argtypes = [p, i32, p, i64, i64, i64, p]
+        _lib.oracle_ste_grad_w.restype = None
         _lib.oracle_abs_buckets.argtypes = [p, i32, i64, p]
         _lib.oracle_abs_buckets.restype = i32
         _lib.oracle_absmean_from_buckets.argtypes = [p, i64, p]
@@ -123,6 +129,40 @@ def unpack_base3(packed3: np.ndarray, K: int) -> np.ndarray:
     if lib().oracle_unpack_base3(_ptr(packed3), N, K, codes.ctypes.data) != 0:
         raise ValueError("bytes that no trit group encodes")
     return codes
+
+
+def dequant_acts_bf16(q: np.ndarray, scale: np.ndarray) -> np.ndarray:
+    """X~ = bf16(fl32(q * s_t)) as bf16 bit patterns (uint16 [M][K])."""
+    q = np.ascontiguousarray(q, dtype=np.int8)
+    scale = np.ascontiguousarray(scale, dtype=np.float32)
+    M, K = q.shape
+    out = np.zeros((M, K), np.uint16)
+    lib().oracle_dequant_acts_bf16(_ptr(q), _ptr(scale), M, K, _ptr(out))
+    return out
+
+
+def ste_grad_x(G: np.ndarray, codes: np.ndarray, gamma: float) -> np.ndarray:
+    """Straight-through dL/dx = gamma * G C, float64 [M][K] (G fp32 or bf16 bits)."""
+    G, dt = _as_input(G)
+    codes = np.ascontiguousarray(codes, dtype=np.int8)
+    M, N = G.shape
+    K = codes.shape[1]
+    assert codes.shape[0] == N
+    out = np.zeros((M, K), np.float64)
+    lib().oracle_ste_grad_x(_ptr(G), dt, _ptr(codes), float(gamma), M, N, K, _ptr(out))
+    return out
+
+
+def ste_grad_w(G: np.ndarray, xt_bf16: np.ndarray) -> np.ndarray:
+    """Straight-through dL/dW = G^T X~, float64 [N][K] (X~ as bf16 bits [M][K])."""
+    G, dt = _as_input(G)
+    xt = np.ascontiguousarray(xt_bf16, dtype=np.uint16)
+    M, N = G.shape
+    K = xt.shape[1]
+    assert xt.shape[0] == M
+    out = np.zeros((N, K), np.float64)
+    lib().oracle_ste_grad_w(_ptr(G), dt, _ptr(xt), M, N, K, _ptr(out))
+    return out
 
 
 def abs_buckets(W: np.ndarray) -> np.ndarray:

@@ -400,3 +400,92 @@ def test_base3_ragged_rows_pad_with_zero_trits():
     bad[0, 16 * 2 + 0] = 255  # chunk 2 byte 0 holds trits 160, 176 (real) and 192.. (padding)
     with pytest.raises(ValueError):
         orc.unpack_base3(bad, 192)
+
+
+# ----------------------------------------------------------------------------- backward
+
+
+def _bilinear_loss(G, Xt, Wt):
+    """L = sum_{t,n} G[t,n] (Xt Wt^T)[t,n] by explicit loops in float64 (tiny sizes)."""
+    M, K = Xt.shape
+    N = Wt.shape[0]
+    total = 0.0
+    for t in range(M):
+        for n in range(N):
+            total += float(G[t, n]) * sum(float(Xt[t, k]) * float(Wt[n, k]) for k in range(K))
+    return total
+
+
+def _bf16_bits_to_f64(b):
+    return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def test_ste_gradients_are_the_bilinear_derivatives():
+    """The straight-through gradients are the partial derivatives of the bilinear
+    surrogate L = sum G * (X~ W~^T) in X~ and W~: unit perturbations of single entries, by
+    brute force, change L by exactly grad_x[t,k] (as X~ moves) and grad_w[n,k] (as W~
+    moves); the loss is linear in each, so the difference quotient is exact."""
+    rng = np.random.default_rng(31)
+    M, N, K = 3, 4, 16
+    G = (rng.standard_normal((M, N))).astype(np.float32)
+    codes = rng.integers(-1, 2, size=(N, K)).astype(np.int8)
+    gamma = np.float32(0.0625)
+    q = rng.integers(-127, 128, size=(M, K)).astype(np.int8)
+    s = np.float32([0.5, 0.25, 0.125])  # q * s exact in bf16? (|q| <= 127: 7 bits) yes
+    xt_bits = orc.dequant_acts_bf16(q, s)
+    Xt = _bf16_bits_to_f64(xt_bits)
+    Wt = codes.astype(np.float64) * float(gamma)
+    gx = orc.ste_grad_x(G, codes, gamma)
+    gw = orc.ste_grad_w(G, xt_bits)
+    base = _bilinear_loss(G, Xt, Wt)
+    for (t, k) in [(0, 0), (2, 15), (1, 7)]:
+        X2 = Xt.copy()
+        X2[t, k] += 1.0
+        assert _bilinear_loss(G, X2, Wt) - base == pytest.approx(gx[t, k], rel=1e-12, abs=1e-12)
+    for (n, k) in [(0, 0), (3, 15), (2, 9)]:
+        W2 = Wt.copy()
+        W2[n, k] += 1.0
+        assert _bilinear_loss(G, Xt, W2) - base == pytest.approx(gw[n, k], rel=1e-12, abs=1e-12)
+
+
+def test_ste_gradients_special_cases_and_adjoint_identity():
+    """One-hot G picks a weight row (grad_x = gamma c[n0]) and an activation row (grad_w
+    row n0 = X~[t0]); and both gradients pair with the forward: sum grad_x * X~ =
+    sum G * y = sum grad_w * W~ (y = X~ W~^T in float64)."""
+    rng = np.random.default_rng(32)
+    M, N, K = 5, 7, 64
+    codes = rng.integers(-1, 2, size=(N, K)).astype(np.int8)
+    gamma = np.float32(0.013)
+    x = rng.standard_normal((M, K)).astype(np.float32)
+    q, s = orc.quantize_acts(x)
+    xt_bits = orc.dequant_acts_bf16(q, s)
+    Xt = _bf16_bits_to_f64(xt_bits)
+    G = np.zeros((M, N), np.float32)
+    G[2, 5] = 1.0
+    np.testing.assert_array_equal(orc.ste_grad_x(G, codes, gamma)[2],
+                                  float(gamma) * codes[5].astype(np.float64))
+    np.testing.assert_array_equal(orc.ste_grad_w(G, xt_bits)[5], Xt[2])
+    G = rng.standard_normal((M, N)).astype(np.float32)
+    gx = orc.ste_grad_x(G, codes, gamma)
+    gw = orc.ste_grad_w(G, xt_bits)
+    Wt = codes.astype(np.float64) * float(gamma)
+    y = Xt @ Wt.T
+    a = float(np.sum(gx * Xt))
+    b = float(np.sum(G.astype(np.float64) * y))
+    c = float(np.sum(gw * Wt))
+    assert a == pytest.approx(b, rel=1e-12) and c == pytest.approx(b, rel=1e-12)
+    # bf16 G is read as its exact value
+    Gb = torch.from_numpy(G).bfloat16()
+    gb = orc.ste_grad_x(Gb.view(torch.int16).numpy().view(np.uint16), codes, gamma)
+    np.testing.assert_allclose(gb, orc.ste_grad_x(Gb.float().numpy(), codes, gamma), rtol=0, atol=0)
+
+
+def test_dequant_acts_bf16_rounds_half_to_even():
+    """X~ = bf16(fl32(q * s)) equals torch's own fp32 -> bf16 conversion (a library
+    routine, round half to even) for every q and three scales, the first with low bits
+    (2^-8 + 2^-9) that the 8-bit bf16 significand must round away."""
+    q = np.arange(-127, 128, dtype=np.int8).reshape(1, -1)[:, :240]
+    for s in (np.float32(1.0 + 2**-8 + 2**-9), np.float32(0.0123), np.float32(3.0)):
+        got = orc.dequant_acts_bf16(q, np.array([s], np.float32))
+        want = torch.from_numpy(q.astype(np.float32) * s).bfloat16()
+        np.testing.assert_array_equal(got, want.view(torch.int16).numpy().view(np.uint16))
