@@ -224,6 +224,37 @@ bl_status bitlinear_forward_base3(const void* x, int x_dtype, const uint8_t* pac
                                   const float* gamma, void* y, int y_dtype, int M, int N, int K,
                                   void* stream);
 
+/* The transposed 2-bit weights: row k of packedT [K][N/4] holds the trits W[., k] along n,
+ * in the packed format above. Input of bitlinear_backward's grad_x (its contraction runs
+ * over n). N % 64 == 0, else BL_ERR_UNSUPPORTED_SHAPE.
+ *   packed  device [N][K/4].   packedT  device [K][N/4], written. */
+bl_status bitlinear_pack_transpose(const uint8_t* packed, int N, int K, uint8_t* packedT,
+                                   void* stream);
+
+/* Workspace bytes of bitlinear_backward (0 for shapes it rejects). Pure host function. */
+size_t bitlinear_backward_workspace_size(int M, int N, int K);
+
+/* BitLinear backward for quantization-aware training with the straight-through
+ * estimator (hackerpaper HN page, thread 21: the quantizers' rounding passes gradients
+ * unchanged; LIT-380 bullet 1: b1.58 is trained with the quantizers in place). With the
+ * forward y = X~ W~^T, X~ = q s (per-token int8 activations), W~ = gamma c:
+ *   grad_x[t,k] = gamma * sum_n G[t,n] c[n,k]          (fp32 [M][K])
+ *   grad_w[n,k] = sum_t G[t,n] X~[t,k]                  (fp32 [N][K])
+ * where X~ is held in bf16, X~ = bf16(q * s), q and s the forward's quantization of x.
+ * Both run on the tcgen05 tensor cores as bf16 x bf16 -> fp32 contractions; products are
+ * exact, only the fp32 accumulation order differs from a sequential sum.
+ *   x        device [M][K] fp32 or bf16: the forward's input (needed for grad_w).
+ *   grad_y   device [M][N] bf16: dL/dy.
+ *   packedT  device [K][N/4] from bitlinear_pack_transpose (needed for grad_x).
+ *   gamma    device, one float (needed for grad_x).
+ *   grad_x   device [M][K] fp32, or NULL to skip.   grad_w  device [N][K] fp32, or NULL.
+ *   ws       device, bitlinear_backward_workspace_size(M, N, K) bytes (for grad_w).
+ * N % 64 == 0, else BL_ERR_UNSUPPORTED_SHAPE. */
+bl_status bitlinear_backward(const void* x, int x_dtype, const void* grad_y,
+                             const uint8_t* packedT, const float* gamma, float* grad_x,
+                             float* grad_w, int M, int N, int K, void* ws, size_t ws_bytes,
+                             void* stream);
+
 /* The integer stage alone (test hook, same kernels as bitlinear_forward):
  * acc[t,n] = sum_k c[n,k] * xq[t,k].
  *   xq      device, [M][K] int8 (values in [-127, 127]).

@@ -27,7 +27,8 @@ EXPORTS = (
     "bitlinear_weight_abssum", "bitlinear_quantize_weights_from_abssum", "bitlinear_act_absmax",
     "bitlinear_quantize_acts_absmax", "bitlinear_rescale", "bitlinear_chain_workspace_size",
     "bitlinear_chain_forward", "bitlinear_base3_row_bytes", "bitlinear_pack_base3",
-    "bitlinear_forward_base3",
+    "bitlinear_forward_base3", "bitlinear_pack_transpose", "bitlinear_backward_workspace_size",
+    "bitlinear_backward",
     "bitlinear_forward", "bitlinear_forward_noalloc", "bitlinear_contract_i32",
     "bitlinear_get_device_status",
     "bitlinear_debug_timeout_probe", "bitlinear_debug_plan", "bitlinear_status_string",
@@ -87,6 +88,12 @@ def load_library() -> ctypes.CDLL:
     lib.bitlinear_pack_base3.restype = i
     lib.bitlinear_forward_base3.argtypes = [p, i, p, p, p, i, i, i, i, p]
     lib.bitlinear_forward_base3.restype = i
+    lib.bitlinear_pack_transpose.argtypes = [p, i, i, p, p]
+    lib.bitlinear_pack_transpose.restype = i
+    lib.bitlinear_backward_workspace_size.argtypes = [i, i, i]
+    lib.bitlinear_backward_workspace_size.restype = sz
+    lib.bitlinear_backward.argtypes = [p, i, p, p, p, p, p, i, i, i, p, sz, p]
+    lib.bitlinear_backward.restype = i
     lib.bitlinear_forward.argtypes = [p, i, p, p, p, i, i, i, i, p, sz, p]
     lib.bitlinear_forward.restype = i
     lib.bitlinear_forward_noalloc.argtypes = [p, i, p, p, p, i, i, i, i, p]
@@ -318,6 +325,42 @@ def forward_base3(x: torch.Tensor, packed3: torch.Tensor, gamma: torch.Tensor,
         _dev(x, "x"), _dtype_code(x), _dev(packed3, "packed3"), _dev(gamma, "gamma"),
         _dev(y, "y"), _dtype_code(y), M, N, K, _stream(stream)), "bitlinear_forward_base3")
     return y
+
+
+def pack_transpose(packed: torch.Tensor, stream=None) -> torch.Tensor:
+    """2-bit weights [N][K/4] -> the transposed 2-bit weights [K][N/4] (N % 64 == 0)."""
+    lib = load_library()
+    N, K = packed.shape[0], packed.shape[1] * 4
+    out = torch.empty((K, N // 4), dtype=torch.uint8, device=packed.device)
+    _check(lib.bitlinear_pack_transpose(_dev(packed, "packed"), N, K, _dev(out, "packedT"),
+                                        _stream(stream)), "bitlinear_pack_transpose")
+    return out
+
+
+def backward(x: torch.Tensor, grad_y: torch.Tensor, packedT: torch.Tensor, gamma: torch.Tensor,
+             need_x: bool = True, need_w: bool = True, ws: torch.Tensor | None = None,
+             stream=None):
+    """Straight-through BitLinear backward: (grad_x fp32 [M][K] or None, grad_w fp32 [N][K]
+    or None) from the forward input x, grad_y bf16 [M][N] and the transposed weights."""
+    lib = load_library()
+    M, K = x.shape
+    N = grad_y.shape[1]
+    if grad_y.dtype != torch.bfloat16:
+        raise TypeError("grad_y must be bf16")
+    gx = torch.empty((M, K), dtype=torch.float32, device=x.device) if need_x else None
+    gw = torch.empty((N, K), dtype=torch.float32, device=x.device) if need_w else None
+    if ws is None and need_w:
+        n = int(lib.bitlinear_backward_workspace_size(M, N, K))
+        if n == 0:
+            raise BitLinearError(2, "bitlinear_backward_workspace_size")
+        ws = torch.empty(n, dtype=torch.uint8, device=x.device)
+    _check(lib.bitlinear_backward(
+        _dev(x, "x"), _dtype_code(x), _dev(grad_y, "grad_y"), _dev(packedT, "packedT"),
+        _dev(gamma, "gamma"), _dev(gx, "grad_x") if gx is not None else None,
+        _dev(gw, "grad_w") if gw is not None else None, M, N, K,
+        _dev(ws, "ws") if ws is not None else None, ws.numel() if ws is not None else 0,
+        _stream(stream)), "bitlinear_backward")
+    return gx, gw
 
 
 def forward(x: torch.Tensor, packed: torch.Tensor, gamma: torch.Tensor,

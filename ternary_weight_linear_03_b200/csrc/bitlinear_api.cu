@@ -15,6 +15,7 @@
 #include "../../include/bitlinear.h"
 #include "act_quant.cuh"
 #include "common.cuh"
+#include "gemm_bf16.cuh"
 #include "gemm_skinny.cuh"
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
@@ -215,6 +216,21 @@ bool make_map_u8(CUtensorMap* map, const void* base, uint64_t cols, uint64_t row
                         swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// bf16 2-D tensor [rows][cols] (row pitch cols * 2 bytes), box [box_rows][64], 128-byte
+// swizzle (64 bf16 = one swizzle row).
+bool make_map_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
+                   uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // ------------------------------------------------------------------ GEMV launch
@@ -718,6 +734,114 @@ bl_status bitlinear_forward(const void* x, int x_dtype, const uint8_t* packed,
   if (M <= kSkinnyMaxM)
     return launch_skinny(w.xq, packed, w.rowsum, w.scale, gamma, y, y_dtype, M, N, K, ws, s);
   return launch_gemm(w.xq, packed, w.rowsum, w.scale, gamma, y, y_dtype, M, N, K, s);
+}
+
+}  // extern "C"
+
+namespace {
+
+// ------------------------------------------------------------------ backward (STE)
+// D[r][c] = alpha * sum_j A[r][j] B[c][j]; A bf16 [R][J]; B bf16 [C][J] or packed trits
+// [C][J/4].
+template <bool kPacked>
+bl_status launch_gemm_bf16(const void* A, const void* B, const float* alpha, float* out, int R,
+                           int C, int J, cudaStream_t s) {
+  CUtensorMap map_a, map_b;
+  if (!make_map_bf16(&map_a, A, J, R, bl::bf::BM)) return BL_ERR_CUDA;
+  if (kPacked) {
+    if (!make_map_u8(&map_b, B, J / 4, C, J / 4, bl::bf::BKE / 4, bl::bf::BN, false))
+      return BL_ERR_CUDA;
+  } else if (!make_map_bf16(&map_b, B, J, C, bl::bf::BN)) {
+    return BL_ERR_CUDA;
+  }
+  auto kern = bl::gemm_bf16_kernel<kPacked>;
+  constexpr int kSmem = bl::bf::smem_bytes<kPacked>();
+  static bl::PerDevice configured;
+  if (!set_smem_limit_once(configured, kern, kSmem)) return BL_ERR_CUDA;
+  const long long tiles = static_cast<long long>((R + bl::bf::BM - 1) / bl::bf::BM) *
+                          ((C + bl::bf::BN - 1) / bl::bf::BN);
+  const int grid = static_cast<int>(std::min<long long>(tiles, num_sms()));
+  return launch_ex(kern, dim3(grid), dim3(bl::bf::THREADS), kSmem, s, false, map_a, map_b,
+                   alpha, out, R, C, J, kWaitLimitNs);
+}
+
+// Workspace of bitlinear_backward: [xq M*K][scale M][rowsum M][G^T N*Mp bf16][X~^T K*Mp bf16].
+struct BwdWs {
+  FwdWs f;
+  __nv_bfloat16* gT;
+  __nv_bfloat16* xT;
+  int Mp;
+  size_t bytes;
+};
+BwdWs bwd_ws_layout(void* base, int M, int N, int K) {
+  BwdWs w{};
+  w.f = fwd_ws_layout(base, M, K);
+  w.Mp = (M + 7) / 8 * 8;
+  char* p = static_cast<char*>(base) + w.f.bytes;
+  const size_t g = align_up(static_cast<size_t>(N) * w.Mp * 2, 256);
+  const size_t x = align_up(static_cast<size_t>(K) * w.Mp * 2, 256);
+  w.gT = reinterpret_cast<__nv_bfloat16*>(p);
+  w.xT = reinterpret_cast<__nv_bfloat16*>(p + g);
+  w.bytes = w.f.bytes + g + x;
+  return w;
+}
+
+int grid_for(long long work, int per_block) {
+  return static_cast<int>(std::max<long long>(
+      1, std::min<long long>((work + per_block - 1) / per_block, 16ll * num_sms())));
+}
+
+}  // namespace
+
+extern "C" {
+
+bl_status bitlinear_pack_transpose(const uint8_t* packed, int N, int K, uint8_t* packedT,
+                                   void* stream) {
+  if (!packed || !packedT) return BL_ERR_INVALID_ARG;
+  if (!shape_ok(1, N, K) || N % 64 != 0) return BL_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(packed) || !aligned16(packedT)) return BL_ERR_MISALIGNED;
+  bl::pack_transpose_kernel<<<grid_for(static_cast<long long>(N / 64) * (K / 64), 1), 256, 0,
+                              static_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const uint32_t*>(packed), reinterpret_cast<uint32_t*>(packedT), N, K);
+  return launch_status();
+}
+
+size_t bitlinear_backward_workspace_size(int M, int N, int K) {
+  if (!shape_ok(M, N, K) || N % 64 != 0) return 0;
+  return align_up(bwd_ws_layout(nullptr, M, N, K).bytes, 256);
+}
+
+bl_status bitlinear_backward(const void* x, int x_dtype, const void* grad_y,
+                             const uint8_t* packedT, const float* gamma, float* grad_x,
+                             float* grad_w, int M, int N, int K, void* ws, size_t ws_bytes,
+                             void* stream) {
+  if (!grad_y || (!grad_x && !grad_w)) return BL_ERR_INVALID_ARG;
+  if (grad_x && (!packedT || !gamma)) return BL_ERR_INVALID_ARG;
+  if (grad_w && (!x || !ws)) return BL_ERR_INVALID_ARG;
+  if (x_dtype != BL_F32 && x_dtype != BL_BF16) return BL_ERR_INVALID_ARG;
+  if (!shape_ok(M, N, K) || N % 64 != 0) return BL_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(grad_y) || (x && !aligned16(x)) || (packedT && !aligned16(packedT)) ||
+      (gamma && !aligned16(gamma)) || (grad_x && !aligned16(grad_x)) ||
+      (grad_w && !aligned16(grad_w)) || (ws && !aligned16(ws)))
+    return BL_ERR_MISALIGNED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (grad_w) {
+    const BwdWs w = bwd_ws_layout(ws, M, N, K);
+    if (ws_bytes < w.bytes) return BL_ERR_WORKSPACE;
+    bl_status st = launch_act_quant(x, x_dtype, M, K, w.f.xq, w.f.scale, nullptr, s);
+    if (st != BL_OK) return st;
+    const int tiles_g = ((w.Mp + 31) / 32) * ((N + 31) / 32);
+    bl::transpose_bf16_kernel<0><<<grid_for(tiles_g, 1), 256, 0, s>>>(grad_y, nullptr, w.gT, M,
+                                                                       N, w.Mp);
+    const int tiles_x = ((w.Mp + 31) / 32) * ((K + 31) / 32);
+    bl::transpose_bf16_kernel<1><<<grid_for(tiles_x, 1), 256, 0, s>>>(w.f.xq, w.f.scale, w.xT,
+                                                                       M, K, w.Mp);
+    if (launch_status() != BL_OK) return BL_ERR_CUDA;
+    st = launch_gemm_bf16<false>(w.gT, w.xT, nullptr, grad_w, N, K, w.Mp, s);
+    if (st != BL_OK) return st;
+  }
+  if (grad_x) return launch_gemm_bf16<true>(grad_y, packedT, gamma, grad_x, M, K, N, s);
+  return BL_OK;
 }
 
 }  // extern "C"
