@@ -239,6 +239,26 @@ def config_of(name: str, M: int, wl: dict, world: int) -> dict:
 # ----------------------------------------------------------------------------- GPU helpers
 
 
+def time_back_to_back(calls, reps: int = 5):
+    """Mean device time (ms) per call of a list of library calls run back to back: one CUDA
+    graph holding them all, replayed `reps` times between two events (the steady state of
+    a stream of such calls, inter-kernel gaps included)."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for c in calls:
+            c()
+    g.replay()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(reps):
+        g.replay()
+    e.record()
+    torch.cuda.synchronize()
+    del g
+    return s.elapsed_time(e) / (reps * len(calls))
+
+
 def time_in_graph(calls, reps: int = 3):
     """Per-call device times (ms) of a list of library calls: one CUDA graph with an event
     node before every call and after the last, replayed `reps` times; the times are those
@@ -301,7 +321,7 @@ def decode_figure(bl, name: str, M: int, device, hbm_peak: float, i8_peak: float
     for c in calls[:2]:
         c()
     torch.cuda.synchronize()
-    ms = statistics.mean(time_in_graph(calls))
+    ms = time_back_to_back(calls)
     alg_bytes = w_bytes + M * K * 2 + M * N * 2
     ops = 2.0 * M * N * K
     gbs = alg_bytes / (ms * 1e-3) / 1e9
@@ -340,8 +360,7 @@ def sweep_3b_figures(bl, device, hbm_peak: float, Ms=(1, 16, 64), blocks: int = 
         ws = bl.chain_workspace(M, chain, device)
         bl.chain_forward(x, chain, y=y, ws=ws)
         torch.cuda.synchronize()
-        ms_chain = statistics.mean(time_in_graph(
-            [lambda: bl.chain_forward(x, chain, y=y, ws=ws)] * 4))
+        ms_chain = time_back_to_back([lambda: bl.chain_forward(x, chain, y=y, ws=ws)] * 4)
         # unchained: separate forwards, each quantizing its input itself
         bufs = {-1: x}
         outs = [torch.empty((M, ly[0].shape[0]), dtype=torch.bfloat16, device=device)
@@ -355,7 +374,7 @@ def sweep_3b_figures(bl, device, hbm_peak: float, Ms=(1, 16, 64), blocks: int = 
 
         separate()
         torch.cuda.synchronize()
-        ms_sep = statistics.mean(time_in_graph([separate] * 2))
+        ms_sep = time_back_to_back([separate] * 2)
         gbs = w_bytes / (ms_chain * 1e-3) / 1e9
         rows.append({"M": M, "ms_per_sweep": ms_chain, "tokens_per_s": M / (ms_chain * 1e-3),
                      "GBps": gbs, "frac_hbm": gbs / hbm_peak,
@@ -383,7 +402,7 @@ def decode3_figure(bl, name: str, M: int, device, hbm_peak: float):
              for i in range(copies)]
     calls[0]()
     torch.cuda.synchronize()
-    ms = statistics.mean(time_in_graph(calls))
+    ms = time_back_to_back(calls)
     alg = w3_bytes + M * K * 2 + M * N * 2
     gbs = alg / (ms * 1e-3) / 1e9
     return {"workload": name, "M": M, "kernel": "gemv3 (base-3)", "ms": ms, "GBps": gbs,
@@ -411,7 +430,7 @@ def weight_quant_figures(bl, device, hbm_peak: float):
                  for W in Ws]
         calls[0]()
         torch.cuda.synchronize()
-        ms = statistics.mean(time_in_graph(calls))
+        ms = time_back_to_back(calls, reps=3)
         alg = n_bytes + N * K // 4
         gbs = alg / (ms * 1e-3) / 1e9
         rows.append({"shape": f"{N}x{K}", "per_layer": count, "ms": ms, "GBps": gbs,

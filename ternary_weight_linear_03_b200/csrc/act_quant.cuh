@@ -90,6 +90,8 @@ __global__ void __launch_bounds__(kAqThreads) act_quant_kernel(
     float* __restrict__ amax = nullptr) {
   __shared__ float redf[32];
   __shared__ int redi[32];
+  // The tensor-core kernel after this one may launch at once: it only loads its weights
+  // and sets up until this grid has finished.
   allow_dependent_launch();
   grid_dependency_wait();  // x (and amax) may come from the kernel before; no-op otherwise
   grid_zero(zero, zero_n16);

@@ -16,6 +16,7 @@
 #include "act_quant.cuh"
 #include "common.cuh"
 #include "gemm_bf16.cuh"
+#include "gemm_prefill.cuh"
 #include "gemm_skinny.cuh"
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
@@ -352,22 +353,25 @@ bl_status launch_gemv3_m(const void* x, const uint8_t* packed3, const float* gam
 }
 
 // ------------------------------------------------------------------ GEMM launch
+// The prefill GEMM (M > 256 tokens): the weights as the TMEM A operand, the tokens by TMA.
 template <int OM>
 bl_status launch_gemm_t(const int8_t* xq, const uint8_t* packed, const int* rowsum,
                         const float* scale, const float* gamma, void* y, int M, int N, int K,
                         cudaStream_t s, const ChainOpts& o) {
-  CUtensorMap map_a, map_b;
-  if (!make_map_u8(&map_a, xq, K, M, K, bl::tc::BK, bl::tc::BM, true)) return BL_ERR_CUDA;
-  if (!make_map_u8(&map_b, packed, K / 4, N, K / 4, bl::tc::BK / 4, bl::tc::BN, false))
+  const int bnt = bl::pf::token_tile(M);
+  CUtensorMap map_x, map_w;
+  if (!make_map_u8(&map_x, xq, K, M, K, bl::pf::BK, bnt, true)) return BL_ERR_CUDA;
+  if (!make_map_u8(&map_w, packed, K / 4, N, K / 4, bl::pf::BK / 4, bl::pf::BW, false))
     return BL_ERR_CUDA;
-  auto kern = bl::gemm_tc_kernel<OM>;
+  auto kern = bl::gemm_prefill_kernel<OM>;
   static bl::PerDevice configured;
-  if (!set_smem_limit_once(configured, kern, bl::tc::SMEM_BYTES)) return BL_ERR_CUDA;
-  const long long tiles = static_cast<long long>((M + bl::tc::BM - 1) / bl::tc::BM) *
-                          ((N + bl::tc::BN - 1) / bl::tc::BN);
+  if (!set_smem_limit_once(configured, kern, bl::pf::SMEM_BYTES)) return BL_ERR_CUDA;
+  const long long tiles = static_cast<long long>((M + bnt - 1) / bnt) *
+                          ((N + bl::pf::BW - 1) / bl::pf::BW);
   const int grid = static_cast<int>(std::min<long long>(tiles, num_sms()));
-  return launch_ex(kern, dim3(grid), dim3(bl::tc::THREADS), bl::tc::SMEM_BYTES, s, o.pdl,
-                   map_a, map_b, rowsum, scale, gamma, y, M, N, K, kWaitLimitNs, o.amax_out);
+  return launch_ex(kern, dim3(grid), dim3(bl::pf::THREADS), bl::pf::SMEM_BYTES, s, o.pdl,
+                   map_x, map_w, rowsum, scale, gamma, y, M, N, K, bnt, kWaitLimitNs,
+                   o.amax_out);
 }
 
 bl_status launch_gemm(const int8_t* xq, const uint8_t* packed, const int* rowsum,

@@ -1,0 +1,313 @@
+// Prefill BitLinear (many tokens) on the 5th-generation tensor cores, operands swapped so
+// that the ternary weights never pass through shared memory unpacked:
+//   D[n][t] = sum_k u[n][k] * xq[t][k]        (tcgen05.mma kind::i8, A from TMEM)
+//   y[t][n] = float(D - rowsum_t) * (scale_t * gamma)
+// the addition-only integer product of BitNet b1.58 (dmarx anthology record LIT-380, Key
+// takeaways bullet 4) in the u = c + 1 form of the other kernels.
+//
+// Why swapped: with the weights as the B operand in shared memory, every K block moves the
+// packed tile in, the unpacked int8 tile out and back in to the tensor core, next to the
+// token tile: about 112 KB of shared-memory traffic per 128 x 256 x 128 block of MMA work,
+// more than shared memory sustains while the tensor core works. Here the four unpack warps
+// turn each thread's weight row (32 packed bytes = 128 trits of a K block) into 32
+// registers and write them with one tcgen05.st into that row's TMEM lane; the MMA reads A
+// from TMEM. Shared memory carries only the token tile (written by TMA, read by the MMA)
+// and the 4 KB packed tile: 56 KB per 128 x 192 x 128 block.
+//
+// Tiles: 128 weight rows (MMA M, TMEM lanes) x bnt <= 192 tokens (MMA N). TMEM (512
+// columns): two accumulators of 192 columns (the epilogue drains one while the MMAs fill
+// the other) and STAGES unpacked K blocks of 32 columns, one per TMA stage: the unpack of
+// stage g may overwrite slot g % STAGES as soon as stage g's TMA data has landed, since
+// the producer re-armed that stage only after the MMAs of stage g - STAGES (the last
+// readers of the slot) had completed.
+//
+// Warps: 0-3 unpack (thread r owns weight row r, TMEM lane r), 4-7 epilogue (tcgen05.ld of
+// their 32 lanes, rowsum, rescale, store), 8 TMA producer, 9 TMEM owner and MMA issuer
+// (whole-warp loop, one elected lane issues). Persistent: one CTA per SM walks the tiles,
+// consecutive CTAs taking consecutive token tiles of one weight tile (L2 reuse of both).
+// Every mbarrier wait is bounded; on a timeout the kernel records BL_ERR_TIMEOUT, waits
+// (bounded) for its own copies and MMAs, frees TMEM and exits.
+#pragma once
+
+#include "common.cuh"
+#include "gemm_skinny.cuh"
+#include "gemm_tc.cuh"
+
+namespace bl {
+
+namespace pf {
+constexpr int BW = 128;                   // weight rows per tile (MMA M)
+constexpr int BK = 128;                   // K per stage (one 128-byte swizzle row of int8)
+constexpr int MMA_K = 32;                 // K per tcgen05.mma kind::i8
+constexpr int STAGES = 4;                 // TMA stages = unpacked A slots in TMEM
+constexpr int MAX_BNT = 192;              // tokens per tile, at most (MMA N)
+constexpr int X_BYTES = MAX_BNT * BK;     // 24 KB token tile (128-byte swizzle)
+constexpr int WP_BYTES = BW * BK / 4;     // 4 KB packed weight tile
+constexpr int A_COLS = BK / 4;            // TMEM columns of one unpacked K block
+constexpr int A_COL0 = 2 * MAX_BNT;       // first A slot column, after two accumulators
+constexpr int TMEM_COLS = 512;
+constexpr int THREADS = 320;
+static_assert(A_COL0 + STAGES * A_COLS <= TMEM_COLS, "TMEM budget");
+static_assert(X_BYTES % 1024 == 0, "swizzle atoms of the token stages stay aligned");
+
+struct Barriers {
+  uint64_t full[STAGES];     // token tile + packed weights of a stage landed
+  uint64_t empty[STAGES];    // the stage's MMAs are done (smem and A slot free)
+  uint64_t a_full[STAGES];   // the stage's weights are in their TMEM slot
+  uint64_t tmem_full[2];
+  uint64_t tmem_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+struct Shared {
+  int rowsum[2][MAX_BNT];
+  float f[2][MAX_BNT];  // scale_t * gamma
+  Barriers bar;
+};
+
+constexpr int SMEM_BYTES = 1024 /* alignment slack */ + STAGES * (X_BYTES + WP_BYTES) +
+                           static_cast<int>(sizeof(Shared));
+
+// Token tile for M tokens: as even as the tile count allows, a multiple of 16, <= 192.
+__host__ __device__ constexpr int token_tile(int M) {
+  const int tiles = (M + MAX_BNT - 1) / MAX_BNT;
+  const int per = (M + tiles - 1) / tiles;
+  return (per + 15) / 16 * 16;
+}
+}  // namespace pf
+
+__device__ __forceinline__ void epi4_bar_sync() {  // the 4 epilogue warps (4-7) only
+  asm volatile("bar.sync 3, 128;" ::: "memory");
+}
+
+// OM: 0 fp32 out, 1 bf16 out, 2 int32 out (acc only). bnt = token tile (multiple of 16,
+// <= MAX_BNT; the token tensor map's box has bnt rows). amax_out (layer chains, may be
+// null): receives the absmax of each token's outputs.
+template <int OM>
+__global__ void __launch_bounds__(pf::THREADS, 1) gemm_prefill_kernel(
+    const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w,
+    const int* __restrict__ rowsum, const float* __restrict__ scale,
+    const float* __restrict__ gamma_ptr, void* __restrict__ y, int M, int N, int K, int bnt,
+    unsigned long long limit_ns, float* __restrict__ amax_out) {
+  using namespace pf;
+  allow_dependent_launch();  // the next kernel may set up (it waits before using y)
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  unsigned char* sX = smem;                          // STAGES x [bnt][128] swizzled
+  unsigned char* sW = sX + STAGES * X_BYTES;         // STAGES x [128][32] packed
+  Shared* sh = reinterpret_cast<Shared*>(sW + STAGES * WP_BYTES);
+  Barriers* bar = &sh->bar;
+  volatile int* abort_flag = &bar->abort;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t_tiles = (M + bnt - 1) / bnt;
+  const int w_tiles = (N + BW - 1) / BW;
+  const int num_tiles = t_tiles * w_tiles;
+  const int KB = (K + BK - 1) / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&bar->full[s], 1);
+      mbar_init(&bar->empty[s], 1);
+      mbar_init(&bar->a_full[s], 4);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bar->tmem_full[b], 1);
+      mbar_init(&bar->tmem_empty[b], 4);
+    }
+    mbar_init(&bar->drain, 1);
+    bar->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(&bar->tmem_base, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = bar->tmem_base;
+  grid_dependency_wait();  // operands from the kernel before (no-op without the attribute)
+
+  if (warp == 8) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&map_x);
+      prefetch_tmap(&map_w);
+      const uint32_t bytes = static_cast<uint32_t>(bnt * BK + WP_BYTES);
+      int s = 0;
+      uint32_t ph = 0;
+      long long issued = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        const int t0 = (tile % t_tiles) * bnt;
+        const int n0 = (tile / t_tiles) * BW;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!tc_wait(&bar->empty[s], ph ^ 1u, limit_ns, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(&bar->full[s], bytes);
+          tma_load_2d(sX + s * X_BYTES, &map_x, kb * BK, t0, &bar->full[s]);
+          tma_load_2d(sW + s * WP_BYTES, &map_w, kb * (BK / 4), n0, &bar->full[s]);
+          ++issued;
+          if (++s == STAGES) { s = 0; ph ^= 1u; }
+        }
+      }
+      if (!ok) {  // wait (bounded) for the copies still in flight
+        const long long last = issued - 1;
+        for (long long i = last; i >= 0 && i > last - STAGES; --i)
+          mbar_wait(&bar->full[i % STAGES], static_cast<uint32_t>((i / STAGES) & 1),
+                    100000000ull);
+      }
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------------ MMA issuer
+    const uint32_t idesc = idesc_i8(BW, bnt);
+    const uint64_t x_desc0 = smem_desc_k128(smem_u32(sX));
+    int s = 0, ab = 0;
+    uint32_t ph = 0, aph = 0;
+    bool ok = true, issued_any = false;
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      bool got = true;
+      if (lane == 0) got = tc_wait(&bar->tmem_empty[ab], aph ^ 1u, limit_ns, abort_flag);
+      if (!__shfl_sync(0xffffffffu, got, 0)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(ab * MAX_BNT);
+      for (int kb = 0; kb < KB; ++kb) {
+        if (lane == 0) got = tc_wait(&bar->a_full[s], ph, limit_ns, abort_flag);
+        if (!__shfl_sync(0xffffffffu, got, 0)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t a_tmem = tmem_base + static_cast<uint32_t>(A_COL0 + s * A_COLS);
+        const uint64_t b_desc = x_desc0 + static_cast<uint64_t>(s * (X_BYTES >> 4));
+#pragma unroll
+        for (int kk = 0; kk < BK / MMA_K; ++kk)
+          mma_i8_ts_elect(d_tmem, a_tmem + static_cast<uint32_t>(kk * (MMA_K / 4)),
+                          b_desc + static_cast<uint64_t>(kk * (MMA_K >> 4)), idesc,
+                          (kb | kk) != 0 ? 1u : 0u);
+        issued_any = true;
+        mma_commit_elect(&bar->empty[s]);
+        if (++s == STAGES) { s = 0; ph ^= 1u; }
+      }
+      if (!ok) break;
+      mma_commit_elect(&bar->tmem_full[ab]);
+      if (++ab == 2) { ab = 0; aph ^= 1u; }
+    }
+    if (!ok && issued_any) {
+      mma_commit_elect(&bar->drain);  // completes once every MMA issued above has finished
+      if (lane == 0) mbar_wait(&bar->drain, 0u, 100000000ull);
+      __syncwarp();
+    }
+  } else if (warp < 4) {
+    // ------------------------------------------------------------------ unpack warps
+    const int r = threadIdx.x;  // weight row of the tile = TMEM lane
+    const uint32_t a_lane = tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + A_COL0;
+    int s = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      for (int kb = 0; kb < KB; ++kb) {
+        const bool got = tc_wait(&bar->full[s], ph, limit_ns, abort_flag);
+        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+        const uint4* src = reinterpret_cast<const uint4*>(sW + s * WP_BYTES + r * 32);
+        uint32_t a[32];  // the row's 128 codes of this K block, 4 per register
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint4 p = src[h];
+          const uint32_t words[4] = {p.x, p.y, p.z, p.w};
+#pragma unroll
+          for (int mq = 0; mq < 4; ++mq) {
+            const int c = 16 * h + 4 * mq;  // column of trits 4c .. 4c + 15
+            a[c + 0] = words[mq] & 0x03030303u;
+            a[c + 1] = (words[mq] >> 2) & 0x03030303u;
+            a[c + 2] = (words[mq] >> 4) & 0x03030303u;
+            a[c + 3] = (words[mq] >> 6) & 0x03030303u;
+          }
+        }
+        tmem_st_x32(a_lane + static_cast<uint32_t>(s * A_COLS), a);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar->a_full[s]);
+        if (++s == STAGES) { s = 0; ph ^= 1u; }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ epilogue
+    const int q = warp - 4;     // TMEM lanes 32q .. 32q + 31
+    const int et = threadIdx.x - 128;  // 0..127
+    const float gamma = (OM == 2) ? 0.0f : *gamma_ptr;
+    int ab = 0;
+    uint32_t aph = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      const int t0 = (tile % t_tiles) * bnt;
+      const int n0 = (tile / t_tiles) * BW;
+      // the tile's per-token factors (the buffer of this accumulator was last read two
+      // tiles ago, before the barrier of the previous tile)
+      for (int j = et; j < bnt; j += 128) {
+        const int t = t0 + j;
+        sh->rowsum[ab][j] = (t < M) ? rowsum[t] : 0;
+        sh->f[ab][j] = (OM != 2 && t < M) ? __fmul_rn(scale[t], gamma) : 0.0f;
+      }
+      epi4_bar_sync();
+      const bool got = tc_wait(&bar->tmem_full[ab], aph, limit_ns, abort_flag);
+      if (!__all_sync(0xffffffffu, got)) break;
+      tc_fence_after();
+      const int n = n0 + q * 32 + lane;
+      const bool nvalid = n < N;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                             static_cast<uint32_t>(ab * MAX_BNT);
+      for (int c0 = 0; c0 < bnt; c0 += 32) {
+        uint32_t v[32];
+        if (c0 + 32 <= bnt) {
+          tmem_ld_x32(taddr + c0, v);
+        } else {  // bnt % 32 == 16: the last 16 columns
+          uint32_t w16[16];
+          tmem_ld_x16(taddr + c0, w16);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) { v[j] = w16[j]; v[j + 16] = 0u; }
+        }
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int tj = c0 + j;
+          const int t = t0 + tj;
+          if (tj >= bnt || t >= M) continue;  // the same for the whole warp
+          const int a = static_cast<int>(v[j]) - sh->rowsum[ab][tj];
+          unsigned mag = 0u;
+          if (nvalid) {
+            const long long o = static_cast<long long>(t) * N + n;
+            if (OM == 2) {
+              static_cast<int*>(y)[o] = a;
+            } else {
+              const float val = __fmul_rn(__int2float_rn(a), sh->f[ab][tj]);
+              if (OM == 0) {
+                static_cast<float*>(y)[o] = val;
+                mag = __float_as_uint(val) & 0x7fffffffu;
+              } else {
+                const __nv_bfloat16 h = __float2bfloat16_rn(val);
+                static_cast<__nv_bfloat16*>(y)[o] = h;
+                mag = __float_as_uint(__bfloat162float(h)) & 0x7fffffffu;
+              }
+            }
+          }
+          if (OM != 2 && amax_out != nullptr) warp_amax_out(amax_out, t, mag);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar->tmem_empty[ab]);
+      if (++ab == 2) { ab = 0; aph ^= 1u; }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+}  // namespace bl

@@ -237,7 +237,9 @@ __global__ void __launch_bounds__(tc::THREADS, 1) gemm_tc_kernel(
                   make_int4(static_cast<int>(v[j]) - rs, static_cast<int>(v[j + 1]) - rs,
                             static_cast<int>(v[j + 2]) - rs, static_cast<int>(v[j + 3]) - rs);
           } else {
-            for (int j = 0; j < 32 && n + j < N; ++j) out[j] = static_cast<int>(v[j]) - rs;
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (n + j < N) out[j] = static_cast<int>(v[j]) - rs;
           }
         } else {
           float r[32];
@@ -258,7 +260,9 @@ __global__ void __launch_bounds__(tc::THREADS, 1) gemm_tc_kernel(
               for (int j = 0; j < 32; j += 4)
                 *reinterpret_cast<float4*>(out + j) = make_float4(r[j], r[j + 1], r[j + 2], r[j + 3]);
             } else {
-              for (int j = 0; j < 32 && n + j < N; ++j) out[j] = r[j];
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (n + j < N) out[j] = r[j];
             }
           } else {
             __nv_bfloat16* out = static_cast<__nv_bfloat16*>(y) + o;
@@ -277,7 +281,9 @@ __global__ void __launch_bounds__(tc::THREADS, 1) gemm_tc_kernel(
                 *reinterpret_cast<uint4*>(out + j) = pk;
               }
             } else {
-              for (int j = 0; j < 32 && n + j < N; ++j) out[j] = __float2bfloat16_rn(r[j]);
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (n + j < N) out[j] = __float2bfloat16_rn(r[j]);
             }
           }
         }

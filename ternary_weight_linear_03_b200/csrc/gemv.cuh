@@ -123,9 +123,9 @@ __device__ __forceinline__ void load16(const void* x, long long off, float (&v)[
 // Layer chains (optional, null when unused): amax_in[t] is the absmax of token t's row of
 // x, formed by the kernel that wrote x, so the prologue skips its max pass; amax_out
 // receives the absmax of this kernel's outputs per token (atomic max; zeroed beforehand).
-// Launched with programmatic dependent launch, the kernel first lets the next kernel of
-// the stream launch, and starts the L2 prefetch of its own weights, before it waits for
-// the kernel that wrote x.
+// Launched with programmatic dependent launch, the kernel starts the L2 prefetch of its own
+// weights before it waits for the kernel that wrote x, and lets the next kernel launch once
+// that wait is over.
 template <int MT, int XM, int OM, bool XR, int R>
 __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(
     const void* __restrict__ x, const uint8_t* __restrict__ packed,
@@ -137,7 +137,6 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int CPR = K >> 6;   // 16-byte packed chunks per weight row
   const int KB = K >> 4;    // 16-element groups per token row
-  allow_dependent_launch();
   if (chain) {
     // L2 prefetch of this block's share of the packed weights (it does not depend on the
     // kernel before), in 4 KB pieces, then wait for that kernel's outputs
@@ -152,6 +151,9 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(
     }
   }
   grid_dependency_wait();
+  // Only now (this kernel's input is complete) may the next kernel start and prefetch its
+  // own weights: one layer ahead, not a cascade of every later layer into L2.
+  allow_dependent_launch();
 
   // ---------------------------------------------------------------- prologue: x -> int8
   if (XM == kXi8) {
