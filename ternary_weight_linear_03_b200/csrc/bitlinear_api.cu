@@ -495,12 +495,21 @@ bl_status launch_act_quant_chain(const void* x, int x_dtype, int M, int K, int8_
 
 // ------------------------------------------------------------------ weight quantization
 // Workspace of bitlinear_quantize_weights: the exact-sum columns and the barrier counters.
-size_t wq_ws_bytes(long long) { return align_up(sizeof(WqWorkspace), 256); }
+// Workspace of bitlinear_quantize_weights: the exact-sum columns and barrier counters, and
+// for matrices of at least kWqSingleMin weights the band lists of the single-read mode.
+constexpr long long kWqSingleMin = 4ll << 20;
+size_t wq_ws_head() { return align_up(sizeof(WqWorkspace), 256); }
+size_t wq_list_bytes() {
+  return static_cast<size_t>(bl::kWqMaxBlocks) * bl::kWqListCap * sizeof(uint2);
+}
+size_t wq_ws_bytes(long long n) {
+  return wq_ws_head() + (n >= kWqSingleMin ? wq_list_bytes() : 0);
+}
 
 template <bool kBf16, int MODE>
 bl_status launch_weight_quant_t(const void* W, long long n, long long n_total, float eps,
-                                void* ws, unsigned long long* sums, float* gamma,
-                                uint32_t* packed, cudaStream_t s) {
+                                void* ws, size_t ws_bytes, unsigned long long* sums,
+                                float* gamma, uint32_t* packed, cudaStream_t s) {
   auto kern = bl::weight_quant_kernel<kBf16, MODE>;
   constexpr int kSmem = bl::kWqStages * bl::kWqStageBytes;
   // blocks of this kernel resident per SM, found once per device after raising its
@@ -525,8 +534,16 @@ bl_status launch_weight_quant_t(const void* W, long long n, long long n_total, f
       cudaMemsetAsync(hdr, 0, sizeof(WqWorkspace), s) != cudaSuccess)
     return BL_ERR_CUDA;
   unsigned long long limit = kWaitLimitNs;
+  // Single-read mode when a block's range does not fit its ring (the two-pass mode would
+  // stream it twice) and the workspace holds the band lists.
+  const long long words = n / 16;
+  const long long range_bytes = (words + grid - 1) / grid * (kBf16 ? 32 : 64);
+  uint2* list = nullptr;
+  if (MODE == bl::kWqFull && range_bytes > 1ll * bl::kWqStages * bl::kWqStageBytes &&
+      grid <= bl::kWqMaxBlocks && ws_bytes >= wq_ws_head() + wq_list_bytes())
+    list = reinterpret_cast<uint2*>(static_cast<char*>(ws) + wq_ws_head());
   void* args[] = {const_cast<void**>(&W), &n, &n_total, &eps, &hdr, &sums, &gamma, &packed,
-                  &limit};
+                  &limit, &list};
   if (cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kern), dim3(grid),
                                   dim3(bl::kWqThreads), args, kSmem, s) != cudaSuccess)
     return BL_ERR_CUDA;
@@ -535,11 +552,12 @@ bl_status launch_weight_quant_t(const void* W, long long n, long long n_total, f
 
 template <int MODE>
 bl_status launch_weight_quant(const void* W, bool bf16, long long n, long long n_total,
-                              float eps, void* ws, unsigned long long* sums, float* gamma,
-                              uint32_t* packed, cudaStream_t s) {
-  return bf16 ? launch_weight_quant_t<true, MODE>(W, n, n_total, eps, ws, sums, gamma, packed, s)
-              : launch_weight_quant_t<false, MODE>(W, n, n_total, eps, ws, sums, gamma, packed,
-                                                   s);
+                              float eps, void* ws, size_t ws_bytes, unsigned long long* sums,
+                              float* gamma, uint32_t* packed, cudaStream_t s) {
+  return bf16 ? launch_weight_quant_t<true, MODE>(W, n, n_total, eps, ws, ws_bytes, sums, gamma,
+                                                  packed, s)
+              : launch_weight_quant_t<false, MODE>(W, n, n_total, eps, ws, ws_bytes, sums, gamma,
+                                                   packed, s);
 }
 
 // ------------------------------------------------------------------ debug probe
@@ -609,7 +627,7 @@ bl_status bitlinear_quantize_weights(const void* W, int w_dtype, int N, int K, f
   if (ws_bytes < sizeof(WqWorkspace)) return BL_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const long long n = static_cast<long long>(N) * K;
-  return launch_weight_quant<bl::kWqFull>(W, w_dtype == BL_BF16, n, n, eps, ws, nullptr, gamma,
+  return launch_weight_quant<bl::kWqFull>(W, w_dtype == BL_BF16, n, n, eps, ws, ws_bytes, nullptr, gamma,
                                           reinterpret_cast<uint32_t*>(packed), s);
 }
 
@@ -622,7 +640,7 @@ bl_status bitlinear_weight_abssum(const void* W, int w_dtype, int N, int K, uint
   if (ws_bytes < sizeof(WqWorkspace)) return BL_ERR_WORKSPACE;
   const long long n = static_cast<long long>(N) * K;
   return launch_weight_quant<bl::kWqPartial>(
-      W, w_dtype == BL_BF16, n, n, 0.0f, ws, reinterpret_cast<unsigned long long*>(sums),
+      W, w_dtype == BL_BF16, n, n, 0.0f, ws, ws_bytes, reinterpret_cast<unsigned long long*>(sums),
       nullptr, nullptr, static_cast<cudaStream_t>(stream));
 }
 
@@ -638,7 +656,7 @@ bl_status bitlinear_quantize_weights_from_abssum(const void* W, int w_dtype, int
   if (!aligned16(W) || !aligned16(sums) || !aligned16(packed) || !aligned16(gamma))
     return BL_ERR_MISALIGNED;
   return launch_weight_quant<bl::kWqFinish>(
-      W, w_dtype == BL_BF16, static_cast<long long>(N) * K, n_total, eps, nullptr,
+      W, w_dtype == BL_BF16, static_cast<long long>(N) * K, n_total, eps, nullptr, 0,
       const_cast<unsigned long long*>(reinterpret_cast<const unsigned long long*>(sums)), gamma,
       reinterpret_cast<uint32_t*>(packed), static_cast<cudaStream_t>(stream));
 }

@@ -21,9 +21,11 @@
 // the producer re-armed that stage only after the MMAs of stage g - STAGES (the last
 // readers of the slot) had completed.
 //
-// Warps: 0-3 unpack (thread r owns weight row r, TMEM lane r), 4-7 epilogue (tcgen05.ld of
-// their 32 lanes, rowsum, rescale, store), 8 TMA producer, 9 TMEM owner and MMA issuer
-// (whole-warp loop, one elected lane issues). Persistent: one CTA per SM walks the tiles,
+// Warps: 0-7 unpack in two sets of four that take alternate stages (each set's chain of
+// barrier wait, shared-memory load, tcgen05.st, wait::st and arrival per stage is longer
+// than the MMAs of one stage; thread r of a set owns weight row r, TMEM lane r), 8-11
+// epilogue (tcgen05.ld of their 32 lanes, rowsum, rescale, store), 12 TMA producer, 13
+// TMEM owner and MMA issuer (whole-warp loop, one elected lane issues). Persistent: one CTA per SM walks the tiles,
 // consecutive CTAs taking consecutive token tiles of one weight tile (L2 reuse of both).
 // Every mbarrier wait is bounded; on a timeout the kernel records BL_ERR_TIMEOUT, waits
 // (bounded) for its own copies and MMAs, frees TMEM and exits.
@@ -46,7 +48,9 @@ constexpr int WP_BYTES = BW * BK / 4;     // 4 KB packed weight tile
 constexpr int A_COLS = BK / 4;            // TMEM columns of one unpacked K block
 constexpr int A_COL0 = 2 * MAX_BNT;       // first A slot column, after two accumulators
 constexpr int TMEM_COLS = 512;
-constexpr int THREADS = 320;
+constexpr int UNPACK_SETS = 2;
+constexpr int THREADS = 448;
+static_assert(STAGES % UNPACK_SETS == 0, "each set keeps to its own stages");
 static_assert(A_COL0 + STAGES * A_COLS <= TMEM_COLS, "TMEM budget");
 static_assert(X_BYTES % 1024 == 0, "swizzle atoms of the token stages stay aligned");
 
@@ -78,7 +82,7 @@ __host__ __device__ constexpr int token_tile(int M) {
 }
 }  // namespace pf
 
-__device__ __forceinline__ void epi4_bar_sync() {  // the 4 epilogue warps (4-7) only
+__device__ __forceinline__ void epi4_bar_sync() {  // the 4 epilogue warps (8-11) only
   asm volatile("bar.sync 3, 128;" ::: "memory");
 }
 
@@ -122,7 +126,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1) gemm_prefill_kernel(
     bar->abort = 0;
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == 13) {
     tmem_alloc(&bar->tmem_base, TMEM_COLS);
     tmem_relinquish();
   }
@@ -132,7 +136,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1) gemm_prefill_kernel(
   const uint32_t tmem_base = bar->tmem_base;
   grid_dependency_wait();  // operands from the kernel before (no-op without the attribute)
 
-  if (warp == 8) {
+  if (warp == 12) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       prefetch_tmap(&map_x);
@@ -161,7 +165,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1) gemm_prefill_kernel(
                     100000000ull);
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == 13) {
     // ------------------------------------------------------------------ MMA issuer
     const uint32_t idesc = idesc_i8(BW, bnt);
     const uint64_t x_desc0 = smem_desc_k128(smem_u32(sX));
@@ -198,22 +202,32 @@ __global__ void __launch_bounds__(pf::THREADS, 1) gemm_prefill_kernel(
       if (lane == 0) mbar_wait(&bar->drain, 0u, 100000000ull);
       __syncwarp();
     }
-  } else if (warp < 4) {
+  } else if (warp < 8) {
     // ------------------------------------------------------------------ unpack warps
-    const int r = threadIdx.x;  // weight row of the tile = TMEM lane
-    const uint32_t a_lane = tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + A_COL0;
-    int s = 0;
-    uint32_t ph = 0;
+    const int set = warp >> 2;   // stages g with g % UNPACK_SETS == set
+    const int wq = warp & 3;     // TMEM lane quarter
+    const int r = wq * 32 + lane;  // weight row of the tile = TMEM lane
+    const uint32_t a_lane = tmem_base + (static_cast<uint32_t>(wq * 32) << 16) + A_COL0;
+    // Rows are 32 bytes apart: lanes 0-3 of each quarter-warp read their first 16-byte
+    // half first and lanes 4-7 their second, so the 8 rows of a 128-byte wavefront fall
+    // in 8 distinct bank groups.
+    const int h0 = (lane >> 2) & 1;
+    long long g = 0;  // stages of this CTA so far
     bool ok = true;
     for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-      for (int kb = 0; kb < KB; ++kb) {
+      for (int kb = 0; kb < KB; ++kb, ++g) {
+        if (static_cast<int>(g % UNPACK_SETS) != set) continue;
+        const int s = static_cast<int>(g % STAGES);
+        const uint32_t ph = static_cast<uint32_t>((g / STAGES) & 1);
         const bool got = tc_wait(&bar->full[s], ph, limit_ns, abort_flag);
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
         const uint4* src = reinterpret_cast<const uint4*>(sW + s * WP_BYTES + r * 32);
+        const uint4 first = src[h0], second = src[h0 ^ 1];
+        const uint4 halves[2] = {h0 ? second : first, h0 ? first : second};
         uint32_t a[32];  // the row's 128 codes of this K block, 4 per register
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          const uint4 p = src[h];
+          const uint4 p = halves[h];
           const uint32_t words[4] = {p.x, p.y, p.z, p.w};
 #pragma unroll
           for (int mq = 0; mq < 4; ++mq) {
@@ -229,13 +243,12 @@ __global__ void __launch_bounds__(pf::THREADS, 1) gemm_prefill_kernel(
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar->a_full[s]);
-        if (++s == STAGES) { s = 0; ph ^= 1u; }
       }
     }
   } else {
     // ------------------------------------------------------------------ epilogue
-    const int q = warp - 4;     // TMEM lanes 32q .. 32q + 31
-    const int et = threadIdx.x - 128;  // 0..127
+    const int q = warp - 8;     // TMEM lanes 32q .. 32q + 31
+    const int et = threadIdx.x - 256;  // 0..127
     const float gamma = (OM == 2) ? 0.0f : *gamma_ptr;
     int ab = 0;
     uint32_t aph = 0;
@@ -272,15 +285,24 @@ __global__ void __launch_bounds__(pf::THREADS, 1) gemm_prefill_kernel(
         for (int j = 0; j < 32; ++j) {
           const int tj = c0 + j;
           const int t = t0 + tj;
+          // the tile's factors four at a time (bnt is a multiple of 16)
+          int4 rs4;
+          float4 f4;
+          if ((j & 3) == 0 && tj < bnt) {
+            rs4 = *reinterpret_cast<const int4*>(&sh->rowsum[ab][tj]);
+            f4 = *reinterpret_cast<const float4*>(&sh->f[ab][tj]);
+          }
           if (tj >= bnt || t >= M) continue;  // the same for the whole warp
-          const int a = static_cast<int>(v[j]) - sh->rowsum[ab][tj];
+          const int rsj = (j & 3) == 0 ? rs4.x : (j & 3) == 1 ? rs4.y : (j & 3) == 2 ? rs4.z : rs4.w;
+          const float fj = (j & 3) == 0 ? f4.x : (j & 3) == 1 ? f4.y : (j & 3) == 2 ? f4.z : f4.w;
+          const int a = static_cast<int>(v[j]) - rsj;
           unsigned mag = 0u;
           if (nvalid) {
             const long long o = static_cast<long long>(t) * N + n;
             if (OM == 2) {
               static_cast<int*>(y)[o] = a;
             } else {
-              const float val = __fmul_rn(__int2float_rn(a), sh->f[ab][tj]);
+              const float val = __fmul_rn(__int2float_rn(a), fj);
               if (OM == 0) {
                 static_cast<float*>(y)[o] = val;
                 mag = __float_as_uint(val) & 0x7fffffffu;
@@ -303,7 +325,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1) gemm_prefill_kernel(
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 13) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem_base, TMEM_COLS);

@@ -52,7 +52,39 @@ constexpr int kWqCopies = 8;       // copies of the column sums and arrival coun
 struct WqWorkspace {
   unsigned long long cols[kWqCopies][kWqLimbs];  // column sums (below 2^39 per block)
   unsigned int arrived[kWqCopies];               // grid-barrier arrivals
+  double est_sum;                                // single-read mode: sampled sum of |w|
+  unsigned long long est_cnt;                    //   and the number of sampled weights
+  unsigned int arrived_est[kWqCopies];           //   arrivals at the estimate barrier
 };
+
+// Single-read mode (large matrices): band entries per block, and the band's half width
+// relative to the estimated threshold.
+constexpr int kWqListCap = 4096;
+constexpr int kWqMaxBlocks = 1024;
+constexpr float kWqBand = 1.0f / 256.0f;
+
+// Bounded grid barrier on spread arrival counters (thread 0 of each block calls it).
+__device__ __forceinline__ bool wq_grid_barrier(unsigned int* arrived, unsigned int nblocks,
+                                                unsigned long long limit_ns) {
+  __threadfence();
+  atomicAdd(&arrived[blockIdx.x % kWqCopies], 1u);
+  const uint64_t t0 = global_ns();
+  while (true) {
+    unsigned int total = 0u;
+#pragma unroll
+    for (int c = 0; c < kWqCopies; ++c) {
+      unsigned v;
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(arrived + c) : "memory");
+      total += v;
+    }
+    if (total >= nblocks) return true;
+    if (global_ns() - t0 > limit_ns) {
+      record_status(kStatusTimeout);
+      return false;
+    }
+    __nanosleep(64);
+  }
+}
 
 // |w| outside the fp64 window: added as (exponent, mantissa) into the shared buckets.
 __device__ __forceinline__ void wq_fallback(uint32_t bits, unsigned long long* sb,
@@ -227,13 +259,17 @@ template <bool kBf16, int MODE>
 __global__ void __launch_bounds__(kWqThreads) weight_quant_kernel(
     const void* __restrict__ W, long long n, long long n_total, float eps,
     WqWorkspace* __restrict__ ws, unsigned long long* __restrict__ sums_io,
-    float* __restrict__ gamma_out, uint32_t* __restrict__ packed, unsigned long long limit_ns) {
+    float* __restrict__ gamma_out, uint32_t* __restrict__ packed, unsigned long long limit_ns,
+    uint2* __restrict__ list) {
   extern __shared__ __align__(128) unsigned char wq_stage[];  // kWqStages x 16 KB
   __shared__ unsigned long long sb[kWqBuckets];
   __shared__ unsigned long long col[kWqLimbs];
   __shared__ uint64_t full[kWqStages];
   __shared__ float s_T;
   __shared__ int s_ok;
+  __shared__ float s_that;          // single-read mode: estimated threshold
+  __shared__ unsigned int s_cnt;    //   band entries of this block
+  __shared__ double s_red[kWqThreads / 32];
   constexpr int E = kBf16 ? 8 : 4;   // weights per 16-byte chunk
   constexpr int PARTS = 16 / E;      // chunks per packed word
   constexpr int WORD_BYTES = kBf16 ? 32 : 64;
@@ -258,6 +294,57 @@ __global__ void __launch_bounds__(kWqThreads) weight_quant_kernel(
     for (int st = 0; st < min(ring.nst, kWqStages); ++st) wq_issue(ring, st, st);
   }
   __syncthreads();
+
+  // Single-read mode (MODE kWqFull with a band list, chosen by the host when the blocks'
+  // ranges do not fit their rings): pass A also codes every weight against an estimated
+  // threshold T^ (from the mean |w| of every block's first stage, after a first grid
+  // barrier) and lists the weights with |w| within kWqBand * T^ of it. Once the exact T is
+  // known, a code can differ from the provisional one only for |w| between T^ and T, so
+  // when T lies inside the band each block patches its listed weights; otherwise (or when
+  // its list overflowed) it streams its range again as in the two-pass mode.
+  const bool single = (MODE == kWqFull) && (list != nullptr);
+  float t_hat = 0.0f, band_lo = 1.0f, band_hi = 0.0f;  // empty band
+  const int mypart = tid & (PARTS - 1);
+  uint32_t mulA[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) mulA[e] = 1u << wq_shift(wq_k<kBf16>(mypart, e));
+  if (single) {
+    double part = 0.0;
+    const int n0c = static_cast<int>(min(static_cast<long long>(kWqStageBytes), ring.bytes) / 16);
+    if (ring.nst > 0) {
+      if (!mbar_wait(&full[0], 0u, limit_ns)) s_ok = 0;
+      const uint4* stage = reinterpret_cast<const uint4*>(wq_stage);
+#pragma unroll
+      for (int i = 0; i < kWqChunks; ++i) {
+        const int c = tid + i * kWqThreads;
+        if (c < n0c) {
+          float w[E];
+          wq_chunk_floats<kBf16>(stage[c], w);
+#pragma unroll
+          for (int e = 0; e < E; ++e) part += static_cast<double>(abs_bits(w[e]));
+        }
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+    if ((tid & 31) == 0) s_red[tid >> 5] = part;
+    __syncthreads();
+    if (tid == 0) {
+      double b = 0.0;
+      for (int w = 0; w < kWqThreads / 32; ++w) b += s_red[w];
+      atomicAdd(&ws->est_sum, b);
+      atomicAdd(&ws->est_cnt, static_cast<unsigned long long>(n0c) * E);
+      if (!wq_grid_barrier(ws->arrived_est, gridDim.x, limit_ns)) s_ok = 0;
+      const unsigned long long cnt = __ldcg(&ws->est_cnt);
+      const double est = __ldcg(&ws->est_sum) / static_cast<double>(cnt > 0ull ? cnt : 1ull);
+      s_that = wq_threshold(__fadd_rn(__double2float_rn(est), eps));
+      s_cnt = 0u;
+    }
+    __syncthreads();
+    t_hat = s_that;
+    band_lo = t_hat * (1.0f - kWqBand);
+    band_hi = t_hat * (1.0f + kWqBand);
+  }
 
   // ---------------------------------------------------------------- pass A: exact sum
   bool resident = false;  // pass B reads pass A's stages from shared memory
@@ -318,6 +405,25 @@ __global__ void __launch_bounds__(kWqThreads) weight_quant_kernel(
             wq_fallback(__float_as_uint(a), sb, nonfinite);
         }
       }
+      if (single) {  // provisional codes against T^, and the band entries
+        const int c = tid + i * kWqThreads;
+        uint32_t bits = 0u;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const float a = abs_bits(w[e]);
+          bits += ((a >= t_hat) ? 2u - ((__float_as_uint(w[e]) >> 30) & 2u) : 1u) * mulA[e];
+          if (c < nchunks && a >= band_lo && a <= band_hi) {
+            const unsigned idx = atomicAdd(&s_cnt, 1u);
+            if (idx < static_cast<unsigned>(kWqListCap))
+              list[static_cast<long long>(blockIdx.x) * kWqListCap + idx] = make_uint2(
+                  static_cast<uint32_t>((1ll * st * kWqStageBytes + 16ll * c) / (16 / E) + e),
+                  __float_as_uint(w[e]));
+          }
+        }
+        bits = wq_or_parts<kBf16>(bits);
+        if (c < nchunks && mypart == 0)
+          packed[wb0 + (1ll * st * kWqStageBytes + 16ll * c) / WORD_BYTES] = bits;
+      }
     }
     if ((st & 15) == 15) wq_flush(acc0, acc1, base, sb);
     __syncthreads();  // every thread is done with this slot
@@ -345,7 +451,7 @@ __global__ void __launch_bounds__(kWqThreads) weight_quant_kernel(
   // (stage st in slot st) and pass B reads them there; otherwise pass B streams the range
   // again, starting now (its stages do not depend on gamma).
   resident = ring.nst <= kWqStages;
-  if (MODE == kWqFull && tid == 0 && !resident)
+  if (MODE == kWqFull && !single && tid == 0 && !resident)
     for (int st = 0; st < kWqStages; ++st) wq_issue(ring, st, ring.nst + st);
 
   // ---------------------------------------------------------------- grid barrier
@@ -398,6 +504,25 @@ __global__ void __launch_bounds__(kWqThreads) weight_quant_kernel(
 
   // ---------------------------------------------------------------- pass B: codes
   const float T = s_T;
+  if (single) {
+    const unsigned cnt = s_cnt;
+    const bool patch = (T >= band_lo) && (T <= band_hi) && cnt <= static_cast<unsigned>(kWqListCap);
+    if (patch) {
+      for (unsigned i = tid; i < cnt; i += kWqThreads) {
+        const uint2 en = list[static_cast<long long>(blockIdx.x) * kWqListCap + i];
+        const float w = __uint_as_float(en.y);
+        const float a = abs_bits(w);
+        const uint32_t neg = (en.y >> 30) & 2u;
+        const uint32_t u_old = (a >= t_hat) ? 2u - neg : 1u;
+        const uint32_t u_new = (a >= T) ? 2u - neg : 1u;
+        if (u_old != u_new)
+          atomicXor(&packed[wb0 + en.x / 16], (u_old ^ u_new) << wq_shift(static_cast<int>(en.x % 16)));
+      }
+      return;
+    }
+    if (tid == 0 && !resident)  // T outside the band, or the list overflowed: stream again
+      for (int st = 0; st < min(ring.nst, kWqStages); ++st) wq_issue(ring, st, ring.nst + st);
+  }
   const int part = tid & (PARTS - 1);  // which part of its packed word this thread holds
   uint32_t mul[E];                     // 1 << bit position of element e of this part
 #pragma unroll

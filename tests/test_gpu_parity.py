@@ -133,6 +133,23 @@ def test_quantize_weights_many_ambiguous(ws_kind):
     np.testing.assert_array_equal(packed.cpu().numpy(), ref_packed)
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_quantize_weights_single_read_band_overflow(dtype):
+    """A matrix large enough for the single-read mode (each block's range exceeds its
+    ring) whose weights crowd the threshold: half of them within 0.1% of (gamma + eps)/2,
+    far more than a block's band list holds, so every block falls back to reading its
+    range again. Codes stay exact, as they do on Gaussian matrices (patched lists)."""
+    rng = np.random.default_rng(8)
+    N, K = 2048, 8192
+    mag = np.where(rng.random(N * K) < 0.5, 0.5 * (1 + 0.001 * rng.uniform(-1, 1, N * K)), 1.5)
+    W = (mag * rng.choice([-1.0, 1.0], N * K) * 0.02).astype(np.float32).reshape(N, K)
+    Wt = torch.from_numpy(W).to(dtype)
+    packed, gamma = bl.quantize_weights(Wt.cuda())
+    ref_packed, ref_gamma = orc.quantize_weights(_np_in(Wt), 1e-5)
+    assert gamma.item() == float(ref_gamma)
+    np.testing.assert_array_equal(packed.cpu().numpy(), ref_packed)
+
+
 def test_ternarize_ties_on_device():
     """Weights exactly at 0.5 (gamma + eps) and one ulp either side."""
     d = np.float32(0.71875)
