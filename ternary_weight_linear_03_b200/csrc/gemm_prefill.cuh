@@ -16,10 +16,10 @@
 //
 // Tiles: 128 weight rows (MMA M, TMEM lanes) x bnt <= 192 tokens (MMA N). TMEM (512
 // columns): two accumulators of 192 columns (the epilogue drains one while the MMAs fill
-// the other) and STAGES unpacked K blocks of 32 columns, one per TMA stage: the unpack of
-// stage g may overwrite slot g % STAGES as soon as stage g's TMA data has landed, since
-// the producer re-armed that stage only after the MMAs of stage g - STAGES (the last
-// readers of the slot) had completed.
+// the other) and ASLOTS unpacked K blocks of 32 columns. Shared memory holds STAGES > ASLOTS
+// TMA stages, deeper than TMEM allows A slots, so that the L2 latency of the token tiles
+// stays covered; stage g's weights go to slot g % ASLOTS once the MMAs of stage
+// g - ASLOTS, its last readers, have completed (their commit arrives on a_empty).
 //
 // Warps: 0-7 unpack in two sets of four that take alternate stages (each set's chain of
 // barrier wait, shared-memory load, tcgen05.st, wait::st and arrival per stage is longer
@@ -41,7 +41,8 @@ namespace pf {
 constexpr int BW = 128;                   // weight rows per tile (MMA M)
 constexpr int BK = 128;                   // K per stage (one 128-byte swizzle row of int8)
 constexpr int MMA_K = 32;                 // K per tcgen05.mma kind::i8
-constexpr int STAGES = 4;                 // TMA stages = unpacked A slots in TMEM
+constexpr int STAGES = 6;                 // TMA stages (token tile + packed weights)
+constexpr int ASLOTS = 4;                 // unpacked A slots in TMEM
 constexpr int MAX_BNT = 192;              // tokens per tile, at most (MMA N)
 constexpr int X_BYTES = MAX_BNT * BK;     // 24 KB token tile (128-byte swizzle)
 constexpr int WP_BYTES = BW * BK / 4;     // 4 KB packed weight tile
@@ -50,14 +51,15 @@ constexpr int A_COL0 = 2 * MAX_BNT;       // first A slot column, after two accu
 constexpr int TMEM_COLS = 512;
 constexpr int UNPACK_SETS = 2;
 constexpr int THREADS = 448;
-static_assert(STAGES % UNPACK_SETS == 0, "each set keeps to its own stages");
-static_assert(A_COL0 + STAGES * A_COLS <= TMEM_COLS, "TMEM budget");
+static_assert(ASLOTS % UNPACK_SETS == 0, "each set keeps to its own A slots");
+static_assert(A_COL0 + ASLOTS * A_COLS <= TMEM_COLS, "TMEM budget");
 static_assert(X_BYTES % 1024 == 0, "swizzle atoms of the token stages stay aligned");
 
 struct Barriers {
   uint64_t full[STAGES];     // token tile + packed weights of a stage landed
-  uint64_t empty[STAGES];    // the stage's MMAs are done (smem and A slot free)
-  uint64_t a_full[STAGES];   // the stage's weights are in their TMEM slot
+  uint64_t empty[STAGES];    // the stage's MMAs are done (its shared memory is free)
+  uint64_t a_full[ASLOTS];   // a stage's weights are in this TMEM slot
+  uint64_t a_empty[ASLOTS];  // the MMAs that read this slot are done
   uint64_t tmem_full[2];
   uint64_t tmem_empty[2];
   uint64_t drain;
@@ -116,7 +118,10 @@ __global__ void __launch_bounds__(pf::THREADS, 1) gemm_prefill_kernel(
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&bar->full[s], 1);
       mbar_init(&bar->empty[s], 1);
-      mbar_init(&bar->a_full[s], 4);
+    }
+    for (int a = 0; a < ASLOTS; ++a) {
+      mbar_init(&bar->a_full[a], 4);
+      mbar_init(&bar->a_empty[a], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bar->tmem_full[b], 1);
@@ -169,20 +174,21 @@ __global__ void __launch_bounds__(pf::THREADS, 1) gemm_prefill_kernel(
     // ------------------------------------------------------------------ MMA issuer
     const uint32_t idesc = idesc_i8(BW, bnt);
     const uint64_t x_desc0 = smem_desc_k128(smem_u32(sX));
-    int s = 0, ab = 0;
-    uint32_t ph = 0, aph = 0;
+    int s = 0, a = 0, ab = 0;
+    uint32_t sph = 0, aph = 0, abph = 0;
     bool ok = true, issued_any = false;
     for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
       bool got = true;
-      if (lane == 0) got = tc_wait(&bar->tmem_empty[ab], aph ^ 1u, limit_ns, abort_flag);
+      if (lane == 0) got = tc_wait(&bar->tmem_empty[ab], abph ^ 1u, limit_ns, abort_flag);
       if (!__shfl_sync(0xffffffffu, got, 0)) { ok = false; break; }
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(ab * MAX_BNT);
       for (int kb = 0; kb < KB; ++kb) {
-        if (lane == 0) got = tc_wait(&bar->a_full[s], ph, limit_ns, abort_flag);
+        // a_full of slot a implies the stage's TMA data landed (the unpack waited for it)
+        if (lane == 0) got = tc_wait(&bar->a_full[a], aph, limit_ns, abort_flag);
         if (!__shfl_sync(0xffffffffu, got, 0)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t a_tmem = tmem_base + static_cast<uint32_t>(A_COL0 + s * A_COLS);
+        const uint32_t a_tmem = tmem_base + static_cast<uint32_t>(A_COL0 + a * A_COLS);
         const uint64_t b_desc = x_desc0 + static_cast<uint64_t>(s * (X_BYTES >> 4));
 #pragma unroll
         for (int kk = 0; kk < BK / MMA_K; ++kk)
@@ -191,12 +197,15 @@ __global__ void __launch_bounds__(pf::THREADS, 1) gemm_prefill_kernel(
                           (kb | kk) != 0 ? 1u : 0u);
         issued_any = true;
         mma_commit_elect(&bar->empty[s]);
-        if (++s == STAGES) { s = 0; ph ^= 1u; }
+        mma_commit_elect(&bar->a_empty[a]);
+        if (++s == STAGES) { s = 0; sph ^= 1u; }
+        if (++a == ASLOTS) { a = 0; aph ^= 1u; }
       }
       if (!ok) break;
       mma_commit_elect(&bar->tmem_full[ab]);
-      if (++ab == 2) { ab = 0; aph ^= 1u; }
+      if (++ab == 2) { ab = 0; abph ^= 1u; }
     }
+    (void)sph;
     if (!ok && issued_any) {
       mma_commit_elect(&bar->drain);  // completes once every MMA issued above has finished
       if (lane == 0) mbar_wait(&bar->drain, 0u, 100000000ull);
@@ -218,13 +227,16 @@ __global__ void __launch_bounds__(pf::THREADS, 1) gemm_prefill_kernel(
       for (int kb = 0; kb < KB; ++kb, ++g) {
         if (static_cast<int>(g % UNPACK_SETS) != set) continue;
         const int s = static_cast<int>(g % STAGES);
+        const int a = static_cast<int>(g % ASLOTS);
         const uint32_t ph = static_cast<uint32_t>((g / STAGES) & 1);
-        const bool got = tc_wait(&bar->full[s], ph, limit_ns, abort_flag);
+        const uint32_t aph = static_cast<uint32_t>((g / ASLOTS) & 1);
+        const bool got = tc_wait(&bar->full[s], ph, limit_ns, abort_flag) &&
+                         tc_wait(&bar->a_empty[a], aph ^ 1u, limit_ns, abort_flag);
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
         const uint4* src = reinterpret_cast<const uint4*>(sW + s * WP_BYTES + r * 32);
         const uint4 first = src[h0], second = src[h0 ^ 1];
         const uint4 halves[2] = {h0 ? second : first, h0 ? first : second};
-        uint32_t a[32];  // the row's 128 codes of this K block, 4 per register
+        uint32_t codes[32];  // the row's 128 codes of this K block, 4 per register
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const uint4 p = halves[h];
@@ -232,17 +244,17 @@ __global__ void __launch_bounds__(pf::THREADS, 1) gemm_prefill_kernel(
 #pragma unroll
           for (int mq = 0; mq < 4; ++mq) {
             const int c = 16 * h + 4 * mq;  // column of trits 4c .. 4c + 15
-            a[c + 0] = words[mq] & 0x03030303u;
-            a[c + 1] = (words[mq] >> 2) & 0x03030303u;
-            a[c + 2] = (words[mq] >> 4) & 0x03030303u;
-            a[c + 3] = (words[mq] >> 6) & 0x03030303u;
+            codes[c + 0] = words[mq] & 0x03030303u;
+            codes[c + 1] = (words[mq] >> 2) & 0x03030303u;
+            codes[c + 2] = (words[mq] >> 4) & 0x03030303u;
+            codes[c + 3] = (words[mq] >> 6) & 0x03030303u;
           }
         }
-        tmem_st_x32(a_lane + static_cast<uint32_t>(s * A_COLS), a);
+        tmem_st_x32(a_lane + static_cast<uint32_t>(a * A_COLS), codes);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bar->a_full[s]);
+        if (lane == 0) mbar_arrive(&bar->a_full[a]);
       }
     }
   } else {

@@ -43,7 +43,7 @@ def _within_bound(got, ref, abs_terms, n):
 @pytest.mark.parametrize("M,N,K,x_dtype", [
     (8, 256, 256, torch.float32), (300, 640, 1536, torch.bfloat16),
     (130, 4096, 1536, torch.bfloat16), (64, 3200, 8640, torch.bfloat16),
-    (1000, 8640, 3200, torch.bfloat16), (5, 128, 64, torch.float32),
+    (520, 1024, 1536, torch.bfloat16), (5, 128, 64, torch.float32),
 ])
 def test_backward_matches_oracle(M, N, K, x_dtype):
     if not torch.cuda.is_available():
@@ -94,8 +94,7 @@ def test_backward_single_gradients_and_exact_cases():
     np.testing.assert_array_equal(gx.cpu().numpy(), ref_x.astype(np.float32))
     q, s = orc.quantize_acts(syn.bf16_bits(x))
     ref_w = orc.ste_grad_w(Gb, orc.dequant_acts_bf16(q, s))
-    # each grad_w entry sums over the tokens whose G row has its one entry at n: several
-    # tokens may share an n (M > N / 37 collisions): compare within the bound, exact where
-    # a single token contributes
-    single = np.bincount((np.arange(M) * 37) % N, minlength=N) <= 1
-    np.testing.assert_array_equal(gw.cpu().numpy()[single], ref_w[single].astype(np.float32))
+    # token t's one entry is at n = 37 t mod 512, distinct for the 128 tokens (37 is odd),
+    # so every grad_w entry has at most one term
+    assert np.bincount((np.arange(M) * 37) % N, minlength=N).max() == 1
+    np.testing.assert_array_equal(gw.cpu().numpy(), ref_w.astype(np.float32))
