@@ -410,6 +410,33 @@ def decode3_figure(bl, name: str, M: int, device, hbm_peak: float):
             "weight_bytes_2bit": N * K // 4, "weight_copies": copies}
 
 
+def backward_figure(bl, device, bf16_peak: float, M: int = 4096, name: str = "700m_up_1536x4096"):
+    """The straight-through backward of one BitLinear layer for a training batch of M tokens
+    (bf16 upstream gradient): grad_x (gamma G C) and grad_w (G^T X~) on the tcgen05 bf16
+    tensor cores, timed back to back; 2 M N K flops each."""
+    wl = syn.WORKLOADS[name]
+    N, K = wl["N"], wl["K"]
+    packed, gamma = packed_copies(bl, name, device, 1)[0]
+    packedT = bl.pack_transpose(packed)
+    x = syn.activations(M, K, seed=11, dtype=torch.bfloat16, device=device)
+    G = (syn.activations(M, N, seed=12, dtype=torch.float32, device=device) * 0.01).bfloat16()
+    n = bl.load_library().bitlinear_backward_workspace_size(M, N, K)
+    ws = torch.empty(n, dtype=torch.uint8, device=device)
+    fx = lambda: bl.backward(x, G, packedT, gamma, need_w=False, ws=ws)  # noqa: E731
+    fw = lambda: bl.backward(x, G, packedT, gamma, need_x=False, ws=ws)  # noqa: E731
+    fx(); fw()
+    torch.cuda.synchronize()
+    flops = 2.0 * M * N * K
+    ms_x = time_back_to_back([fx] * 4)
+    ms_w = time_back_to_back([fw] * 4)
+    tx = flops / (ms_x * 1e-3) / 1e12
+    tw = flops / (ms_w * 1e-3) / 1e12
+    return {"workload": name, "M": M, "grad_x_ms": ms_x, "grad_x_TFLOPs": tx,
+            "grad_x_frac_bf16": tx / bf16_peak, "grad_w_ms": ms_w, "grad_w_TFLOPs": tw,
+            "grad_w_frac_bf16": tw / bf16_peak,
+            "note": "grad_w includes the activation quantization and both transposes"}
+
+
 # LLaMA-70B-style layer matrices (out x in) and how many of each one layer holds; 80 layers.
 WQ_70B_SHAPES = [(8192, 8192, 2), (1024, 8192, 2), (28672, 8192, 3)]
 WQ_70B_LAYERS = 80
@@ -615,6 +642,7 @@ def main():
                                                ("700m_up_1536x4096", 1)]]
         others["weight_quant_70b"] = weight_quant_figures(bl, device, hbm_peak)
         others["sweep_3b_26_layers"] = sweep_3b_figures(bl, device, hbm_peak)
+        others["backward_ste"] = backward_figure(bl, device, bf16_peak)
     roofline["others"] = others
 
     cpu = None

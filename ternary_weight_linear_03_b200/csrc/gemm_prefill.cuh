@@ -14,17 +14,17 @@
 // from TMEM. Shared memory carries only the token tile (written by TMA, read by the MMA)
 // and the 4 KB packed tile: 56 KB per 128 x 192 x 128 block.
 //
-// Tiles: 128 weight rows (MMA M, TMEM lanes) x bnt <= 192 tokens (MMA N). TMEM (512
-// columns): two accumulators of 192 columns (the epilogue drains one while the MMAs fill
+// Tiles: 128 weight rows (MMA M, TMEM lanes) x bnt <= 176 tokens (MMA N). TMEM (512
+// columns): two accumulators of 176 columns (the epilogue drains one while the MMAs fill
 // the other) and ASLOTS unpacked K blocks of 32 columns. Shared memory holds STAGES > ASLOTS
 // TMA stages, deeper than TMEM allows A slots, so that the L2 latency of the token tiles
 // stays covered; stage g's weights go to slot g % ASLOTS once the MMAs of stage
 // g - ASLOTS, its last readers, have completed (their commit arrives on a_empty).
 //
-// Warps: 0-7 unpack in two sets of four that take alternate stages (each set's chain of
-// barrier wait, shared-memory load, tcgen05.st, wait::st and arrival per stage is longer
-// than the MMAs of one stage; thread r of a set owns weight row r, TMEM lane r), 8-11
-// epilogue (tcgen05.ld of their 32 lanes, rowsum, rescale, store), 12 TMA producer, 13
+// Warps: 0-11 unpack in three sets of four that take stages in turn (each set's chain of
+// barrier waits, shared-memory load, tcgen05.st, wait::st and arrival per stage is longer
+// than the MMAs of one stage; thread r of a set owns weight row r, TMEM lane r), 12-15
+// epilogue (tcgen05.ld of their 32 lanes, rowsum, rescale, store), 16 TMA producer, 17
 // TMEM owner and MMA issuer (whole-warp loop, one elected lane issues). Persistent: one CTA per SM walks the tiles,
 // consecutive CTAs taking consecutive token tiles of one weight tile (L2 reuse of both).
 // Every mbarrier wait is bounded; on a timeout the kernel records BL_ERR_TIMEOUT, waits
@@ -41,19 +41,23 @@ namespace pf {
 constexpr int BW = 128;                   // weight rows per tile (MMA M)
 constexpr int BK = 128;                   // K per stage (one 128-byte swizzle row of int8)
 constexpr int MMA_K = 32;                 // K per tcgen05.mma kind::i8
-constexpr int STAGES = 6;                 // TMA stages (token tile + packed weights)
-constexpr int ASLOTS = 4;                 // unpacked A slots in TMEM
-constexpr int MAX_BNT = 192;              // tokens per tile, at most (MMA N)
-constexpr int X_BYTES = MAX_BNT * BK;     // 24 KB token tile (128-byte swizzle)
+constexpr int STAGES = 7;                 // TMA stages (token tile + packed weights)
+constexpr int ASLOTS = 5;                 // unpacked A slots in TMEM
+constexpr int MAX_BNT = 176;              // tokens per tile, at most (MMA N)
+constexpr int X_BYTES = MAX_BNT * BK;     // 22 KB token tile (128-byte swizzle)
 constexpr int WP_BYTES = BW * BK / 4;     // 4 KB packed weight tile
 constexpr int A_COLS = BK / 4;            // TMEM columns of one unpacked K block
 constexpr int A_COL0 = 2 * MAX_BNT;       // first A slot column, after two accumulators
 constexpr int TMEM_COLS = 512;
-constexpr int UNPACK_SETS = 2;
-constexpr int THREADS = 448;
-static_assert(ASLOTS % UNPACK_SETS == 0, "each set keeps to its own A slots");
+constexpr int UNPACK_SETS = 3;
+constexpr int UNPACK_WARPS = 4 * UNPACK_SETS;
+constexpr int EPI_WARP0 = UNPACK_WARPS;        // 4 epilogue warps
+constexpr int TMA_WARP = EPI_WARP0 + 4;
+constexpr int MMA_WARP = TMA_WARP + 1;
+constexpr int THREADS = 32 * (MMA_WARP + 1);
 static_assert(A_COL0 + ASLOTS * A_COLS <= TMEM_COLS, "TMEM budget");
 static_assert(X_BYTES % 1024 == 0, "swizzle atoms of the token stages stay aligned");
+static_assert(EPI_WARP0 % 4 == 0, "epilogue warp q reads TMEM lanes 32 q");
 
 struct Barriers {
   uint64_t full[STAGES];     // token tile + packed weights of a stage landed
@@ -76,7 +80,7 @@ struct Shared {
 constexpr int SMEM_BYTES = 1024 /* alignment slack */ + STAGES * (X_BYTES + WP_BYTES) +
                            static_cast<int>(sizeof(Shared));
 
-// Token tile for M tokens: as even as the tile count allows, a multiple of 16, <= 192.
+// Token tile for M tokens: as even as the tile count allows, a multiple of 16, <= 176.
 __host__ __device__ constexpr int token_tile(int M) {
   const int tiles = (M + MAX_BNT - 1) / MAX_BNT;
   const int per = (M + tiles - 1) / tiles;
@@ -84,7 +88,7 @@ __host__ __device__ constexpr int token_tile(int M) {
 }
 }  // namespace pf
 
-__device__ __forceinline__ void epi4_bar_sync() {  // the 4 epilogue warps (8-11) only
+__device__ __forceinline__ void epi4_bar_sync() {  // the 4 epilogue warps only
   asm volatile("bar.sync 3, 128;" ::: "memory");
 }
 
@@ -131,7 +135,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1) gemm_prefill_kernel(
     bar->abort = 0;
     fence_mbar_init();
   }
-  if (warp == 13) {
+  if (warp == MMA_WARP) {
     tmem_alloc(&bar->tmem_base, TMEM_COLS);
     tmem_relinquish();
   }
@@ -141,7 +145,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1) gemm_prefill_kernel(
   const uint32_t tmem_base = bar->tmem_base;
   grid_dependency_wait();  // operands from the kernel before (no-op without the attribute)
 
-  if (warp == 12) {
+  if (warp == TMA_WARP) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       prefetch_tmap(&map_x);
@@ -170,7 +174,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1) gemm_prefill_kernel(
                     100000000ull);
       }
     }
-  } else if (warp == 13) {
+  } else if (warp == MMA_WARP) {
     // ------------------------------------------------------------------ MMA issuer
     const uint32_t idesc = idesc_i8(BW, bnt);
     const uint64_t x_desc0 = smem_desc_k128(smem_u32(sX));
@@ -211,7 +215,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1) gemm_prefill_kernel(
       if (lane == 0) mbar_wait(&bar->drain, 0u, 100000000ull);
       __syncwarp();
     }
-  } else if (warp < 8) {
+  } else if (warp < UNPACK_WARPS) {
     // ------------------------------------------------------------------ unpack warps
     const int set = warp >> 2;   // stages g with g % UNPACK_SETS == set
     const int wq = warp & 3;     // TMEM lane quarter
@@ -259,8 +263,8 @@ __global__ void __launch_bounds__(pf::THREADS, 1) gemm_prefill_kernel(
     }
   } else {
     // ------------------------------------------------------------------ epilogue
-    const int q = warp - 8;     // TMEM lanes 32q .. 32q + 31
-    const int et = threadIdx.x - 256;  // 0..127
+    const int q = warp - EPI_WARP0;  // TMEM lanes 32q .. 32q + 31
+    const int et = threadIdx.x - 32 * EPI_WARP0;  // 0..127
     const float gamma = (OM == 2) ? 0.0f : *gamma_ptr;
     int ab = 0;
     uint32_t aph = 0;
@@ -337,7 +341,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1) gemm_prefill_kernel(
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 13) {
+  if (warp == MMA_WARP) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem_base, TMEM_COLS);

@@ -290,22 +290,20 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(
       }
     const long long stride = warps_total * RPW;  // rows between two turns of this warp
     const long long rows_of = (static_cast<long long>(blockIdx.x) * kGemvWarps + warp) * RPW;
-    // Which of this lane's chunks exist (fixed for every row), and the row pointer stepped
-    // by whole turns, so the loop carries no per-chunk bounds arithmetic.
-    bool cval[kGemvRegChunks];
-#pragma unroll
-    for (int u = 0; u < kGemvRegChunks; ++u) cval[u] = (sub + u * LPR) < CPR;
-    const long long row_words = K >> 6;  // 16-byte chunks per row
-    const uint4* lane_base = reinterpret_cast<const uint4*>(packed) + sub;
+    uint4 wv[kGemvRegChunks];
     auto load_row = [&](long long row, uint4 (&w)[kGemvRegChunks]) {
-      const uint4* prow = lane_base + row * row_words;
+      const uint4* prow = reinterpret_cast<const uint4*>(packed + row * (K >> 2));
 #pragma unroll
-      for (int u = 0; u < kGemvRegChunks; ++u)
-        w[u] = (row < N && cval[u]) ? ld_stream_v4(prow + u * LPR) : make_uint4(0u, 0u, 0u, 0u);
+      for (int u = 0; u < kGemvRegChunks; ++u) {
+        const int c = sub + u * LPR;
+        w[u] = (row < N && c < CPR) ? ld_stream_v4(prow + c) : make_uint4(0u, 0u, 0u, 0u);
+      }
     };
-    // One row: its sum over this lane's chunks, reduced over the row's lanes, rescaled and
-    // stored by the row's first lane.
-    auto do_row = [&](long long n, const uint4 (&w)[kGemvRegChunks]) {
+    load_row(rows_of + rsel, wv);
+    for (long long rbase = rows_of; rbase < N; rbase += stride) {
+      const long long n = rbase + rsel;
+      uint4 wn[kGemvRegChunks];
+      load_row(n + stride, wn);  // next turn's row, in flight while this one is summed
       int ch[MT][4];
 #pragma unroll
       for (int t = 0; t < MT; ++t)
@@ -313,7 +311,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(
         for (int j = 0; j < 4; ++j) ch[t][j] = 0;
 #pragma unroll
       for (int u = 0; u < kGemvRegChunks; ++u) {
-        const uint32_t words[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
+        const uint32_t words[4] = {wv[u].x, wv[u].y, wv[u].z, wv[u].w};
 #pragma unroll
         for (int g = 0; g < 4; ++g)
 #pragma unroll
@@ -341,18 +339,8 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(
           }
         }
       }
-    };
-    // Two rows per turn with ping-pong registers: each row's loads are in flight while the
-    // row before is summed, with no register copies between turns.
-    uint4 wa[kGemvRegChunks], wb[kGemvRegChunks];
-    load_row(rows_of + rsel, wa);
-    for (long long rbase = rows_of; rbase < N; rbase += 2 * stride) {
-      const long long n = rbase + rsel;
-      load_row(n + stride, wb);
-      do_row(n, wa);
-      if (rbase + stride >= N) break;  // the same for the whole warp
-      load_row(n + 2 * stride, wa);
-      do_row(n + stride, wb);
+#pragma unroll
+      for (int u = 0; u < kGemvRegChunks; ++u) wv[u] = wn[u];
     }
   } else {
     // ------------------------------------------------------------ activations in smem

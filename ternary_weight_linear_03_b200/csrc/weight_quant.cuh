@@ -384,6 +384,12 @@ __global__ void __launch_bounds__(kWqThreads) weight_quant_kernel(
                  ? __uint_as_float(static_cast<uint32_t>(base + kWqWindow) << 23)
                  : __int_as_float(0x7f800000);
     }
+    // Non-negative floats order like their bit patterns: the window test and (single-read
+    // mode) the threshold and band tests are single unsigned compares of |w|'s bits.
+    const uint32_t lo_b = __float_as_uint(lo_f), span_b = __float_as_uint(hi_f) - lo_b;
+    const uint32_t t_b = __float_as_uint(t_hat);
+    const uint32_t band_b = __float_as_uint(band_lo);
+    const uint32_t bspan_b = __float_as_uint(band_hi) - band_b;
 #pragma unroll
     for (int i = 0; i < kWqChunks; ++i) {
       float w[E];
@@ -391,11 +397,12 @@ __global__ void __launch_bounds__(kWqThreads) weight_quant_kernel(
       bool out_any = false;
 #pragma unroll
       for (int e = 0; e < E; ++e) {
-        const float a = abs_bits(w[e]);
-        const bool in = (a >= lo_f) & (a < hi_f);
+        const uint32_t ab = __float_as_uint(w[e]) & 0x7fffffffu;
+        const bool in = (ab - lo_b) < span_b;  // lo_f <= |w| < hi_f
         out_any |= !in;
-        if (e & 1) acc1 += static_cast<double>(in ? a : 0.0f);  // exact: see the header
-        else acc0 += static_cast<double>(in ? a : 0.0f);
+        const float a = __uint_as_float(in ? ab : 0u);
+        if (e & 1) acc1 += static_cast<double>(a);  // exact: see the header
+        else acc0 += static_cast<double>(a);
       }
       if (out_any) {  // rare: zeros and values outside the window
 #pragma unroll
@@ -410,9 +417,10 @@ __global__ void __launch_bounds__(kWqThreads) weight_quant_kernel(
         uint32_t bits = 0u;
 #pragma unroll
         for (int e = 0; e < E; ++e) {
-          const float a = abs_bits(w[e]);
-          bits += ((a >= t_hat) ? 2u - ((__float_as_uint(w[e]) >> 30) & 2u) : 1u) * mulA[e];
-          if (c < nchunks && a >= band_lo && a <= band_hi) {
+          const uint32_t wb = __float_as_uint(w[e]);
+          const uint32_t ab = wb & 0x7fffffffu;
+          bits += ((ab >= t_b) ? 2u - ((wb >> 30) & 2u) : 1u) * mulA[e];  // |w| >= T^
+          if (c < nchunks && (ab - band_b) <= bspan_b) {  // |w| within the band
             const unsigned idx = atomicAdd(&s_cnt, 1u);
             if (idx < static_cast<unsigned>(kWqListCap))
               list[static_cast<long long>(blockIdx.x) * kWqListCap + idx] = make_uint2(
