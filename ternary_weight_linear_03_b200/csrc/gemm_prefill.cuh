@@ -14,18 +14,19 @@
 // from TMEM. Shared memory carries only the token tile (written by TMA, read by the MMA)
 // and the 4 KB packed tile: 56 KB per 128 x 192 x 128 block.
 //
-// Tiles: 128 weight rows (MMA M, TMEM lanes) x bnt <= 176 tokens (MMA N). TMEM (512
-// columns): two accumulators of 176 columns (the epilogue drains one while the MMAs fill
+// Tiles: 128 weight rows (MMA M, TMEM lanes) x bnt <= 192 tokens (MMA N). TMEM (512
+// columns): two accumulators of 192 columns (the epilogue drains one while the MMAs fill
 // the other) and ASLOTS unpacked K blocks of 32 columns. Shared memory holds STAGES > ASLOTS
 // TMA stages, deeper than TMEM allows A slots, so that the L2 latency of the token tiles
 // stays covered; stage g's weights go to slot g % ASLOTS once the MMAs of stage
 // g - ASLOTS, its last readers, have completed (their commit arrives on a_empty).
 //
-// Warps: 0-11 unpack in three sets of four that take stages in turn (each set's chain of
+// Warps: 0-7 unpack in two sets of four that take alternate stages (each set's chain of
 // barrier waits, shared-memory load, tcgen05.st, wait::st and arrival per stage is longer
-// than the MMAs of one stage; thread r of a set owns weight row r, TMEM lane r), 12-15
-// epilogue (tcgen05.ld of their 32 lanes, rowsum, rescale, store), 16 TMA producer, 17
-// TMEM owner and MMA issuer (whole-warp loop, one elected lane issues). Persistent: one CTA per SM walks the tiles,
+// than the MMAs of one stage; thread r of a set owns weight row r, TMEM lane r), 8-11
+// epilogue (tcgen05.ld of their 32 lanes, rowsum, rescale, store), 12 TMA producer, 13
+// TMEM owner and MMA issuer (whole-warp loop, one elected lane issues). Three sets over five
+// slots of 176 columns measured slower on B200 (0.89 ms against 0.77 ms at M = 4096). Persistent: one CTA per SM walks the tiles,
 // consecutive CTAs taking consecutive token tiles of one weight tile (L2 reuse of both).
 // Every mbarrier wait is bounded; on a timeout the kernel records BL_ERR_TIMEOUT, waits
 // (bounded) for its own copies and MMAs, frees TMEM and exits.
@@ -42,14 +43,14 @@ constexpr int BW = 128;                   // weight rows per tile (MMA M)
 constexpr int BK = 128;                   // K per stage (one 128-byte swizzle row of int8)
 constexpr int MMA_K = 32;                 // K per tcgen05.mma kind::i8
 constexpr int STAGES = 7;                 // TMA stages (token tile + packed weights)
-constexpr int ASLOTS = 5;                 // unpacked A slots in TMEM
-constexpr int MAX_BNT = 176;              // tokens per tile, at most (MMA N)
-constexpr int X_BYTES = MAX_BNT * BK;     // 22 KB token tile (128-byte swizzle)
+constexpr int ASLOTS = 4;                 // unpacked A slots in TMEM
+constexpr int MAX_BNT = 192;              // tokens per tile, at most (MMA N)
+constexpr int X_BYTES = MAX_BNT * BK;     // 24 KB token tile (128-byte swizzle)
 constexpr int WP_BYTES = BW * BK / 4;     // 4 KB packed weight tile
 constexpr int A_COLS = BK / 4;            // TMEM columns of one unpacked K block
 constexpr int A_COL0 = 2 * MAX_BNT;       // first A slot column, after two accumulators
 constexpr int TMEM_COLS = 512;
-constexpr int UNPACK_SETS = 3;
+constexpr int UNPACK_SETS = 2;
 constexpr int UNPACK_WARPS = 4 * UNPACK_SETS;
 constexpr int EPI_WARP0 = UNPACK_WARPS;        // 4 epilogue warps
 constexpr int TMA_WARP = EPI_WARP0 + 4;
@@ -58,6 +59,7 @@ constexpr int THREADS = 32 * (MMA_WARP + 1);
 static_assert(A_COL0 + ASLOTS * A_COLS <= TMEM_COLS, "TMEM budget");
 static_assert(X_BYTES % 1024 == 0, "swizzle atoms of the token stages stay aligned");
 static_assert(EPI_WARP0 % 4 == 0, "epilogue warp q reads TMEM lanes 32 q");
+static_assert(ASLOTS % UNPACK_SETS == 0, "each set keeps to its own A slots");
 
 struct Barriers {
   uint64_t full[STAGES];     // token tile + packed weights of a stage landed
@@ -80,7 +82,7 @@ struct Shared {
 constexpr int SMEM_BYTES = 1024 /* alignment slack */ + STAGES * (X_BYTES + WP_BYTES) +
                            static_cast<int>(sizeof(Shared));
 
-// Token tile for M tokens: as even as the tile count allows, a multiple of 16, <= 176.
+// Token tile for M tokens: as even as the tile count allows, a multiple of 16, <= 192.
 __host__ __device__ constexpr int token_tile(int M) {
   const int tiles = (M + MAX_BNT - 1) / MAX_BNT;
   const int per = (M + tiles - 1) / tiles;
