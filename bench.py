@@ -56,6 +56,10 @@ def parse():
     p.add_argument("--workload", default=HEADLINE)
     p.add_argument("--M", type=int, default=None, help="tokens (default: the workload's largest)")
     p.add_argument("--no-others", action="store_true", help="skip the secondary figures")
+    p.add_argument("--figure", default="headline",
+                   choices=["headline", "decode", "decode_base3", "weight_quant", "sweep",
+                            "backward"],
+                   help="run one secondary figure alone and print it (for profiling)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     a = p.parse_args()
@@ -64,7 +68,8 @@ def parse():
     return a
 
 
-KERNEL_SOURCES = {"weight_quant_kernel": "weight_quant.cuh", "gemm_tc_kernel": "gemm_tc.cuh",
+KERNEL_SOURCES = {"weight_quant_kernel": "weight_quant.cuh",
+                  "gemm_prefill_kernel": "gemm_prefill.cuh",
                   "gemm_skinny_kernel": "gemm_skinny.cuh", "gemv_kernel": "gemv.cuh"}
 
 
@@ -257,25 +262,6 @@ def time_back_to_back(calls, reps: int = 5):
     torch.cuda.synchronize()
     del g
     return s.elapsed_time(e) / (reps * len(calls))
-
-
-def time_in_graph(calls, reps: int = 3):
-    """Per-call device times (ms) of a list of library calls: one CUDA graph with an event
-    node before every call and after the last, replayed `reps` times; the times are those
-    of the last replay. Every call must have run eagerly once before (kernel set-up)."""
-    evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(calls) + 1)]
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g):
-        for i, c in enumerate(calls):
-            evs[i].record()
-            c()
-        evs[-1].record()
-    for _ in range(reps):
-        g.replay()
-    torch.cuda.synchronize()
-    times = [evs[i].elapsed_time(evs[i + 1]) for i in range(len(calls))]
-    del g
-    return times
 
 
 def forward_launches(bl, M: int, N: int, K: int) -> int:
@@ -476,6 +462,31 @@ def weight_quant_figures(bl, device, hbm_peak: float):
 # ----------------------------------------------------------------------------- main
 
 
+DECODE_SHAPES = [("70b_up_8192x28672", 1), ("70b_up_8192x28672", 16), ("70b_up_8192x28672", 176),
+                 ("70b_down_28672x8192", 1), ("70b_down_28672x8192", 16),
+                 ("70b_down_28672x8192", 176), ("700m_up_1536x4096", 1),
+                 ("700m_up_1536x4096", 4), ("700m_up_1536x4096", 16)]
+BASE3_SHAPES = [("70b_up_8192x28672", 1), ("70b_down_28672x8192", 1), ("70b_up_8192x28672", 4),
+                ("700m_up_1536x4096", 1)]
+
+
+def secondary(bl, which: str, device):
+    """One secondary figure (all of them for the headline line's roofline.others)."""
+    hbm_peak, bf16_peak, _, _ = peaks()
+    i8_peak = 2.0 * bf16_peak
+    if which == "decode":
+        return [decode_figure(bl, n, m, device, hbm_peak, i8_peak) for n, m in DECODE_SHAPES]
+    if which == "decode_base3":
+        return [decode3_figure(bl, n, m, device, hbm_peak) for n, m in BASE3_SHAPES]
+    if which == "weight_quant":
+        return weight_quant_figures(bl, device, hbm_peak)
+    if which == "sweep":
+        return sweep_3b_figures(bl, device, hbm_peak)
+    if which == "backward":
+        return backward_figure(bl, device, bf16_peak)
+    raise ValueError(which)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -483,6 +494,14 @@ def main():
         return
 
     import ternary_weight_linear_03_b200 as bl
+
+    if args.figure != "headline":
+        if not torch.cuda.is_available():
+            raise SystemExit("bench.py needs a CUDA device (no CPU fallback)")
+        device = torch.device("cuda", 0)
+        torch.cuda.set_device(device)
+        print(json.dumps({"figure": args.figure, "result": secondary(bl, args.figure, device)}))
+        return
 
     rank, world, local = bldist.rank_env()
     if not torch.cuda.is_available():
@@ -522,18 +541,14 @@ def main():
     torch.cuda.synchronize()
     assert bl.get_device_status() == 0
 
-    # One CUDA graph per copy (event node, forward, event node); the timed loop replays
-    # them in turn, one graph per step.
-    graphs, evs = [], []
+    # One CUDA graph per copy holding that step's forward; the timed loop replays them in
+    # turn, one graph per step.
+    graphs = []
     for i in range(copies):
-        ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            ev[0].record()
             step(i)
-            ev[1].record()
         graphs.append(g)
-        evs.append(ev)
     for i in range(max(3, args.warmup)):
         graphs[i % copies].replay()
     torch.cuda.synchronize()
@@ -556,7 +571,6 @@ def main():
     status = bl.get_device_status()
     if status != 0:
         raise SystemExit(f"device status {bl.status_string(status)} after the timed region")
-    fw_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs[:min(copies, args.steps)])
     del graphs
     tokens = M * args.steps * world
     value = tokens / (elapsed_ms * 1e-3)
@@ -600,6 +614,9 @@ def main():
         return
 
     # ------------------------------------------------------------------ roofline
+    # One step is one bitlinear_forward call (its kernels back to back), so the launch time
+    # is the timed region's average step.
+    fw_ms = elapsed_ms / args.steps
     path, splits = bl.debug_plan(M, N, K)
     fw_ops = 2.0 * M * N * K
     fw_bytes = N * K // 4 + M * K * 2 + M * N * 2
@@ -607,14 +624,14 @@ def main():
         # the activation quantization of the same batch timed alone, for the GEMM's share
         xq_calls = [(lambda i=i: bl.quantize_acts(xs[i])) for i in range(min(copies, 4))]
         xq_calls[0]()
-        aq_ms = statistics.mean(time_in_graph(xq_calls))
+        aq_ms = time_back_to_back(xq_calls)
         achieved = fw_ops / (fw_ms * 1e-3) / 1e12
         roofline = {"bound": "tensor", "achieved": achieved, "peak": i8_peak, "unit": "TFLOP/s",
                     "frac": achieved / i8_peak,
-                    "traffic": ncu_traffic("gemm_tc_kernel", name, M),
+                    "traffic": ncu_traffic("gemm_prefill_kernel", name, M),
                     "peak_source": f"{peak_kind} bf16 burst x 2 (int8 ops, nominal ratio)",
-                    "kernel": "bitlinear_forward = act_quant_kernel + gemm_tc_kernel "
-                              "(tcgen05 kind::i8)",
+                    "kernel": "bitlinear_forward = act_quant_kernel + gemm_prefill_kernel "
+                              "(tcgen05 kind::i8, weights in TMEM)",
                     "algorithmic_ops_per_launch": fw_ops, "ms_per_launch": fw_ms,
                     "act_quant_ms": aq_ms, "gemm_ms_est": fw_ms - aq_ms,
                     "gemm_frac_est": fw_ops / ((fw_ms - aq_ms) * 1e-3) / 1e12 / i8_peak}
@@ -628,21 +645,11 @@ def main():
 
     others = {}
     if not args.no_others:
-        others["decode"] = [decode_figure(bl, n, m, device, hbm_peak, i8_peak)
-                            for n, m in [("70b_up_8192x28672", 1), ("70b_up_8192x28672", 16),
-                                         ("70b_up_8192x28672", 176),
-                                         ("70b_down_28672x8192", 1), ("70b_down_28672x8192", 16),
-                                         ("70b_down_28672x8192", 176),
-                                         ("700m_up_1536x4096", 1), ("700m_up_1536x4096", 4),
-                                         ("700m_up_1536x4096", 16)]]
-        others["decode_base3"] = [decode3_figure(bl, n, m, device, hbm_peak)
-                                  for n, m in [("70b_up_8192x28672", 1),
-                                               ("70b_down_28672x8192", 1),
-                                               ("70b_up_8192x28672", 4),
-                                               ("700m_up_1536x4096", 1)]]
-        others["weight_quant_70b"] = weight_quant_figures(bl, device, hbm_peak)
-        others["sweep_3b_26_layers"] = sweep_3b_figures(bl, device, hbm_peak)
-        others["backward_ste"] = backward_figure(bl, device, bf16_peak)
+        others["decode"] = secondary(bl, "decode", device)
+        others["decode_base3"] = secondary(bl, "decode_base3", device)
+        others["weight_quant_70b"] = secondary(bl, "weight_quant", device)
+        others["sweep_3b_26_layers"] = secondary(bl, "sweep", device)
+        others["backward_ste"] = secondary(bl, "backward", device)
     roofline["others"] = others
 
     cpu = None

@@ -235,6 +235,19 @@ bool make_map_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t r
 }
 
 // ------------------------------------------------------------------ GEMV launch
+// Lanes per weight row of the GEMV (log2): the fewest lanes whose blocks still cover every
+// SM (16 warps x 32 / lanes rows per block) when the matrix has few rows, else the count
+// that wastes the fewest lane slots on the row's chunks.
+int choose_lpr_log2(int cpr);
+int gemv_lpr_log2(int cpr, int N) {
+  const int best = choose_lpr_log2(cpr);
+  for (int l = best; l <= 5; ++l) {
+    const long long rows_per_block = static_cast<long long>(bl::kGemvWarps) * (32 >> l);
+    if ((N + rows_per_block - 1) / rows_per_block >= num_sms()) return l;
+  }
+  return 5;
+}
+
 int choose_lpr_log2(int cpr) {
   int best = 5;
   long long best_cost = (cpr + 31) / 32 * 32;
@@ -258,7 +271,7 @@ bl_status launch_gemv_t(const void* x, const uint8_t* packed, const float* gamma
                                                     smem) != cudaSuccess ||
       blocks_per_sm < 1)
     blocks_per_sm = 1;
-  const int lpr_log2 = choose_lpr_log2(K / 64);
+  const int lpr_log2 = gemv_lpr_log2(K / 64, N);
   const long long rows_per_block = static_cast<long long>(bl::kGemvWarps) * (32 >> lpr_log2) * R;
   const long long need = (N + rows_per_block - 1) / rows_per_block;
   const int grid = static_cast<int>(std::min<long long>(need, 1ll * blocks_per_sm * num_sms()));
@@ -269,16 +282,16 @@ bl_status launch_gemv_t(const void* x, const uint8_t* packed, const float* gamma
 
 // Activations stay in registers for one token when a lane owns at most kGemvRegChunks
 // chunks of a row (two tokens would spill).
-bool gemv_x_in_registers(int M, int K) {
+bool gemv_x_in_registers(int M, int N, int K) {
   const int cpr = K / 64;
-  const int lpr = 1 << choose_lpr_log2(cpr);
+  const int lpr = 1 << gemv_lpr_log2(cpr, N);
   return M == 1 && (cpr + lpr - 1) / lpr <= bl::kGemvRegChunks;
 }
 
 // Rows summed at once per warp on the shared-memory path: two when one warp covers a
 // whole row (large K) and there are rows enough for every warp of the GPU twice over.
 bool gemv_two_rows(int N, int K) {
-  return choose_lpr_log2(K / 64) == 5 && N >= 2 * bl::kGemvWarps * num_sms();
+  return gemv_lpr_log2(K / 64, N) == 5 && N >= 2 * bl::kGemvWarps * num_sms();
 }
 
 template <int MT, int XM, int OM>
@@ -294,7 +307,7 @@ bl_status launch_gemv_m(const void* x, const uint8_t* packed, const float* gamma
                         int M, int N, int K, cudaStream_t s, const ChainOpts& o) {
   switch (M) {
     case 1:
-      return gemv_x_in_registers(M, K)
+      return gemv_x_in_registers(M, N, K)
                  ? launch_gemv_t<1, XM, OM, true, 1>(x, packed, gamma, y, N, K, s, o)
                  : launch_gemv_r<1, XM, OM>(x, packed, gamma, y, N, K, s, o);
     case 2: return launch_gemv_r<2, XM, OM>(x, packed, gamma, y, N, K, s, o);
