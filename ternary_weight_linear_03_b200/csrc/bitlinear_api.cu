@@ -235,16 +235,24 @@ bool make_map_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t r
 }
 
 // ------------------------------------------------------------------ GEMV launch
-// Lanes per weight row of the GEMV (log2): the fewest lanes whose blocks still cover every
-// SM (16 warps x 32 / lanes rows per block) when the matrix has few rows, else the count
-// that wastes the fewest lane slots on the row's chunks.
+// Lanes per weight row of the GEMV (log2). Small matrices need more lanes per row to give
+// every SM work, at the price of idle lanes on short rows; measured on B200 (3B, 700M
+// shapes), the balance is the fewest lanes whose blocks (16 warps x 32 / lanes rows each)
+// cover at least half the SMs, and for one token the fewest such lanes that still keep
+// the row's activations in registers (at most kGemvRegChunks chunks per lane).
 int choose_lpr_log2(int cpr);
-int gemv_lpr_log2(int cpr, int N) {
+int gemv_lpr_log2(int cpr, int N, int M) {
   const int best = choose_lpr_log2(cpr);
-  for (int l = best; l <= 5; ++l) {
+  const long long half = (num_sms() + 1) / 2;
+  auto blocks = [&](int l) {
     const long long rows_per_block = static_cast<long long>(bl::kGemvWarps) * (32 >> l);
-    if ((N + rows_per_block - 1) / rows_per_block >= num_sms()) return l;
-  }
+    return (N + rows_per_block - 1) / rows_per_block;
+  };
+  if (M == 1)
+    for (int l = best; l <= 5; ++l)
+      if (((cpr + (1 << l) - 1) >> l) <= bl::kGemvRegChunks && blocks(l) >= half) return l;
+  for (int l = best; l <= 5; ++l)
+    if (blocks(l) >= half) return l;
   return 5;
 }
 
@@ -271,7 +279,7 @@ bl_status launch_gemv_t(const void* x, const uint8_t* packed, const float* gamma
                                                     smem) != cudaSuccess ||
       blocks_per_sm < 1)
     blocks_per_sm = 1;
-  const int lpr_log2 = gemv_lpr_log2(K / 64, N);
+  const int lpr_log2 = gemv_lpr_log2(K / 64, N, MT);
   const long long rows_per_block = static_cast<long long>(bl::kGemvWarps) * (32 >> lpr_log2) * R;
   const long long need = (N + rows_per_block - 1) / rows_per_block;
   const int grid = static_cast<int>(std::min<long long>(need, 1ll * blocks_per_sm * num_sms()));
@@ -284,20 +292,20 @@ bl_status launch_gemv_t(const void* x, const uint8_t* packed, const float* gamma
 // chunks of a row (two tokens would spill).
 bool gemv_x_in_registers(int M, int N, int K) {
   const int cpr = K / 64;
-  const int lpr = 1 << gemv_lpr_log2(cpr, N);
+  const int lpr = 1 << gemv_lpr_log2(cpr, N, M);
   return M == 1 && (cpr + lpr - 1) / lpr <= bl::kGemvRegChunks;
 }
 
 // Rows summed at once per warp on the shared-memory path: two when one warp covers a
 // whole row (large K) and there are rows enough for every warp of the GPU twice over.
-bool gemv_two_rows(int N, int K) {
-  return gemv_lpr_log2(K / 64, N) == 5 && N >= 2 * bl::kGemvWarps * num_sms();
+bool gemv_two_rows(int M, int N, int K) {
+  return gemv_lpr_log2(K / 64, N, M) == 5 && N >= 2 * bl::kGemvWarps * num_sms();
 }
 
 template <int MT, int XM, int OM>
 bl_status launch_gemv_r(const void* x, const uint8_t* packed, const float* gamma, void* y,
                         int N, int K, cudaStream_t s, const ChainOpts& o) {
-  return gemv_two_rows(N, K)
+  return gemv_two_rows(MT, N, K)
              ? launch_gemv_t<MT, XM, OM, false, 2>(x, packed, gamma, y, N, K, s, o)
              : launch_gemv_t<MT, XM, OM, false, 1>(x, packed, gamma, y, N, K, s, o);
 }
