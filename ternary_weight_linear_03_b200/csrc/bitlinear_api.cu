@@ -236,10 +236,11 @@ bool make_map_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t r
 
 // ------------------------------------------------------------------ GEMV launch
 // Lanes per weight row of the GEMV (log2). Small matrices need more lanes per row to give
-// every SM work, at the price of idle lanes on short rows; measured on B200 (3B, 700M
-// shapes), the balance is the fewest lanes whose blocks (16 warps x 32 / lanes rows each)
-// cover at least half the SMs, and for one token the fewest such lanes that still keep
-// the row's activations in registers (at most kGemvRegChunks chunks per lane).
+// every SM work, at the price of idle lanes on short rows. Measured on B200 (3B and 700M
+// shapes): for one token, the fewest lanes that keep the row's activations in registers
+// (at most kGemvRegChunks chunks per lane) with blocks (16 warps x 32 / lanes rows each)
+// for at least half the SMs; otherwise the fewest lanes whose blocks cover every SM for
+// long rows (64 chunks or more), half of them for short rows.
 int choose_lpr_log2(int cpr);
 int gemv_lpr_log2(int cpr, int N, int M) {
   const int best = choose_lpr_log2(cpr);
@@ -251,8 +252,9 @@ int gemv_lpr_log2(int cpr, int N, int M) {
   if (M == 1)
     for (int l = best; l <= 5; ++l)
       if (((cpr + (1 << l) - 1) >> l) <= bl::kGemvRegChunks && blocks(l) >= half) return l;
+  const long long want = (cpr >= 64) ? num_sms() : half;
   for (int l = best; l <= 5; ++l)
-    if (blocks(l) >= half) return l;
+    if (blocks(l) >= want) return l;
   return 5;
 }
 

@@ -19,7 +19,7 @@
 // the other) and ASLOTS unpacked K blocks of 32 columns. Shared memory holds STAGES > ASLOTS
 // TMA stages, deeper than TMEM allows A slots, so that the L2 latency of the token tiles
 // stays covered. The unpack warps hand the MMA warp GST stages at a time (one barrier wait
-// and 8 MMAs per handoff): group h's weights go to group slot h % NGS (GST A slots) once
+// and 4 GST MMAs per handoff): group h's weights go to group slot h % NGS (GST A slots) once
 // the MMAs of group h - NGS, its last readers, have completed (their commit arrives on
 // a_empty).
 //
@@ -53,7 +53,7 @@ constexpr int A_COLS = BK / 4;            // TMEM columns of one unpacked K bloc
 constexpr int A_COL0 = 2 * MAX_BNT;       // first A slot column, after two accumulators
 constexpr int TMEM_COLS = 512;
 constexpr int UNPACK_SETS = 2;
-constexpr int GST = 2;                    // stages per handoff group (one wait, 8 MMAs)
+constexpr int GST = 1;                    // stages per handoff group (2 measured slower)
 constexpr int NGS = ASLOTS / GST;         // group slots in TMEM
 constexpr int UNPACK_WARPS = 4 * UNPACK_SETS;
 constexpr int EPI_WARP0 = UNPACK_WARPS;        // 4 epilogue warps
