@@ -18,12 +18,10 @@
 // columns): two accumulators of 192 columns (the epilogue drains one while the MMAs fill
 // the other) and ASLOTS unpacked K blocks of 32 columns. Shared memory holds STAGES > ASLOTS
 // TMA stages, deeper than TMEM allows A slots, so that the L2 latency of the token tiles
-// stays covered. The unpack warps hand the MMA warp GST stages at a time (one barrier wait
-// and 4 GST MMAs per handoff): group h's weights go to group slot h % NGS (GST A slots) once
-// the MMAs of group h - NGS, its last readers, have completed (their commit arrives on
-// a_empty).
+// stays covered; stage g's weights go to slot g % ASLOTS once the MMAs of stage
+// g - ASLOTS, its last readers, have completed (their commit arrives on a_empty).
 //
-// Warps: 0-7 unpack in two sets of four that take alternate groups (each set's chain of
+// Warps: 0-7 unpack in two sets of four that take alternate stages (each set's chain of
 // barrier waits, shared-memory load, tcgen05.st, wait::st and arrival per stage is longer
 // than the MMAs of one stage; thread r of a set owns weight row r, TMEM lane r), 8-11
 // epilogue (tcgen05.ld of their 32 lanes, rowsum, rescale, store), 12 TMA producer, 13
@@ -53,8 +51,6 @@ constexpr int A_COLS = BK / 4;            // TMEM columns of one unpacked K bloc
 constexpr int A_COL0 = 2 * MAX_BNT;       // first A slot column, after two accumulators
 constexpr int TMEM_COLS = 512;
 constexpr int UNPACK_SETS = 2;
-constexpr int GST = 1;                    // stages per handoff group (2 measured slower)
-constexpr int NGS = ASLOTS / GST;         // group slots in TMEM
 constexpr int UNPACK_WARPS = 4 * UNPACK_SETS;
 constexpr int EPI_WARP0 = UNPACK_WARPS;        // 4 epilogue warps
 constexpr int TMA_WARP = EPI_WARP0 + 4;
@@ -63,13 +59,13 @@ constexpr int THREADS = 32 * (MMA_WARP + 1);
 static_assert(A_COL0 + ASLOTS * A_COLS <= TMEM_COLS, "TMEM budget");
 static_assert(X_BYTES % 1024 == 0, "swizzle atoms of the token stages stay aligned");
 static_assert(EPI_WARP0 % 4 == 0, "epilogue warp q reads TMEM lanes 32 q");
-static_assert(ASLOTS % GST == 0 && NGS % UNPACK_SETS == 0, "each set keeps to its own slots");
+static_assert(ASLOTS % UNPACK_SETS == 0, "each set keeps to its own A slots");
 
 struct Barriers {
   uint64_t full[STAGES];     // token tile + packed weights of a stage landed
   uint64_t empty[STAGES];    // the stage's MMAs are done (its shared memory is free)
-  uint64_t a_full[NGS];      // a group's weights are in this group slot
-  uint64_t a_empty[NGS];     // the MMAs that read this group slot are done
+  uint64_t a_full[ASLOTS];   // a stage's weights are in this TMEM slot
+  uint64_t a_empty[ASLOTS];  // the MMAs that read this slot are done
   uint64_t tmem_full[2];
   uint64_t tmem_empty[2];
   uint64_t drain;
@@ -129,7 +125,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1) gemm_prefill_kernel(
       mbar_init(&bar->full[s], 1);
       mbar_init(&bar->empty[s], 1);
     }
-    for (int a = 0; a < NGS; ++a) {
+    for (int a = 0; a < ASLOTS; ++a) {
       mbar_init(&bar->a_full[a], 4);
       mbar_init(&bar->a_empty[a], 1);
     }
@@ -184,9 +180,8 @@ __global__ void __launch_bounds__(pf::THREADS, 1) gemm_prefill_kernel(
     // ------------------------------------------------------------------ MMA issuer
     const uint32_t idesc = idesc_i8(BW, bnt);
     const uint64_t x_desc0 = smem_desc_k128(smem_u32(sX));
-    int s = 0, ab = 0;
-    long long gg = 0;  // handoff groups so far
-    uint32_t abph = 0;
+    int s = 0, a = 0, ab = 0;
+    uint32_t sph = 0, aph = 0, abph = 0;
     bool ok = true, issued_any = false;
     for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
       bool got = true;
@@ -194,37 +189,29 @@ __global__ void __launch_bounds__(pf::THREADS, 1) gemm_prefill_kernel(
       if (!__shfl_sync(0xffffffffu, got, 0)) { ok = false; break; }
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(ab * MAX_BNT);
-      for (int kb0 = 0; kb0 < KB; kb0 += GST, ++gg) {
-        // a_full of the group implies its stages' TMA data landed (the unpack waited)
-        const int gs = static_cast<int>(gg % NGS);
-        if (lane == 0)
-          got = tc_wait(&bar->a_full[gs], static_cast<uint32_t>((gg / NGS) & 1), limit_ns,
-                        abort_flag);
+      for (int kb = 0; kb < KB; ++kb) {
+        // a_full of slot a implies the stage's TMA data landed (the unpack waited for it)
+        if (lane == 0) got = tc_wait(&bar->a_full[a], aph, limit_ns, abort_flag);
         if (!__shfl_sync(0xffffffffu, got, 0)) { ok = false; break; }
         tc_fence_after();
-        const int nst = min(GST, KB - kb0);
+        const uint32_t a_tmem = tmem_base + static_cast<uint32_t>(A_COL0 + a * A_COLS);
+        const uint64_t b_desc = x_desc0 + static_cast<uint64_t>(s * (X_BYTES >> 4));
 #pragma unroll
-        for (int j = 0; j < GST; ++j) {
-          if (j >= nst) break;
-          const int kb = kb0 + j;
-          const uint32_t a_tmem =
-              tmem_base + static_cast<uint32_t>(A_COL0 + (gs * GST + j) * A_COLS);
-          const uint64_t b_desc = x_desc0 + static_cast<uint64_t>(s * (X_BYTES >> 4));
-#pragma unroll
-          for (int kk = 0; kk < BK / MMA_K; ++kk)
-            mma_i8_ts_elect(d_tmem, a_tmem + static_cast<uint32_t>(kk * (MMA_K / 4)),
-                            b_desc + static_cast<uint64_t>(kk * (MMA_K >> 4)), idesc,
-                            (kb | kk) != 0 ? 1u : 0u);
-          mma_commit_elect(&bar->empty[s]);
-          if (++s == STAGES) s = 0;
-        }
+        for (int kk = 0; kk < BK / MMA_K; ++kk)
+          mma_i8_ts_elect(d_tmem, a_tmem + static_cast<uint32_t>(kk * (MMA_K / 4)),
+                          b_desc + static_cast<uint64_t>(kk * (MMA_K >> 4)), idesc,
+                          (kb | kk) != 0 ? 1u : 0u);
         issued_any = true;
-        mma_commit_elect(&bar->a_empty[gs]);
+        mma_commit_elect(&bar->empty[s]);
+        mma_commit_elect(&bar->a_empty[a]);
+        if (++s == STAGES) { s = 0; sph ^= 1u; }
+        if (++a == ASLOTS) { a = 0; aph ^= 1u; }
       }
       if (!ok) break;
       mma_commit_elect(&bar->tmem_full[ab]);
       if (++ab == 2) { ab = 0; abph ^= 1u; }
     }
+    (void)sph;
     if (!ok && issued_any) {
       mma_commit_elect(&bar->drain);  // completes once every MMA issued above has finished
       if (lane == 0) mbar_wait(&bar->drain, 0u, 100000000ull);
@@ -240,49 +227,40 @@ __global__ void __launch_bounds__(pf::THREADS, 1) gemm_prefill_kernel(
     // half first and lanes 4-7 their second, so the 8 rows of a 128-byte wavefront fall
     // in 8 distinct bank groups.
     const int h0 = (lane >> 2) & 1;
-    long long g = 0;   // stages of this CTA so far
-    long long gg = 0;  // handoff groups so far
+    long long g = 0;  // stages of this CTA so far
     bool ok = true;
     for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-      for (int kb0 = 0; kb0 < KB; kb0 += GST, ++gg) {
-        const int nst = min(GST, KB - kb0);
-        if (static_cast<int>(gg % UNPACK_SETS) != set) { g += nst; continue; }
-        const int gs = static_cast<int>(gg % NGS);
-        bool got = tc_wait(&bar->a_empty[gs], static_cast<uint32_t>(((gg / NGS) & 1) ^ 1),
-                           limit_ns, abort_flag);
-#pragma unroll
-        for (int j = 0; j < GST; ++j) {
-          if (j >= nst) break;
-          const long long gj = g + j;
-          const int s = static_cast<int>(gj % STAGES);
-          got = got && tc_wait(&bar->full[s], static_cast<uint32_t>((gj / STAGES) & 1),
-                               limit_ns, abort_flag);
-          if (!__all_sync(0xffffffffu, got)) break;
-          const uint4* src = reinterpret_cast<const uint4*>(sW + s * WP_BYTES + r * 32);
-          const uint4 first = src[h0], second = src[h0 ^ 1];
-          const uint4 halves[2] = {h0 ? second : first, h0 ? first : second};
-          uint32_t codes[32];  // the row's 128 codes of this K block, 4 per register
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const uint4 p = halves[h];
-            const uint32_t words[4] = {p.x, p.y, p.z, p.w};
-#pragma unroll
-            for (int mq = 0; mq < 4; ++mq) {
-              const int c = 16 * h + 4 * mq;  // column of trits 4c .. 4c + 15
-              codes[c + 0] = words[mq] & 0x03030303u;
-              codes[c + 1] = (words[mq] >> 2) & 0x03030303u;
-              codes[c + 2] = (words[mq] >> 4) & 0x03030303u;
-              codes[c + 3] = (words[mq] >> 6) & 0x03030303u;
-            }
-          }
-          tmem_st_x32(a_lane + static_cast<uint32_t>((gs * GST + j) * A_COLS), codes);
-        }
+      for (int kb = 0; kb < KB; ++kb, ++g) {
+        if (static_cast<int>(g % UNPACK_SETS) != set) continue;
+        const int s = static_cast<int>(g % STAGES);
+        const int a = static_cast<int>(g % ASLOTS);
+        const uint32_t ph = static_cast<uint32_t>((g / STAGES) & 1);
+        const uint32_t aph = static_cast<uint32_t>((g / ASLOTS) & 1);
+        const bool got = tc_wait(&bar->full[s], ph, limit_ns, abort_flag) &&
+                         tc_wait(&bar->a_empty[a], aph ^ 1u, limit_ns, abort_flag);
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+        const uint4* src = reinterpret_cast<const uint4*>(sW + s * WP_BYTES + r * 32);
+        const uint4 first = src[h0], second = src[h0 ^ 1];
+        const uint4 halves[2] = {h0 ? second : first, h0 ? first : second};
+        uint32_t codes[32];  // the row's 128 codes of this K block, 4 per register
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint4 p = halves[h];
+          const uint32_t words[4] = {p.x, p.y, p.z, p.w};
+#pragma unroll
+          for (int mq = 0; mq < 4; ++mq) {
+            const int c = 16 * h + 4 * mq;  // column of trits 4c .. 4c + 15
+            codes[c + 0] = words[mq] & 0x03030303u;
+            codes[c + 1] = (words[mq] >> 2) & 0x03030303u;
+            codes[c + 2] = (words[mq] >> 4) & 0x03030303u;
+            codes[c + 3] = (words[mq] >> 6) & 0x03030303u;
+          }
+        }
+        tmem_st_x32(a_lane + static_cast<uint32_t>(a * A_COLS), codes);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bar->a_full[gs]);
-        g += nst;
+        if (lane == 0) mbar_arrive(&bar->a_full[a]);
       }
     }
   } else {

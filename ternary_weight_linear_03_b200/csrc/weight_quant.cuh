@@ -265,7 +265,6 @@ __global__ void __launch_bounds__(kWqThreads) weight_quant_kernel(
   __shared__ unsigned long long sb[kWqBuckets];
   __shared__ unsigned long long col[kWqLimbs];
   __shared__ uint64_t full[kWqStages];
-  __shared__ uint64_t consumed[kWqStages];  // pass A: every warp is done with the slot
   __shared__ float s_T;
   __shared__ int s_ok;
   __shared__ float s_that;          // single-read mode: estimated threshold
@@ -290,10 +289,7 @@ __global__ void __launch_bounds__(kWqThreads) weight_quant_kernel(
   ring.nst = static_cast<int>((ring.bytes + kWqStageBytes - 1) / kWqStageBytes);
   if (tid == 0) {
     s_ok = 1;
-    for (int i = 0; i < kWqStages; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&consumed[i], kWqThreads / 32);
-    }
+    for (int i = 0; i < kWqStages; ++i) mbar_init(&full[i], 1);
     fence_mbar_init();
     for (int st = 0; st < min(ring.nst, kWqStages); ++st) wq_issue(ring, st, st);
   }
@@ -438,16 +434,8 @@ __global__ void __launch_bounds__(kWqThreads) weight_quant_kernel(
       }
     }
     if ((st & 15) == 15) wq_flush(acc0, acc1, base, sb);
-    // This warp is done with the slot. Only the thread that refills it waits for the other
-    // warps, so the rest run ahead into the stages already in flight instead of meeting
-    // at a block barrier every stage.
-    __syncwarp();
-    if ((tid & 31) == 0) mbar_arrive(&consumed[slot]);
-    if (tid == 0 && st + kWqStages < ring.nst) {
-      if (!mbar_wait(&consumed[slot], static_cast<uint32_t>((st / kWqStages) & 1), limit_ns))
-        s_ok = 0;
-      wq_issue(ring, st + kWqStages, st + kWqStages);
-    }
+    __syncthreads();  // every thread is done with this slot
+    if (tid == 0 && st + kWqStages < ring.nst) wq_issue(ring, st + kWqStages, st + kWqStages);
   }
   wq_flush(acc0, acc1, base, sb);
   if (nonfinite) record_status(kStatusNonfinite);
