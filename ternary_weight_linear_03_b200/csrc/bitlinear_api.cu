@@ -31,6 +31,7 @@ using bl::WqWorkspace;
 
 constexpr int kGemvMaxM = 4;            // M above this runs a tensor-core kernel
 constexpr int kSkinnyMaxM = 256;        // M above this runs the prefill GEMM
+static_assert(kSkinnyMaxM <= bl::sk::MAX_M, "the skinny kernel stages per-token factors for MAX_M tokens");
 constexpr int kGemvMaxSmem = 200 * 1024;  // xq rows held in shared memory by the GEMV
 constexpr unsigned long long kWaitLimitNs = 4000000000ull;  // 4 s per mbarrier wait
 constexpr int kMinKbPerSplit = 8;  // skinny split-K: K blocks per split, at least

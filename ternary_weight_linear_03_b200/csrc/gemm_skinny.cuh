@@ -23,21 +23,30 @@
 // adds, so the split does not change a single bit.
 //
 // The loop moves in groups of KG = 2 K blocks. Per group the four unpack warps write
-// their rows' codes to TMEM and meet the MMA warp at a hardware named barrier (bar.red of
-// 160 threads, far cheaper than an mbarrier arrive/poll round trip; the reduction also
-// makes every abort decision uniform, so no participant can be left waiting). The MMA
-// warp then issues the group's 8 MMAs and one commit while the unpack warps go on to the
-// next group; the commit's barrier (done ring) frees the A slot and the token tile. At
-// small M each MMA is a few tens of cycles of tensor work, so these per-group handoffs,
-// not bandwidth, set the pace, and the unpack warps are the critical path: every mbarrier
-// wait (a hundred to three hundred cycles on B200 even for a completed phase) is done by
-// the MMA warp, which has slack. Before the handoff of group g it makes sure that group
-// g + 1 may start (its W super-tile has landed, the MMAs that last read its A slot are
-// done), so the unpack warps never wait on an mbarrier.
+// their rows' codes to TMEM and meet the MMA and sentinel warps at a hardware named
+// barrier (bar.red of 192 threads, far cheaper than an mbarrier arrive/poll round trip;
+// the reduction also makes every abort decision uniform, so no participant can be left
+// waiting). The MMA warp then issues the group's 8 MMAs and one commit while the unpack
+// warps go on to the next group; the commit's barrier (done ring) frees the A slot and
+// the token tile.
 //
-// 6 warps: warps 0-3 unpack (thread t owns weight row t, TMEM lane t) and run the
+// At small M these per-group handoffs, not bandwidth, set the pace. Measured on B200 with
+// clock64 stamps (70B up projection, M = 16): issuing the 8 MMAs and the commit takes
+// about 400 cycles, unpacking a group about 430 (plus 50 for the stores to land), and
+// every mbarrier test 200 to 450 cycles even for a phase completed long before. So
+// neither the MMA warp nor the unpack warps test anything: a sentinel warp joins every
+// handoff, and each handoff also certifies what the next steps need. Before the handoff
+// of group g the sentinel has seen, with three lanes testing at once,
+//   lane 0: group g's token tile land (the MMAs of g read it),
+//   lane 1: group g + 1's W super-tile land, when g + 1 starts one,
+//   lane 2: the MMAs of group g + 1 - SU complete (the last readers of the A slot that
+//           group g + 1 is unpacked into),
+// while the unpack warps work on group g.
+//
+// 7 warps: warps 0-3 unpack (thread t owns weight row t, TMEM lane t) and run the
 // epilogue at the end; warp 4 issues the TMA loads; warp 5 owns the TMEM allocation and
-// issues the MMAs (whole-warp loop, one elected lane issues, operands precomputed).
+// issues the MMAs (whole-warp loop, one elected lane issues, operands precomputed);
+// warp 6 is the sentinel.
 #pragma once
 
 #include "common.cuh"
@@ -55,8 +64,9 @@ constexpr int WP_BYTES = BW * BK * KPS / 4;  // 16 KB packed super-tile
 constexpr int A_COLS = BK / 4;               // TMEM columns of one unpacked K block
 constexpr int G_COLS = KG * A_COLS;          // TMEM columns of one unpacked group
 constexpr int MAX_SU = 8;                    // unpacked groups in flight (TMEM slots), at most
-constexpr int THREADS = 192;
+constexpr int THREADS = 224;
 constexpr int MAX_SW = 4, MAX_SX = 16;
+constexpr int MAX_M = 256;  // tokens, at most
 
 static_assert(KPS % KG == 0, "groups tile a super-tile");
 // Ring of per-group completion barriers. Group g's MMAs arrive on done[g % SD]; the MMA
@@ -77,6 +87,8 @@ struct Barriers {
   uint32_t tmem_base;
   int abort;
   int last;
+  int rowsum[MAX_M];  // per token, staged once for the epilogue
+  float f[MAX_M];     // per token s_t * gamma
 };
 
 struct Plan {
@@ -172,8 +184,8 @@ __device__ __forceinline__ void epi_bar_sync() {  // the 4 unpack/epilogue warps
   asm volatile("bar.sync 1, 128;" ::: "memory");
 }
 // Named barriers that also return the OR of every participant's flag, so that all of them
-// take the same branch afterwards: id 1 = the 4 unpack/epilogue warps, id 2 = those and
-// the MMA warp (the per-group handoff).
+// take the same branch afterwards: id 1 = the 4 unpack/epilogue warps, id 2 = those, the
+// MMA warp and the sentinel warp (the per-group handoff).
 template <int ID, int COUNT>
 __device__ __forceinline__ bool bar_or(bool v) {
   uint32_t r;
@@ -188,19 +200,18 @@ __device__ __forceinline__ bool bar_or(bool v) {
   return r != 0;
 }
 __device__ __forceinline__ bool epi_bar_or(bool v) { return bar_or<1, 128>(v); }
-__device__ __forceinline__ bool group_bar_or(bool v) { return bar_or<2, 160>(v); }
+__device__ __forceinline__ bool group_bar_or(bool v) { return bar_or<2, 192>(v); }
 
 // Rescales one accumulator and stores it. OM: 0 fp32, 1 bf16, 2 int32 (acc only).
 // Returns the bit pattern of |stored value| (0 for int32 output), for the absmax of a
 // chain's next layer: non-negative floats order like their bits.
 template <int OM>
-__device__ __forceinline__ unsigned store_out(void* y, long long o, int a, float scale_t,
-                                              float gamma) {
+__device__ __forceinline__ unsigned store_out(void* y, long long o, int a, float f_t) {
   if (OM == 2) {
     static_cast<int*>(y)[o] = a;
     return 0u;
   } else {
-    const float val = __fmul_rn(__int2float_rn(a), __fmul_rn(scale_t, gamma));
+    const float val = __fmul_rn(__int2float_rn(a), f_t);
     if (OM == 0) {
       static_cast<float*>(y)[o] = val;
       return __float_as_uint(val) & 0x7fffffffu;
@@ -227,8 +238,10 @@ __device__ __forceinline__ void warp_amax_out(float* amax_out, int t, unsigned b
 // tile u / splits and the K blocks [split * kbps, min(KB, (split + 1) * kbps)), kbps a
 // multiple of KPS. A trailing partial group reads K blocks past KB, which the tensor maps
 // fill with zeros (their products vanish).
+// Two CTAs per SM for token tiles up to 64 (the 110 KB shared-memory plan): the bound keeps
+// the registers within 128 per thread, the most that 2 x 7 warps leave on one SM quarter.
 template <int OM>
-__global__ void __launch_bounds__(sk::THREADS, 1) gemm_skinny_kernel(
+__global__ void __launch_bounds__(sk::THREADS, 2) gemm_skinny_kernel(
     const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w,
     const int* __restrict__ rowsum, const float* __restrict__ scale,
     const float* __restrict__ gamma_ptr, void* __restrict__ y, int* __restrict__ partial,
@@ -283,13 +296,13 @@ __global__ void __launch_bounds__(sk::THREADS, 1) gemm_skinny_kernel(
 
   if (warp == 4) {
     // ------------------------------------------------------------------ TMA producer
+    bool ok = true;  // lane 0's verdict on its loads
     if (lane == 0) {
       prefetch_tmap(&map_x);
       prefetch_tmap(&map_w);
       int sw = 0, sx = 0;
       uint32_t wph = 0;
       long long w_issued = 0, x_issued = 0;
-      bool ok = true;
       // The first W super-tiles fill the empty ring before the wait for the kernel that
       // produced the token tiles (programmatic dependent launch): W does not depend on it.
       const int nst = (kb1 - kb0 + KPS - 1) / KPS;
@@ -323,13 +336,7 @@ __global__ void __launch_bounds__(sk::THREADS, 1) gemm_skinny_kernel(
         ++x_issued;
         if (++sx == pl.sx) sx = 0;
       }
-      if (ok) {
-        // The last commits' arrivals land on done[] asynchronously: see each barrier's final
-        // phase before the CTA can exit, so no arrival reaches a later CTA's shared memory.
-        for (int i = max(0, ng - SD); i < ng; ++i)
-          if (!tc_wait(&bar->done[i & (SD - 1)], static_cast<uint32_t>((i / SD) & 1), limit_ns,
-                       abort_flag)) break;
-      } else {  // wait (bounded) for the copies still in flight
+      if (!ok) {  // wait (bounded) for the copies still in flight
         for (long long i = w_issued - 1; i >= 0 && i > w_issued - 1 - pl.sw; --i)
           mbar_wait(&bar->w_full[i % pl.sw], static_cast<uint32_t>((i / pl.sw) & 1),
                     100000000ull);
@@ -338,6 +345,16 @@ __global__ void __launch_bounds__(sk::THREADS, 1) gemm_skinny_kernel(
                     100000000ull);
       }
     }
+    // The last commits' arrivals land on done[] asynchronously: see each barrier's final
+    // phase before the CTA can exit, so no arrival reaches a later CTA's shared memory.
+    // One barrier per lane (a test costs a few hundred cycles; in series they would
+    // outlast the epilogue).
+    if (__shfl_sync(0xffffffffu, ok, 0)) {
+      const int i = ng - 1 - lane;
+      if (lane < SD && i >= 0)
+        tc_wait(&bar->done[i & (SD - 1)], static_cast<uint32_t>((i / SD) & 1), limit_ns, abort_flag);
+    }
+    __syncwarp();
   } else if (warp == 5) {
     // ------------------------------------------------------------------ MMA issuer
     const uint32_t idesc = idesc_i8(BW, bnt);
@@ -345,72 +362,76 @@ __global__ void __launch_bounds__(sk::THREADS, 1) gemm_skinny_kernel(
     const uint64_t x_desc0 = smem_desc_k128(smem_u32(sX));
     const uint32_t a_tmem0 = tmem_base + a_col0;
     int su = 0, sx = 0, sw = 0;
-    uint32_t xph = 0;
-    bool failed = false;  // a wait gave up (the abort flag is set)
-    // Waits (all lanes) until group gn may be unpacked: its W super-tile has landed and the
-    // MMAs of group gn - SU, the last readers of its A slot, are done.
-    auto prepare = [&](int gn) -> bool {
-      bool ok = true;
-      if (((gn * KG) & (KPS - 1)) == 0) {
-        const int st = (gn * KG) / KPS;  // super-tiles before this one
-        ok = tc_wait(&bar->w_full[st % pl.sw], static_cast<uint32_t>((st / pl.sw) & 1),
-                     limit_ns, abort_flag);
-      }
-      if (gn >= SU) {
-        const int i = gn - SU;
-        ok = ok && tc_wait(&bar->done[i & (SD - 1)], static_cast<uint32_t>((i / SD) & 1),
-                           limit_ns, abort_flag);
-      }
-      return __all_sync(0xffffffffu, ok);
-    };
-    bool stop = group_bar_or(ng > 0 && !prepare(0));  // group 0 may start
+    bool stop = group_bar_or(false);  // the sentinel has seen group 0's W land
     int g = 0;
     for (; !stop && g < ng; ++g) {
-      const bool next_ok = (g + 1 < ng) ? prepare(g + 1) : true;
       tc_fence_before();
-      if (group_bar_or(!next_ok || *abort_flag != 0)) break;  // group g's rows are in TMEM
+      // group g's rows are in TMEM, its token tile has landed, its W reads are over
+      if (group_bar_or(false)) break;
+      tc_fence_after();
       const int q0 = (g * KG) & (KPS - 1);
       const bool last_of_tile = (q0 + KG == KPS) || (g == ng - 1);
-      bool xok = true;
-      if (lane == 0) {
-        xok = tc_wait(&bar->x_full[sx], xph, limit_ns, abort_flag);
-        if (last_of_tile) mbar_arrive(&bar->w_empty[sw]);  // every row has read this super-tile
-      }
-      xok = __shfl_sync(0xffffffffu, xok, 0);
-      __syncwarp();
-      if (xok) {
-        tc_fence_after();
-        const uint32_t a_tmem = a_tmem0 + static_cast<uint32_t>(su * G_COLS);
-        const uint64_t b_desc = x_desc0 + static_cast<uint64_t>(sx * (XG >> 4));
+      if (lane == 0 && last_of_tile) mbar_arrive(&bar->w_empty[sw]);  // every row has read it
+      const uint32_t a_tmem = a_tmem0 + static_cast<uint32_t>(su * G_COLS);
+      const uint64_t b_desc = x_desc0 + static_cast<uint64_t>(sx * (XG >> 4));
 #pragma unroll
-        for (int kq = 0; kq < KG; ++kq)
+      for (int kq = 0; kq < KG; ++kq)
 #pragma unroll
-          for (int kk = 0; kk < BK / MMA_K; ++kk)
-            mma_i8_ts_elect(tmem_base,
-                            a_tmem + static_cast<uint32_t>(kq * A_COLS + kk * (MMA_K / 4)),
-                            b_desc + static_cast<uint64_t>(kq * (XB >> 4) + kk * (MMA_K >> 4)),
-                            idesc, (g | kq | kk) != 0 ? 1u : 0u);
-        mma_commit_elect(&bar->done[g & (SD - 1)]);
-      } else {
-        // stay in step with the unpack warps: the next handoff sees the abort flag and
-        // every participant leaves the loop there
-        failed = true;
-      }
+        for (int kk = 0; kk < BK / MMA_K; ++kk)
+          mma_i8_ts_elect(tmem_base,
+                          a_tmem + static_cast<uint32_t>(kq * A_COLS + kk * (MMA_K / 4)),
+                          b_desc + static_cast<uint64_t>(kq * (XB >> 4) + kk * (MMA_K >> 4)),
+                          idesc, (g | kq | kk) != 0 ? 1u : 0u);
+      mma_commit_elect(&bar->done[g & (SD - 1)]);
       if (++su == SU) su = 0;
-      if (++sx == pl.sx) { sx = 0; xph ^= 1u; }
+      if (++sx == pl.sx) sx = 0;
       if (last_of_tile && ++sw == pl.sw) sw = 0;
     }
-    if (g == ng && !failed) {
+    if (g == ng) {
       mma_commit_elect(&bar->acc_full);
     } else if (g > 0) {
       mma_commit_elect(&bar->drain);  // completes once every MMA issued above has finished
       if (lane == 0) mbar_wait(&bar->drain, 0u, 100000000ull);
       __syncwarp();
     }
+  } else if (warp == 6) {
+    // ------------------------------------------------------------------ sentinel
+    // Lane i tests barrier b_i for phase p_i (lanes without one pass); the warp's verdict
+    // is the AND over its lanes.
+    auto test_lanes = [&](uint64_t* b, uint32_t parity, bool active) -> bool {
+      bool ok = true;
+      if (active) ok = tc_wait(b, parity, limit_ns, abort_flag);
+      return __all_sync(0xffffffffu, ok);
+    };
+    int sx = 0;
+    uint32_t xph = 0;
+    bool stop = group_bar_or(ng > 0 && !test_lanes(&bar->w_full[0], 0u, lane == 0));
+    int g = 0;
+    for (; !stop && g < ng; ++g) {
+      const int gn = g + 1;
+      uint64_t* b = &bar->x_full[sx];
+      uint32_t parity = xph;
+      bool active = (lane == 0);
+      if (lane == 1 && gn < ng && ((gn * KG) & (KPS - 1)) == 0) {
+        const int st = (gn * KG) / KPS;  // super-tiles before group gn's
+        b = &bar->w_full[st % pl.sw];
+        parity = static_cast<uint32_t>((st / pl.sw) & 1);
+        active = true;
+      }
+      if (lane == 2 && gn < ng && gn >= SU) {
+        const int i = gn - SU;
+        b = &bar->done[i & (SD - 1)];
+        parity = static_cast<uint32_t>((i / SD) & 1);
+        active = true;
+      }
+      const bool ok = test_lanes(b, parity, active);
+      if (group_bar_or(!ok)) break;  // the handoff of group g
+      if (++sx == pl.sx) { sx = 0; xph ^= 1u; }
+    }
   } else {
     // ------------------------------------------------------------------ warps 0-3
-    // No mbarrier waits here: passing the handoff before group g means the MMA warp has
-    // seen group g's W super-tile land and its A slot freed.
+    // Passing the handoff before group g means group g's W super-tile has landed and its
+    // A slot is free (tested by the sentinel before the previous handoff).
     const int r = threadIdx.x;  // weight row of the tile owned by this thread (0..127)
     const int rs = r & 7;       // its 128-byte swizzle phase
     const uint32_t a_lane = tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + a_col0;
@@ -421,15 +442,20 @@ __global__ void __launch_bounds__(sk::THREADS, 1) gemm_skinny_kernel(
       const int q0 = (g * KG) & (KPS - 1);  // first K block of the group in its super-tile
       tc_fence_after();
       const unsigned char* src = sWp + sw * WP_BYTES + r * 128;
+      // The group's packed chunks (logical 16-byte chunk 2q+h of the row = K block q,
+      // words 4h .. 4h+3), all loaded before any is unpacked.
+      uint4 pk[KG][2];
+#pragma unroll
+      for (int kq = 0; kq < KG; ++kq)
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          pk[kq][h] = *reinterpret_cast<const uint4*>(src + (((2 * (q0 + kq) + h) ^ rs) << 4));
 #pragma unroll
       for (int kq = 0; kq < KG; ++kq) {
-        const int q = q0 + kq;
-        uint32_t a[32];  // the row's 128 unpacked codes of K block q, 4 per register
+        uint32_t a[32];  // the row's 128 unpacked codes of K block q0 + kq, 4 per register
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          // logical 16-byte chunk 2q+h of the packed row = K block q, words 4h .. 4h+3
-          const uint4 p = *reinterpret_cast<const uint4*>(src + (((2 * q + h) ^ rs) << 4));
-          const uint32_t words[4] = {p.x, p.y, p.z, p.w};
+          const uint32_t words[4] = {pk[kq][h].x, pk[kq][h].y, pk[kq][h].z, pk[kq][h].w};
 #pragma unroll
           for (int mq = 0; mq < 4; ++mq) {
             const uint32_t w = words[mq];
@@ -454,10 +480,19 @@ __global__ void __launch_bounds__(sk::THREADS, 1) gemm_skinny_kernel(
     grid_dependency_wait();  // rowsum, scale and the zeroed split-K sums come from it
     const bool got = ok && tc_wait(&bar->acc_full, 0u, limit_ns, abort_flag);
     if (!epi_bar_or(!got)) {  // the same decision in all four warps
+      // Per-token rowsum and s_t * gamma, staged once: read in the store loops below, global
+      // loads would wait behind the stores (up to one memory round trip per token).
+      {
+        const float gamma = (OM == 2) ? 0.0f : *gamma_ptr;
+        for (int t = threadIdx.x; t < M; t += 128) {
+          bar->rowsum[t] = rowsum[t];
+          bar->f[t] = (OM == 2) ? 0.0f : __fmul_rn(scale[t], gamma);
+        }
+      }
+      epi_bar_sync();
       tc_fence_after();
       const int n = n0 + warp * 32 + lane;  // this thread's TMEM lane = weight row
       const bool nvalid = n < N;
-      const float gamma = (OM == 2) ? 0.0f : *gamma_ptr;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
       if (splits == 1) {
         for (int c0 = 0; c0 < bnt; c0 += 16) {
@@ -469,8 +504,7 @@ __global__ void __launch_bounds__(sk::THREADS, 1) gemm_skinny_kernel(
             unsigned mag = 0u;
             if (t < M && nvalid)
               mag = store_out<OM>(y, static_cast<long long>(t) * N + n,
-                                  static_cast<int>(v[j]) - rowsum[t],
-                                  OM == 2 ? 0.0f : scale[t], gamma);
+                                  static_cast<int>(v[j]) - bar->rowsum[t], bar->f[t]);
             if (amax_out != nullptr && t < M) warp_amax_out(amax_out, t, mag);
           }
         }
@@ -497,20 +531,22 @@ __global__ void __launch_bounds__(sk::THREADS, 1) gemm_skinny_kernel(
           __threadfence();
           for (int t0 = 0; t0 < M; t0 += 16) {
             int a[16];
+            // all 16 loads first (a store between them would order each behind the last)
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              int* pp = partial + static_cast<long long>(t0 + j) * N + n;
-              a[j] = (t0 + j < M && nvalid) ? __ldcg(pp) : 0;
-              // leave the sums zeroed for the next launch that shares them (layer chains)
-              if (t0 + j < M && nvalid) __stcg(pp, 0);
-            }
+            for (int j = 0; j < 16; ++j)
+              a[j] = (t0 + j < M && nvalid) ? __ldcg(partial + static_cast<long long>(t0 + j) * N + n)
+                                            : 0;
+            // leave the sums zeroed for the next launch that shares them (layer chains)
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              if (t0 + j < M && nvalid) __stcg(partial + static_cast<long long>(t0 + j) * N + n, 0);
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
               const int t = t0 + j;
               unsigned mag = 0u;
               if (t < M && nvalid)
-                mag = store_out<OM>(y, static_cast<long long>(t) * N + n, a[j] - rowsum[t],
-                                    OM == 2 ? 0.0f : scale[t], gamma);
+                mag = store_out<OM>(y, static_cast<long long>(t) * N + n, a[j] - bar->rowsum[t],
+                                    bar->f[t]);
               if (amax_out != nullptr && t < M) warp_amax_out(amax_out, t, mag);
             }
           }
