@@ -49,6 +49,8 @@
 // warp 6 is the sentinel.
 #pragma once
 
+#include <cstddef>
+
 #include "common.cuh"
 #include "gemm_tc.cuh"
 
@@ -90,6 +92,11 @@ struct Barriers {
   int rowsum[MAX_M];  // per token, staged once for the epilogue
   float f[MAX_M];     // per token s_t * gamma
 };
+
+// The mbarriers above, w_full through drain, are consecutive 8-byte words.
+constexpr int kNumMbar = 2 * MAX_SW + MAX_SX + SD + 2;
+static_assert(offsetof(Barriers, drain) - offsetof(Barriers, w_full) == (kNumMbar - 1) * 8,
+              "mbarriers are contiguous");
 
 struct Plan {
   int sw, sx;
@@ -202,26 +209,6 @@ __device__ __forceinline__ bool bar_or(bool v) {
 __device__ __forceinline__ bool epi_bar_or(bool v) { return bar_or<1, 128>(v); }
 __device__ __forceinline__ bool group_bar_or(bool v) { return bar_or<2, 192>(v); }
 
-// Rescales one accumulator and stores it. OM: 0 fp32, 1 bf16, 2 int32 (acc only).
-// Returns the bit pattern of |stored value| (0 for int32 output), for the absmax of a
-// chain's next layer: non-negative floats order like their bits.
-template <int OM>
-__device__ __forceinline__ unsigned store_out(void* y, long long o, int a, float f_t) {
-  if (OM == 2) {
-    static_cast<int*>(y)[o] = a;
-    return 0u;
-  } else {
-    const float val = __fmul_rn(__int2float_rn(a), f_t);
-    if (OM == 0) {
-      static_cast<float*>(y)[o] = val;
-      return __float_as_uint(val) & 0x7fffffffu;
-    }
-    const __nv_bfloat16 h = __float2bfloat16_rn(val);
-    static_cast<__nv_bfloat16*>(y)[o] = h;
-    return __float_as_uint(__bfloat162float(h)) & 0x7fffffffu;
-  }
-}
-
 // Atomic max of a non-negative float given by its bits (fire and forget).
 __device__ __forceinline__ void red_max_u32(float* p, unsigned bits) {
   asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" ::"l"(p), "r"(bits) : "memory");
@@ -232,6 +219,60 @@ __device__ __forceinline__ void red_max_u32(float* p, unsigned bits) {
 __device__ __forceinline__ void warp_amax_out(float* amax_out, int t, unsigned bits) {
   const unsigned m = __reduce_max_sync(0xffffffffu, bits);
   if ((threadIdx.x & 31) == 0 && m != 0u) red_max_u32(amax_out + t, m);
+}
+
+// Rescales and writes the 16 values of tokens c0 .. c0 + 15 of this thread's weight row
+// (a[j] = accumulator - rowsum) to y. With vec (rows of y 16-byte aligned: N a multiple of
+// 16 / element size) they go through a 16 x 128 tile in shared memory and leave as 16-byte
+// row pieces, else one store per value. Called by all 128 epilogue threads.
+template <int OM>
+__device__ __forceinline__ void epi_store_chunk(const int (&a)[16], const float (&fs)[16], int c0,
+                                                int M, int N, int n0, bool nvalid, bool vec,
+                                                unsigned char* stage, void* y, float* amax_out) {
+  constexpr int ES = (OM == 1) ? 2 : 4;  // bytes per element of y
+  const int nl = threadIdx.x;            // row within the tile
+  const int n = n0 + nl;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const int t = c0 + j;
+    uint32_t bits;
+    unsigned mag = 0u;
+    if (OM == 2) {
+      bits = static_cast<uint32_t>(a[j]);
+    } else {
+      const float val = __fmul_rn(__int2float_rn(a[j]), fs[j]);
+      if (OM == 0) {
+        bits = __float_as_uint(val);
+        mag = bits & 0x7fffffffu;
+      } else {
+        const __nv_bfloat16 h = __float2bfloat16_rn(val);
+        bits = static_cast<uint32_t>(__bfloat16_as_ushort(h));
+        mag = (bits << 16) & 0x7fffffffu;
+      }
+    }
+    if (vec) {
+      if (ES == 2) reinterpret_cast<uint16_t*>(stage)[j * 128 + nl] = static_cast<uint16_t>(bits);
+      else reinterpret_cast<uint32_t*>(stage)[j * 128 + nl] = bits;
+    } else if (t < M && nvalid) {
+      const long long o = static_cast<long long>(t) * N + n;
+      if (ES == 2) static_cast<uint16_t*>(y)[o] = static_cast<uint16_t>(bits);
+      else static_cast<uint32_t*>(y)[o] = bits;
+    }
+    if (OM != 2 && amax_out != nullptr && t < M) warp_amax_out(amax_out, t, nvalid ? mag : 0u);
+  }
+  if (vec) {
+    epi_bar_sync();
+    constexpr int PPR = 128 * ES / 16;  // 16-byte pieces per tile row
+    for (int p = threadIdx.x; p < 16 * PPR; p += 128) {
+      const int j = p / PPR, q = p % PPR;
+      const int t = c0 + j, col = n0 + q * (16 / ES);
+      if (t < M && col < N)
+        *reinterpret_cast<uint4*>(static_cast<unsigned char*>(y) +
+                                  (static_cast<long long>(t) * N + col) * ES) =
+            *reinterpret_cast<const uint4*>(stage + (j * 128 + q * (16 / ES)) * ES);
+    }
+    epi_bar_sync();  // the tile is rewritten by the next chunk
+  }
 }
 
 // bnt = token tile (multiple of 16, >= M). grid = n_tiles * splits; CTA u handles weight
@@ -272,18 +313,29 @@ __global__ void __launch_bounds__(sk::THREADS, 2) gemm_skinny_kernel(
   const uint32_t a_col0 = acc_cols(bnt);  // first TMEM column of the unpacked A slots
   const int SU = n_slots(bnt);
 
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < pl.sw; ++i) {
-      mbar_init(&bar->w_full[i], 1);
-      mbar_init(&bar->w_empty[i], 1);
+  // The first W super-tiles (at most the ring) do not depend on the kernel before, nor on
+  // the TMEM allocation: the producer warp initialises the mbarriers (every one has one
+  // arrival per phase; a lane each) and issues those loads before the block-wide sync.
+  const int pre = min(pl.sw, (kb1 - kb0 + KPS - 1) / KPS);
+  if (warp == 4) {
+    if (lane == 0) {
+      prefetch_tmap(&map_x);
+      prefetch_tmap(&map_w);
     }
-    for (int i = 0; i < pl.sx; ++i) mbar_init(&bar->x_full[i], 1);
-    for (int i = 0; i < SD; ++i) mbar_init(&bar->done[i], 1);
-    mbar_init(&bar->acc_full, 1);
-    mbar_init(&bar->drain, 1);
-    bar->abort = 0;
-    bar->last = 0;
+    uint64_t* first = &bar->w_full[0];
+    for (int i = lane; i < kNumMbar; i += 32) mbar_init(first + i, 1);
+    if (lane == 0) {
+      bar->abort = 0;
+      bar->last = 0;
+    }
     fence_mbar_init();
+    __syncwarp();
+    if (lane == 0) {
+      for (int i = 0; i < pre; ++i) {
+        mbar_arrive_expect_tx(&bar->w_full[i], WP_BYTES);
+        tma_load_2d(sWp + i * WP_BYTES, &map_w, (kb0 + i * KPS) * (BK / 4), n0, &bar->w_full[i]);
+      }
+    }
   }
   if (warp == 5) {
     tmem_alloc(&bar->tmem_base, ncols);
@@ -298,21 +350,10 @@ __global__ void __launch_bounds__(sk::THREADS, 2) gemm_skinny_kernel(
     // ------------------------------------------------------------------ TMA producer
     bool ok = true;  // lane 0's verdict on its loads
     if (lane == 0) {
-      prefetch_tmap(&map_x);
-      prefetch_tmap(&map_w);
       int sw = 0, sx = 0;
       uint32_t wph = 0;
-      long long w_issued = 0, x_issued = 0;
-      // The first W super-tiles fill the empty ring before the wait for the kernel that
-      // produced the token tiles (programmatic dependent launch): W does not depend on it.
-      const int nst = (kb1 - kb0 + KPS - 1) / KPS;
-      const int pre = min(pl.sw, nst);
-      for (int i = 0; i < pre; ++i) {
-        mbar_arrive_expect_tx(&bar->w_full[i], WP_BYTES);
-        tma_load_2d(sWp + i * WP_BYTES, &map_w, (kb0 + i * KPS) * (BK / 4), n0, &bar->w_full[i]);
-      }
-      w_issued = pre;
-      grid_dependency_wait();
+      long long w_issued = pre, x_issued = 0;  // the first W loads went out before the sync
+      grid_dependency_wait();  // the token tiles come from the kernel before
       for (int g = 0; g < ng; ++g) {
         const int kb = kb0 + g * KG;
         if (((g * KG) & (KPS - 1)) == 0) {
@@ -493,20 +534,27 @@ __global__ void __launch_bounds__(sk::THREADS, 2) gemm_skinny_kernel(
       tc_fence_after();
       const int n = n0 + warp * 32 + lane;  // this thread's TMEM lane = weight row
       const bool nvalid = n < N;
+      // output tiles leave through the token ring, free once the last MMA is done
+      const bool vec = (N % (OM == 1 ? 8 : 4)) == 0;
+      unsigned char* stage = sX;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
       if (splits == 1) {
         for (int c0 = 0; c0 < bnt; c0 += 16) {
           uint32_t v[16];
           ld_acc16(taddr + c0, v);
+          // the chunk's factors into registers first: a shared-memory read after a global
+          // store would wait for it (the compiler cannot tell the two apart)
+          int rs[16];
+          float fs[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            const int t = c0 + j;
-            unsigned mag = 0u;
-            if (t < M && nvalid)
-              mag = store_out<OM>(y, static_cast<long long>(t) * N + n,
-                                  static_cast<int>(v[j]) - bar->rowsum[t], bar->f[t]);
-            if (amax_out != nullptr && t < M) warp_amax_out(amax_out, t, mag);
+            rs[j] = bar->rowsum[c0 + j];
+            fs[j] = bar->f[c0 + j];
           }
+          int a[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) a[j] = static_cast<int>(v[j]) - rs[j];
+          epi_store_chunk<OM>(a, fs, c0, M, N, n0, nvalid, vec, stage, y, amax_out);
         }
       } else {
         // exact int32 partial of this split, added into acc32[t][n] (zeroed by the host)
@@ -540,15 +588,16 @@ __global__ void __launch_bounds__(sk::THREADS, 2) gemm_skinny_kernel(
 #pragma unroll
             for (int j = 0; j < 16; ++j)
               if (t0 + j < M && nvalid) __stcg(partial + static_cast<long long>(t0 + j) * N + n, 0);
+            int rs[16];
+            float fs[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-              const int t = t0 + j;
-              unsigned mag = 0u;
-              if (t < M && nvalid)
-                mag = store_out<OM>(y, static_cast<long long>(t) * N + n, a[j] - bar->rowsum[t],
-                                    bar->f[t]);
-              if (amax_out != nullptr && t < M) warp_amax_out(amax_out, t, mag);
+              rs[j] = bar->rowsum[t0 + j];
+              fs[j] = bar->f[t0 + j];
             }
+#pragma unroll
+            for (int j = 0; j < 16; ++j) a[j] -= rs[j];
+            epi_store_chunk<OM>(a, fs, t0, M, N, n0, nvalid, vec, stage, y, amax_out);
           }
           if (threadIdx.x == 0) counters[tile] = 0u;  // every split has arrived
         }

@@ -118,6 +118,47 @@ __device__ __forceinline__ void load16(const void* x, long long off, float (&v)[
   }
 }
 
+// Per-halfword unsigned maximum.
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// Largest |x| of 16 bf16 values (two 16-byte vectors at p), kept as two halfword bit
+// patterns: with the sign cleared, bf16 patterns order like their values, and the NaN
+// patterns lie above infinity (0x7f80), so a maximum at or above 0x7f80 flags a
+// non-finite value.
+__device__ __forceinline__ uint32_t absmax16_bf16(const void* p, uint32_t m2) {
+  const uint4 a = reinterpret_cast<const uint4*>(p)[0], b = reinterpret_cast<const uint4*>(p)[1];
+  const uint32_t h[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+  for (int q = 0; q < 8; ++q) m2 = max_u16x2(m2, h[q] & 0x7fff7fffu);
+  return m2;
+}
+
+// Quantizes 16 bf16 values with a finite r (the same rounding and clamping as quant_i8;
+// its zero test only matters for an infinite r) into four words of int8, byte i & 3 of
+// word i >> 2 holding element i, and adds their sum into *sum.
+__device__ __forceinline__ uint4 quant16_bf16(const void* p, float r, int* sum) {
+  const uint4 a = reinterpret_cast<const uint4*>(p)[0], b = reinterpret_cast<const uint4*>(p)[1];
+  const uint32_t h[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+  uint32_t w[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    int q[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t hw = h[2 * j + (e >> 1)];
+      const float v = __uint_as_float((e & 1) ? (hw & 0xffff0000u) : (hw << 16));
+      q[e] = max(-127, min(127, __float2int_rn(__fmul_rn(v, r))));
+    }
+    w[j] = __byte_perm(__byte_perm(q[0], q[1], 0x0040), __byte_perm(q[2], q[3], 0x0040), 0x5410);
+    *sum = __dp4a(static_cast<int>(w[j]), 0x01010101, *sum);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
 // XR: activations in registers (one token). R: rows a warp sums at once on the shared-
 // memory path (2 lets every activation load feed two rows; worth it only with many rows).
 // Layer chains (optional, null when unused): amax_in[t] is the absmax of token t's row of
@@ -192,19 +233,42 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(
     bool bad = false;
 #pragma unroll
     for (int t = 0; t < MT; ++t) amax[t] = 0.0f;
-    if (amax_in == nullptr) {
+    // The float form of the max pass (fp32 x, or a bf16 thread that saw a non-finite value:
+    // NaN is skipped by fmaxf and flagged).
+    auto amax_pass = [&](int t) {
+      float a = 0.0f;
       for (int kb = tid; kb < KB; kb += kGemvThreads) {
+        float v[16];
+        load16<XM>(x, static_cast<long long>(t) * K + 16 * kb, v);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float m = abs_bits(v[i]);
+          bad |= !(m <= 3.4028234663852886e38f);
+          a = fmaxf(a, m);
+        }
+      }
+      return a;
+    };
+    if (amax_in == nullptr) {
+      if (XM == kXbf16) {
+        // one max.u16x2 per two values on the sign-cleared bit patterns
+        uint32_t m2[MT];
+#pragma unroll
+        for (int t = 0; t < MT; ++t) m2[t] = 0u;
+        for (int kb = tid; kb < KB; kb += kGemvThreads) {
+#pragma unroll
+          for (int t = 0; t < MT; ++t)
+            m2[t] = absmax16_bf16(static_cast<const uint16_t*>(x) + static_cast<long long>(t) * K + 16 * kb,
+                                  m2[t]);
+        }
 #pragma unroll
         for (int t = 0; t < MT; ++t) {
-          float v[16];
-          load16<XM>(x, static_cast<long long>(t) * K + 16 * kb, v);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float m = abs_bits(v[i]);
-            bad |= !(m <= 3.4028234663852886e38f);
-            amax[t] = fmaxf(amax[t], m);
-          }
+          const uint32_t m = max(m2[t] & 0xffffu, m2[t] >> 16);
+          amax[t] = (m < 0x7f80u) ? __uint_as_float(m << 16) : amax_pass(t);
         }
+      } else {
+#pragma unroll
+        for (int t = 0; t < MT; ++t) amax[t] = amax_pass(t);
       }
     } else if (tid == 0) {
 #pragma unroll
@@ -234,16 +298,23 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(
       const int unit = (kb & 3) * CPR + (kb >> 2);
 #pragma unroll
       for (int t = 0; t < MT; ++t) {
-        float v[16];
-        load16<XM>(x, static_cast<long long>(t) * K + 16 * kb, v);
-        uint32_t w4[4] = {0u, 0u, 0u, 0u};
+        uint4 q4;
+        if (XM == kXbf16 && r[t] <= 3.4028234663852886e38f) {  // finite r (0 when amax is 0)
+          q4 = quant16_bf16(static_cast<const uint16_t*>(x) + static_cast<long long>(t) * K + 16 * kb,
+                            r[t], &sum[t]);
+        } else {
+          float v[16];
+          load16<XM>(x, static_cast<long long>(t) * K + 16 * kb, v);
+          uint32_t w4[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int q = (amax[t] > 0.0f) ? quant_i8(v[i], r[t]) : 0;
-          sum[t] += q;
-          w4[i >> 2] |= (static_cast<uint32_t>(q) & 0xffu) << (8 * (i & 3));
+          for (int i = 0; i < 16; ++i) {
+            const int q = (amax[t] > 0.0f) ? quant_i8(v[i], r[t]) : 0;
+            sum[t] += q;
+            w4[i >> 2] |= (static_cast<uint32_t>(q) & 0xffu) << (8 * (i & 3));
+          }
+          q4 = make_uint4(w4[0], w4[1], w4[2], w4[3]);
         }
-        reinterpret_cast<uint4*>(xs_raw + t * K)[unit] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        reinterpret_cast<uint4*>(xs_raw + t * K)[unit] = q4;
       }
     }
 #pragma unroll

@@ -198,6 +198,7 @@ CONTRACT_SHAPES = [
     (1, 256, 256), (2, 293, 192), (3, 1000, 1536), (4, 777, 64),       # CUDA-core path
     (1, 4099, 8192), (1, 3001, 2048),            # one token, activations in registers
     (1, 5000, 28672), (2, 4800, 2048), (4, 4737, 4096),  # large K: two rows per warp
+    (1, 3001, 16384), (1, 600, 57344), (1, 200, 131072),  # one token, long rows
     (5, 300, 640), (16, 4096, 1536), (130, 293, 8640), (300, 520, 1536),  # tensor-core path
     (129, 257, 128), (64, 64, 64), (256, 1000, 3200), (257, 300, 640), (17, 8640, 3200),
     (48, 129, 8640), (176, 520, 8192),
@@ -240,6 +241,44 @@ def test_forward_matches_oracle(M, N, K, x_dtype, out):
         got = y.cpu().view(torch.int16).numpy().view(np.uint16)
         assert_bf16_within_1ulp(got, ref)
         np.testing.assert_array_equal(got, ref)
+
+
+def _edge_row(kind: str, K: int, seed: int) -> torch.Tensor:
+    g = torch.Generator().manual_seed(seed)
+    v = torch.randn(K, generator=g)
+    if kind == "tiny":          # absmax ~4e-38: 127 / absmax overflows fp32 to +inf
+        v = v * 1e-38
+    elif kind == "zeros":
+        v = torch.zeros(K)
+    elif kind == "onehot":
+        v = torch.zeros(K)
+        v[K // 3] = -2.75
+    elif kind == "subnormal_mix":  # bf16 subnormals next to a few ordinary values
+        v = v * 1e-39
+        v[::997] = torch.randn(len(v[::997]), generator=g)
+    return v.bfloat16()
+
+
+@pytest.mark.parametrize("K", [1536, 8192, 28672])
+@pytest.mark.parametrize("kinds", [("normal",), ("tiny",), ("zeros",), ("onehot",),
+                                   ("subnormal_mix",), ("tiny", "normal"), ("zeros", "onehot")])
+def test_gemv_prologue_edge_rows(K, kinds):
+    """bf16 tokens through the CUDA-core path (one or two tokens, activations in registers
+    or in shared memory): ordinary rows, rows whose 127 / absmax overflows (every nonzero
+    value quantizes to +-127), all-zero, one-hot and subnormal rows, bit for bit."""
+    N = {1536: 4096, 8192: 2048, 28672: 4800}[K]  # registers, registers, two rows per warp
+    W = syn.weights(N, K, 0.02, seed=K + 5)
+    x = torch.stack([_edge_row(k, K, 31 * i + K) for i, k in enumerate(kinds)]).contiguous()
+    packed, gamma = bl.quantize_weights(W.cuda())
+    path, _ = bl.debug_plan(x.shape[0], N, K)
+    assert path == "gemv"
+    for out in ("f32", "bf16"):
+        y = bl.forward(x.cuda(), packed, gamma,
+                       out_dtype=torch.float32 if out == "f32" else torch.bfloat16)
+        ref = orc.forward(_np_in(x), packed.cpu().numpy(), gamma.item(), out=out)
+        got = y.cpu().numpy() if out == "f32" else y.cpu().view(torch.int16).numpy().view(np.uint16)
+        np.testing.assert_array_equal(got, ref)
+    assert bl.get_device_status() == 0
 
 
 def test_forward_tiny_config_end_to_end():
