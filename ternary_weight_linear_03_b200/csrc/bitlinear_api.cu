@@ -115,13 +115,16 @@ SkinnyPlan skinny_plan_for(int M, int N, int K, int sms) {
   p.bnt = (M + 15) / 16 * 16;
   p.tiles = (N + bl::sk::BW - 1) / bl::sk::BW;
   const int KB = (K + bl::sk::BK - 1) / bl::sk::BK;
-  // Split K only when the weight tiles alone leave most SMs idle; keep at least
-  // kMinKbPerSplit K blocks per split so that each CTA streams long enough to cover its
-  // fixed costs, and keep the int32 sums the splits exchange (M x N x 4 bytes each)
+  // Split K only when the weight tiles alone leave CTA slots idle (two per SM for token
+  // tiles up to 64, one above), and only as far as every CTA still has a slot: a CTA
+  // runs at the pace of its handoffs, so a second wave would double the time. Keep at
+  // least kMinKbPerSplit K blocks per split so that each CTA streams long enough to cover
+  // its fixed costs, and keep the int32 sums the splits exchange (M x N x 4 bytes each)
   // within a quarter of the packed weight bytes (measured on B200: beyond that the
   // reduction costs more than the extra SMs bring).
+  const long long slots = static_cast<long long>(p.bnt <= 64 ? 2 : 1) * sms;
   long long splits = 1;
-  if (p.tiles < sms) splits = (sms + p.tiles - 1) / p.tiles;
+  if (p.tiles < slots) splits = std::max<long long>(1, slots / p.tiles);
   const long long by_traffic = static_cast<long long>(
       (static_cast<double>(N) * K / 4.0) / (4.0 * 4.0 * static_cast<double>(M) * N));
   splits = std::max<long long>(

@@ -232,33 +232,43 @@ __device__ __forceinline__ void epi_store_chunk(const int (&a)[16], const float 
   constexpr int ES = (OM == 1) ? 2 : 4;  // bytes per element of y
   const int nl = threadIdx.x;            // row within the tile
   const int n = n0 + nl;
+  // Values first, stores next, the chain's absmax last: a branch inside the value loop
+  // would make each value's convert-multiply-convert chain wait for the one before.
+  uint32_t bits[16];
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
-    const int t = c0 + j;
-    uint32_t bits;
-    unsigned mag = 0u;
     if (OM == 2) {
-      bits = static_cast<uint32_t>(a[j]);
+      bits[j] = static_cast<uint32_t>(a[j]);
     } else {
       const float val = __fmul_rn(__int2float_rn(a[j]), fs[j]);
-      if (OM == 0) {
-        bits = __float_as_uint(val);
-        mag = bits & 0x7fffffffu;
-      } else {
-        const __nv_bfloat16 h = __float2bfloat16_rn(val);
-        bits = static_cast<uint32_t>(__bfloat16_as_ushort(h));
-        mag = (bits << 16) & 0x7fffffffu;
+      bits[j] = (OM == 0) ? __float_as_uint(val)
+                          : static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(val)));
+    }
+  }
+  if (vec) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      if (ES == 2) reinterpret_cast<uint16_t*>(stage)[j * 128 + nl] = static_cast<uint16_t>(bits[j]);
+      else reinterpret_cast<uint32_t*>(stage)[j * 128 + nl] = bits[j];
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const long long o = static_cast<long long>(c0 + j) * N + n;
+      if (c0 + j < M && nvalid) {
+        if (ES == 2) static_cast<uint16_t*>(y)[o] = static_cast<uint16_t>(bits[j]);
+        else static_cast<uint32_t*>(y)[o] = bits[j];
       }
     }
-    if (vec) {
-      if (ES == 2) reinterpret_cast<uint16_t*>(stage)[j * 128 + nl] = static_cast<uint16_t>(bits);
-      else reinterpret_cast<uint32_t*>(stage)[j * 128 + nl] = bits;
-    } else if (t < M && nvalid) {
-      const long long o = static_cast<long long>(t) * N + n;
-      if (ES == 2) static_cast<uint16_t*>(y)[o] = static_cast<uint16_t>(bits);
-      else static_cast<uint32_t*>(y)[o] = bits;
+  }
+  if (OM != 2 && amax_out != nullptr) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      if (c0 + j < M) {  // the same for the whole warp
+        const uint32_t mag = (OM == 0) ? (bits[j] & 0x7fffffffu) : ((bits[j] << 16) & 0x7fffffffu);
+        warp_amax_out(amax_out, c0 + j, nvalid ? mag : 0u);
+      }
     }
-    if (OM != 2 && amax_out != nullptr && t < M) warp_amax_out(amax_out, t, nvalid ? mag : 0u);
   }
   if (vec) {
     epi_bar_sync();
