@@ -64,6 +64,47 @@ __device__ __forceinline__ float abs_bits(float x) {
   return __uint_as_float(__float_as_uint(x) & 0x7fffffffu);
 }
 
+// Per-halfword unsigned maximum.
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// Largest |x| of 16 bf16 values (two 16-byte vectors at p), kept as two halfword bit
+// patterns: with the sign cleared, bf16 patterns order like their values, and the NaN
+// patterns lie above infinity (0x7f80), so a maximum at or above 0x7f80 flags a
+// non-finite value.
+__device__ __forceinline__ uint32_t absmax16_bf16(const void* p, uint32_t m2) {
+  const uint4 a = reinterpret_cast<const uint4*>(p)[0], b = reinterpret_cast<const uint4*>(p)[1];
+  const uint32_t h[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+  for (int q = 0; q < 8; ++q) m2 = max_u16x2(m2, h[q] & 0x7fff7fffu);
+  return m2;
+}
+
+// Quantizes 16 bf16 values with a finite r (the same rounding and clamping as quant_i8;
+// its zero test only matters for an infinite r) into four words of int8, byte i & 3 of
+// word i >> 2 holding element i, and adds their sum into *sum.
+__device__ __forceinline__ uint4 quant16_bf16(const void* p, float r, int* sum) {
+  const uint4 a = reinterpret_cast<const uint4*>(p)[0], b = reinterpret_cast<const uint4*>(p)[1];
+  const uint32_t h[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+  uint32_t w[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    int q[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t hw = h[2 * j + (e >> 1)];
+      const float v = __uint_as_float((e & 1) ? (hw & 0xffff0000u) : (hw << 16));
+      q[e] = max(-127, min(127, __float2int_rn(__fmul_rn(v, r))));
+    }
+    w[j] = __byte_perm(__byte_perm(q[0], q[1], 0x0040), __byte_perm(q[2], q[3], 0x0040), 0x5410);
+    *sum = __dp4a(static_cast<int>(w[j]), 0x01010101, *sum);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
 // Zeroes n16 16-byte words at z with the whole grid (the split-K sums and counters of the
 // tensor-core kernel that follows, so that no separate memset sits between the two).
 __device__ __forceinline__ void grid_zero(uint4* __restrict__ z, long long n16) {
@@ -83,8 +124,8 @@ enum AqMode : int {
 // grid = M blocks, K % 8 == 0. rowsum may be null; zero/zero_n16 name an extra region to
 // clear (may be null/0). Lets the dependent kernel launch at once (it waits for this
 // grid's completion before reading any of these outputs).
-template <bool kBf16, int AMODE = kAqRow>
-__global__ void __launch_bounds__(kAqThreads) act_quant_kernel(
+template <bool kBf16, int AMODE = kAqRow, int NT = kAqThreads>
+__global__ void __launch_bounds__(NT) act_quant_kernel(
     const void* __restrict__ x, int K, int8_t* __restrict__ xq, float* __restrict__ scale,
     int* __restrict__ rowsum, uint4* __restrict__ zero, long long zero_n16,
     float* __restrict__ amax = nullptr) {
@@ -104,15 +145,30 @@ __global__ void __launch_bounds__(kAqThreads) act_quant_kernel(
     if (!(a <= 3.4028234663852886e38f)) record_status(kStatusNonfinite);
   } else {
     bool bad = false;
-    for (int c = threadIdx.x; c < nc; c += blockDim.x) {
-      float v[8];
-      load8<kBf16>(row, c, v);
+    // the float pass (fp32 x, or a bf16 thread that saw a non-finite value: NaN is skipped
+    // by fmaxf and flagged)
+    auto float_pass = [&]() {
+      float m = 0.0f;
+      for (int c = threadIdx.x; c < nc; c += blockDim.x) {
+        float v[8];
+        load8<kBf16>(row, c, v);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float m = abs_bits(v[i]);
-        bad |= !(m <= 3.4028234663852886e38f);
-        a = fmaxf(a, m);
+        for (int i = 0; i < 8; ++i) {
+          const float e = abs_bits(v[i]);
+          bad |= !(e <= 3.4028234663852886e38f);
+          m = fmaxf(m, e);
+        }
       }
+      return m;
+    };
+    if (kBf16) {  // K % 16 == 0: one max.u16x2 per two values
+      uint32_t m2 = 0u;
+      for (int c = threadIdx.x; c < K / 16; c += blockDim.x)
+        m2 = absmax16_bf16(row + 32 * static_cast<size_t>(c), m2);
+      const uint32_t m = max(m2 & 0xffffu, m2 >> 16);
+      a = (m < 0x7f80u) ? __uint_as_float(m << 16) : float_pass();
+    } else {
+      a = float_pass();
     }
     if (bad) record_status(kStatusNonfinite);
     a = block_max(a, redf);
@@ -124,7 +180,10 @@ __global__ void __launch_bounds__(kAqThreads) act_quant_kernel(
   const float r = (a > 0.0f) ? __fdiv_rn(127.0f, a) : 0.0f;
   int8_t* qrow = xq + static_cast<size_t>(t) * K;
   int sum = 0;
-  for (int c = threadIdx.x; c < nc; c += blockDim.x) {
+  if (kBf16 && r <= 3.4028234663852886e38f) {  // finite r; 16 values a step (K % 16 == 0)
+    for (int c = threadIdx.x; c < K / 16; c += blockDim.x)
+      reinterpret_cast<uint4*>(qrow)[c] = quant16_bf16(row + 32 * static_cast<size_t>(c), r, &sum);
+  } else for (int c = threadIdx.x; c < nc; c += blockDim.x) {
     float v[8];
     load8<kBf16>(row, c, v);
     uint32_t lo = 0u, hi = 0u;

@@ -118,47 +118,6 @@ __device__ __forceinline__ void load16(const void* x, long long off, float (&v)[
   }
 }
 
-// Per-halfword unsigned maximum.
-__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
-
-// Largest |x| of 16 bf16 values (two 16-byte vectors at p), kept as two halfword bit
-// patterns: with the sign cleared, bf16 patterns order like their values, and the NaN
-// patterns lie above infinity (0x7f80), so a maximum at or above 0x7f80 flags a
-// non-finite value.
-__device__ __forceinline__ uint32_t absmax16_bf16(const void* p, uint32_t m2) {
-  const uint4 a = reinterpret_cast<const uint4*>(p)[0], b = reinterpret_cast<const uint4*>(p)[1];
-  const uint32_t h[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-#pragma unroll
-  for (int q = 0; q < 8; ++q) m2 = max_u16x2(m2, h[q] & 0x7fff7fffu);
-  return m2;
-}
-
-// Quantizes 16 bf16 values with a finite r (the same rounding and clamping as quant_i8;
-// its zero test only matters for an infinite r) into four words of int8, byte i & 3 of
-// word i >> 2 holding element i, and adds their sum into *sum.
-__device__ __forceinline__ uint4 quant16_bf16(const void* p, float r, int* sum) {
-  const uint4 a = reinterpret_cast<const uint4*>(p)[0], b = reinterpret_cast<const uint4*>(p)[1];
-  const uint32_t h[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-  uint32_t w[4];
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    int q[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const uint32_t hw = h[2 * j + (e >> 1)];
-      const float v = __uint_as_float((e & 1) ? (hw & 0xffff0000u) : (hw << 16));
-      q[e] = max(-127, min(127, __float2int_rn(__fmul_rn(v, r))));
-    }
-    w[j] = __byte_perm(__byte_perm(q[0], q[1], 0x0040), __byte_perm(q[2], q[3], 0x0040), 0x5410);
-    *sum = __dp4a(static_cast<int>(w[j]), 0x01010101, *sum);
-  }
-  return make_uint4(w[0], w[1], w[2], w[3]);
-}
-
 // XR: activations in registers (one token). R: rows a warp sums at once on the shared-
 // memory path (2 lets every activation load feed two rows; worth it only with many rows).
 // Layer chains (optional, null when unused): amax_in[t] is the absmax of token t's row of

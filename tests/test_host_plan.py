@@ -2,7 +2,8 @@
 
 Pins the measured rules: the CUDA-core GEMV for one or two tokens, or up to four when the
 packed weights are at most 2 MB; the skinny tensor-core kernel up to 256 tokens, splitting K
-only while each split keeps at least 8 K blocks and the int32 sums the splits exchange stay
+into as many parts as the CTA slots (two per SM for up to 64 tokens, one above) hold in one
+wave, while each split keeps at least 8 K blocks and the int32 sums the splits exchange stay
 within a quarter of the packed weight bytes; the prefill GEMM above 256 tokens."""
 import ctypes
 
@@ -21,8 +22,8 @@ PLANS = [
     ((16, 8640, 3200), ("skinny", 3)),
     ((64, 8640, 3200), ("skinny", 1)),        # the sums of a split would outweigh W / 4
     ((16, 3200, 8640), ("skinny", 6)),
-    ((16, 8192, 28672), ("skinny", 3)),
-    ((176, 8192, 28672), ("skinny", 2)),
+    ((16, 8192, 28672), ("skinny", 4)),       # 64 tiles x 4 splits = 256 CTAs <= 296 slots
+    ((176, 8192, 28672), ("skinny", 2)),      # one CTA per SM above 64 tokens: 128 CTAs
     ((16, 28672, 8192), ("skinny", 1)),       # 224 weight tiles already fill the GPU
     ((256, 1000, 3200), ("skinny", 1)),
     ((257, 1000, 3200), ("prefill", 1)),
@@ -47,7 +48,8 @@ def test_split_rule_invariants():
                     assert kb // splits >= 4  # whole 4-block super-tiles, no empty split
                     assert splits <= kb // 8
                     assert M * N * 4 * splits * 4 <= N * K // 4 + M * N * 4 * 4
-                    assert (N + 127) // 128 < 148
+                    slots = (2 if (M + 15) // 16 * 16 <= 64 else 1) * 148
+                    assert (N + 127) // 128 * splits <= slots  # one wave of CTAs
 
 
 def test_argument_errors():
