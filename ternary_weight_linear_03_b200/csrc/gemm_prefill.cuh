@@ -299,39 +299,53 @@ __global__ void __launch_bounds__(pf::THREADS, 1) gemm_prefill_kernel(
           for (int j = 0; j < 16; ++j) { v[j] = w16[j]; v[j + 16] = 0u; }
         }
         tmem_ld_wait();
+        // Per half (bnt is a multiple of 16, so a 16-column half is all in or all out): the
+        // factors, then the values, the stores and the chain's absmax, each in its own loop.
+        // A branch inside the value loop would make every value's convert-multiply-convert
+        // chain wait for the one before.
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int tj = c0 + j;
-          const int t = t0 + tj;
-          // the tile's factors four at a time (bnt is a multiple of 16)
-          int4 rs4;
-          float4 f4;
-          if ((j & 3) == 0 && tj < bnt) {
-            rs4 = *reinterpret_cast<const int4*>(&sh->rowsum[ab][tj]);
-            f4 = *reinterpret_cast<const float4*>(&sh->f[ab][tj]);
+        for (int hh = 0; hh < 32; hh += 16) {  // halves of 16 columns (fewer live registers)
+          if (c0 + hh >= bnt) break;  // the same for the whole warp
+          int rs[16];
+          float fs[16];
+#pragma unroll
+          for (int j = 0; j < 16; j += 4) {
+            const int4 r4 = *reinterpret_cast<const int4*>(&sh->rowsum[ab][c0 + hh + j]);
+            const float4 f4 = *reinterpret_cast<const float4*>(&sh->f[ab][c0 + hh + j]);
+            rs[j] = r4.x; rs[j + 1] = r4.y; rs[j + 2] = r4.z; rs[j + 3] = r4.w;
+            fs[j] = f4.x; fs[j + 1] = f4.y; fs[j + 2] = f4.z; fs[j + 3] = f4.w;
           }
-          if (tj >= bnt || t >= M) continue;  // the same for the whole warp
-          const int rsj = (j & 3) == 0 ? rs4.x : (j & 3) == 1 ? rs4.y : (j & 3) == 2 ? rs4.z : rs4.w;
-          const float fj = (j & 3) == 0 ? f4.x : (j & 3) == 1 ? f4.y : (j & 3) == 2 ? f4.z : f4.w;
-          const int a = static_cast<int>(v[j]) - rsj;
-          unsigned mag = 0u;
-          if (nvalid) {
-            const long long o = static_cast<long long>(t) * N + n;
+          uint32_t bits[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int a = static_cast<int>(v[hh + j]) - rs[j];
             if (OM == 2) {
-              static_cast<int*>(y)[o] = a;
+              bits[j] = static_cast<uint32_t>(a);
             } else {
-              const float val = __fmul_rn(__int2float_rn(a), fj);
-              if (OM == 0) {
-                static_cast<float*>(y)[o] = val;
-                mag = __float_as_uint(val) & 0x7fffffffu;
-              } else {
-                const __nv_bfloat16 h = __float2bfloat16_rn(val);
-                static_cast<__nv_bfloat16*>(y)[o] = h;
-                mag = __float_as_uint(__bfloat162float(h)) & 0x7fffffffu;
+              const float val = __fmul_rn(__int2float_rn(a), fs[j]);
+              bits[j] = (OM == 0) ? __float_as_uint(val)
+                                  : static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(val)));
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int t = t0 + c0 + hh + j;
+            if (t < M && nvalid) {
+              const long long o = static_cast<long long>(t) * N + n;
+              if (OM == 1) static_cast<uint16_t*>(y)[o] = static_cast<uint16_t>(bits[j]);
+              else static_cast<uint32_t*>(y)[o] = bits[j];
+            }
+          }
+          if (OM != 2 && amax_out != nullptr) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int t = t0 + c0 + hh + j;
+              if (t < M) {  // the same for the whole warp
+                const uint32_t mag = (OM == 0) ? (bits[j] & 0x7fffffffu) : ((bits[j] << 16) & 0x7fffffffu);
+                warp_amax_out(amax_out, t, nvalid ? mag : 0u);
               }
             }
           }
-          if (OM != 2 && amax_out != nullptr) warp_amax_out(amax_out, t, mag);
         }
       }
       tc_fence_before();
