@@ -25,9 +25,22 @@
 // barrier waits, shared-memory load, tcgen05.st, wait::st and arrival per stage is longer
 // than the MMAs of one stage; thread r of a set owns weight row r, TMEM lane r), 8-11
 // epilogue (tcgen05.ld of their 32 lanes, rowsum, rescale, store), 12 TMA producer, 13
-// TMEM owner and MMA issuer (whole-warp loop, one elected lane issues). Three sets over five
-// slots of 176 columns measured slower on B200 (0.89 ms against 0.77 ms at M = 4096). Persistent: one CTA per SM walks the tiles,
-// consecutive CTAs taking consecutive token tiles of one weight tile (L2 reuse of both).
+// TMEM owner and MMA issuer (whole-warp loop, one elected lane issues), 14-16 sentinels.
+// Three sets over five slots of 176 columns measured slower on B200 (0.89 ms against
+// 0.77 ms at M = 4096).
+//
+// Sentinels take every per-stage mbarrier test off the MMA and unpack warps. Measured with
+// clock64 stamps on B200, a test costs 150 to 450 cycles even for a phase completed long
+// before: the MMA warp's (is the stage's A slot written?) cost it about 190 cycles per
+// stage against about 250 for the four MMAs and two commits, and an unpack set's two
+// (stage landed, A slot free) about 335 of its 765 cycles per stage. Warp 14 tests for
+// the MMA warp, warps 15 and 16 for unpack sets 0 and 1. Each pair meets once per stage at
+// a named barrier (bar.red, which also ORs the failure flags so that both sides leave
+// together), and the sentinel tests the next stage while its partner works on the
+// current one (0.68 against 0.70 ms per step at M = 4096).
+//
+// Persistent: one CTA per SM walks the tiles, consecutive CTAs taking consecutive token
+// tiles of one weight tile (L2 reuse of both).
 // Every mbarrier wait is bounded; on a timeout the kernel records BL_ERR_TIMEOUT, waits
 // (bounded) for its own copies and MMAs, frees TMEM and exits.
 #pragma once
@@ -55,7 +68,9 @@ constexpr int UNPACK_WARPS = 4 * UNPACK_SETS;
 constexpr int EPI_WARP0 = UNPACK_WARPS;        // 4 epilogue warps
 constexpr int TMA_WARP = EPI_WARP0 + 4;
 constexpr int MMA_WARP = TMA_WARP + 1;
-constexpr int THREADS = 32 * (MMA_WARP + 1);
+constexpr int SENTINEL_WARP = MMA_WARP + 1;        // tests for the MMA warp
+constexpr int SET_SENTINEL0 = SENTINEL_WARP + 1;    // tests for unpack set 0, then set 1
+constexpr int THREADS = 32 * (SET_SENTINEL0 + UNPACK_SETS);
 static_assert(A_COL0 + ASLOTS * A_COLS <= TMEM_COLS, "TMEM budget");
 static_assert(X_BYTES % 1024 == 0, "swizzle atoms of the token stages stay aligned");
 static_assert(EPI_WARP0 % 4 == 0, "epilogue warp q reads TMEM lanes 32 q");
@@ -92,6 +107,14 @@ __host__ __device__ constexpr int token_tile(int M) {
 
 __device__ __forceinline__ void epi4_bar_sync() {  // the 4 epilogue warps only
   asm volatile("bar.sync 3, 128;" ::: "memory");
+}
+// The per-stage handoff of the sentinel and MMA warps (named barrier 4): returns the OR of
+// both warps' flags.
+__device__ __forceinline__ bool stage_bar_or(bool v) { return bar_or<4, 64>(v); }
+// The per-stage handoff of unpack set `set` and its sentinel (named barriers 5 and 6, the
+// set's four warps and the sentinel warp).
+__device__ __forceinline__ bool set_bar_or(int set, bool v) {
+  return set == 0 ? bar_or<5, 160>(v) : bar_or<6, 160>(v);
 }
 
 // OM: 0 fp32 out, 1 bf16 out, 2 int32 out (acc only). bnt = token tile (multiple of 16,
@@ -181,18 +204,18 @@ __global__ void __launch_bounds__(pf::THREADS, 1) gemm_prefill_kernel(
     const uint32_t idesc = idesc_i8(BW, bnt);
     const uint64_t x_desc0 = smem_desc_k128(smem_u32(sX));
     int s = 0, a = 0, ab = 0;
-    uint32_t sph = 0, aph = 0, abph = 0;
+    uint32_t sph = 0, abph = 0;
     bool ok = true, issued_any = false;
     for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
       bool got = true;
       if (lane == 0) got = tc_wait(&bar->tmem_empty[ab], abph ^ 1u, limit_ns, abort_flag);
-      if (!__shfl_sync(0xffffffffu, got, 0)) { ok = false; break; }
+      got = __shfl_sync(0xffffffffu, got, 0);
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(ab * MAX_BNT);
       for (int kb = 0; kb < KB; ++kb) {
-        // a_full of slot a implies the stage's TMA data landed (the unpack waited for it)
-        if (lane == 0) got = tc_wait(&bar->a_full[a], aph, limit_ns, abort_flag);
-        if (!__shfl_sync(0xffffffffu, got, 0)) { ok = false; break; }
+        // The sentinel has seen a_full of slot a, which implies the stage's TMA data landed
+        // (the unpack waited for it). A failed accumulator wait leaves at the first handoff.
+        if (stage_bar_or(!got)) { ok = false; break; }
         tc_fence_after();
         const uint32_t a_tmem = tmem_base + static_cast<uint32_t>(A_COL0 + a * A_COLS);
         const uint64_t b_desc = x_desc0 + static_cast<uint64_t>(s * (X_BYTES >> 4));
@@ -205,7 +228,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1) gemm_prefill_kernel(
         mma_commit_elect(&bar->empty[s]);
         mma_commit_elect(&bar->a_empty[a]);
         if (++s == STAGES) { s = 0; sph ^= 1u; }
-        if (++a == ASLOTS) { a = 0; aph ^= 1u; }
+        if (++a == ASLOTS) a = 0;
       }
       if (!ok) break;
       mma_commit_elect(&bar->tmem_full[ab]);
@@ -216,6 +239,37 @@ __global__ void __launch_bounds__(pf::THREADS, 1) gemm_prefill_kernel(
       mma_commit_elect(&bar->drain);  // completes once every MMA issued above has finished
       if (lane == 0) mbar_wait(&bar->drain, 0u, 100000000ull);
       __syncwarp();
+    }
+  } else if (warp == SENTINEL_WARP) {
+    // ------------------------------------------------------------------ sentinel
+    int a = 0;
+    uint32_t aph = 0;
+    bool stop = false;
+    for (int tile = blockIdx.x; tile < num_tiles && !stop; tile += gridDim.x) {
+      for (int kb = 0; kb < KB; ++kb) {
+        bool got = true;
+        if (lane == 0) got = tc_wait(&bar->a_full[a], aph, limit_ns, abort_flag);
+        if (stage_bar_or(!__shfl_sync(0xffffffffu, got, 0))) { stop = true; break; }
+        if (++a == ASLOTS) { a = 0; aph ^= 1u; }
+      }
+    }
+  } else if (warp >= SET_SENTINEL0) {
+    // ------------------------------------------------------------------ set sentinels
+    const int set = warp - SET_SENTINEL0;
+    long long g = 0;
+    bool stop = false;
+    for (int tile = blockIdx.x; tile < num_tiles && !stop; tile += gridDim.x) {
+      for (int kb = 0; kb < KB; ++kb, ++g) {
+        if (static_cast<int>(g % UNPACK_SETS) != set) continue;
+        bool got = true;
+        if (lane == 0)
+          got = tc_wait(&bar->full[g % STAGES], static_cast<uint32_t>((g / STAGES) & 1),
+                        limit_ns, abort_flag);
+        else if (lane == 1)
+          got = tc_wait(&bar->a_empty[g % ASLOTS], static_cast<uint32_t>(((g / ASLOTS) & 1) ^ 1),
+                        limit_ns, abort_flag);
+        if (set_bar_or(set, !__all_sync(0xffffffffu, got))) { stop = true; break; }
+      }
     }
   } else if (warp < UNPACK_WARPS) {
     // ------------------------------------------------------------------ unpack warps
@@ -234,11 +288,9 @@ __global__ void __launch_bounds__(pf::THREADS, 1) gemm_prefill_kernel(
         if (static_cast<int>(g % UNPACK_SETS) != set) continue;
         const int s = static_cast<int>(g % STAGES);
         const int a = static_cast<int>(g % ASLOTS);
-        const uint32_t ph = static_cast<uint32_t>((g / STAGES) & 1);
-        const uint32_t aph = static_cast<uint32_t>((g / ASLOTS) & 1);
-        const bool got = tc_wait(&bar->full[s], ph, limit_ns, abort_flag) &&
-                         tc_wait(&bar->a_empty[a], aph ^ 1u, limit_ns, abort_flag);
-        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+        // the set's sentinel has seen the stage land and the slot freed
+        if (set_bar_or(set, false)) { ok = false; break; }
+        tc_fence_after();
         const uint4* src = reinterpret_cast<const uint4*>(sW + s * WP_BYTES + r * 32);
         const uint4 first = src[h0], second = src[h0 ^ 1];
         const uint4 halves[2] = {h0 ? second : first, h0 ? first : second};
