@@ -415,17 +415,26 @@ __global__ void __launch_bounds__(kWqThreads) weight_quant_kernel(
       if (single) {  // provisional codes against T^, and the band entries
         const int c = tid + i * kWqThreads;
         uint32_t bits = 0u;
+        uint32_t in_band = 0u;  // bit e: |w[e]| within the band
 #pragma unroll
         for (int e = 0; e < E; ++e) {
           const uint32_t wb = __float_as_uint(w[e]);
           const uint32_t ab = wb & 0x7fffffffu;
           bits += ((ab >= t_b) ? 2u - ((wb >> 30) & 2u) : 1u) * mulA[e];  // |w| >= T^
-          if (c < nchunks && (ab - band_b) <= bspan_b) {  // |w| within the band
-            const unsigned idx = atomicAdd(&s_cnt, 1u);
-            if (idx < static_cast<unsigned>(kWqListCap))
-              list[static_cast<long long>(blockIdx.x) * kWqListCap + idx] = make_uint2(
-                  static_cast<uint32_t>((1ll * st * kWqStageBytes + 16ll * c) / (16 / E) + e),
-                  __float_as_uint(w[e]));
+          in_band |= ((ab - band_b) <= bspan_b ? 1u : 0u) << e;
+        }
+        // Rare: list the band entries. Kept out of the loop above, where a branch holding
+        // the atomic would make every weight's work wait for the one before.
+        if (c < nchunks && in_band != 0u) {
+#pragma unroll
+          for (int e = 0; e < E; ++e) {
+            if ((in_band >> e) & 1u) {
+              const unsigned idx = atomicAdd(&s_cnt, 1u);
+              if (idx < static_cast<unsigned>(kWqListCap))
+                list[static_cast<long long>(blockIdx.x) * kWqListCap + idx] = make_uint2(
+                    static_cast<uint32_t>((1ll * st * kWqStageBytes + 16ll * c) / (16 / E) + e),
+                    __float_as_uint(w[e]));
+            }
           }
         }
         bits = wq_or_parts<kBf16>(bits);
