@@ -13,14 +13,20 @@
 // The trits are exact in bf16 (+-1, 0) and every bf16 x bf16 product is exact in fp32, so
 // the only rounding is the fp32 accumulation.
 //
-// One persistent CTA per SM, 10 warps as the int8 prefill GEMM: warp 0 issues the TMA
-// loads (A tile 128 x 64, B tile 256 x 64 bf16, or the packed B tile 256 x 16 bytes),
-// warp 1 owns TMEM (two 128 x 256 fp32 accumulators) and issues 4 MMAs (K = 16) per
-// stage, warps 2, 3, 8, 9 unpack the trits to bf16 (when B is packed), warps 4..7 drain
-// the accumulator (tcgen05.ld), scale and store. Every wait is bounded (status word).
+// One persistent CTA per SM, 12 warps: warp 0 issues the TMA loads (A tile 128 x 64, B
+// tile 256 x 64 bf16, or the packed B tile 256 x 16 bytes), warp 1 owns TMEM (two
+// 128 x 256 fp32 accumulators) and issues 4 MMAs (K = 16) per stage (whole-warp loop, one
+// elected lane issues), warps 2, 3, 8, 9 unpack the trits to bf16 (when B is packed),
+// warps 4..7 drain the accumulator (tcgen05.ld), scale and store. Warps 10 and 11 are
+// sentinels: they do the per-stage mbarrier tests for the MMA warp (stage landed, B
+// unpacked) and for the unpack warps (stage landed, unpacked slot free), each test about
+// 200 to 450 cycles on B200 even for a completed phase, and hand over once per stage at a
+// named barrier (bar.red, which also ORs the failure flags so that both sides leave
+// together). Every wait is bounded (status word).
 #pragma once
 
 #include "common.cuh"
+#include "gemm_skinny.cuh"
 #include "gemm_tc.cuh"
 
 namespace bl {
@@ -36,7 +42,8 @@ constexpr int A_BYTES = BM * 128;      // 16 KB
 constexpr int BT_BYTES = BN * 128;     // 32 KB bf16 B tile
 constexpr int BP_BYTES = BN * BKE / 4; // 4 KB packed B tile
 constexpr int TMEM_COLS = 2 * BN;
-constexpr int THREADS = 320;
+constexpr int THREADS = 384;
+constexpr int MMA_SENTINEL = 10, UNPACK_SENTINEL = 11;
 
 // D fp32 (bits 4-5 = 1), A and B bf16 (bits 7-9 = 1, 10-12 = 1), both K-major, N >> 3 in
 // bits 17-22, M >> 4 in bits 24-28.
@@ -67,15 +74,22 @@ __host__ __device__ constexpr int smem_bytes() {
 }
 }  // namespace bf
 
-__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                         uint32_t idesc, uint32_t accumulate) {
+// Warp-collective bf16 MMA: every lane calls it, one elected lane issues.
+__device__ __forceinline__ void mma_bf16_elect(uint32_t d_tmem, uint64_t a_desc,
+                                               uint64_t b_desc, uint32_t idesc,
+                                               uint32_t accumulate) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// The per-stage handoffs: MMA warp and its sentinel (named barrier 4, 64 threads); the
+// four unpack warps and theirs (named barrier 5, 160 threads).
+__device__ __forceinline__ bool bf_mma_bar_or(bool v) { return bar_or<4, 64>(v); }
+__device__ __forceinline__ bool bf_unp_bar_or(bool v) { return bar_or<5, 160>(v); }
 
 // Two trits of one packed word as two bf16 codes c = u - 1 (low half = the first):
 // t holds u of the first trit in bits 0-1 and of the second in bits 8-9. The byte permute
@@ -171,40 +185,78 @@ __global__ void __launch_bounds__(bf::THREADS, 1) gemm_bf16_kernel(
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint64_t a_desc0 = smem_desc_k128(smem_u32(sA));
-      const uint64_t b_desc0 = smem_desc_k128(smem_u32(sB));
-      int s = 0, u = 0, ab = 0;
-      uint32_t ph = 0, uph = 0, aph = 0;
-      bool ok = true, issued_any = false;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        if (!tc_wait(&bar->tmem_empty[ab], aph ^ 1u, limit_ns, abort_flag)) { ok = false; break; }
+    const uint64_t a_desc0 = smem_desc_k128(smem_u32(sA));
+    const uint64_t b_desc0 = smem_desc_k128(smem_u32(sB));
+    int s = 0, u = 0, ab = 0;
+    uint32_t aph = 0;
+    bool ok = true, issued_any = false;
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      bool got = true;
+      if (lane == 0) got = tc_wait(&bar->tmem_empty[ab], aph ^ 1u, limit_ns, abort_flag);
+      got = __shfl_sync(0xffffffffu, got, 0);
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(ab * BN);
+      for (int kb = 0; kb < KB; ++kb) {
+        // the sentinel has seen the stage land (and its B unpacked); a failed accumulator
+        // wait leaves at the first handoff
+        if (bf_mma_bar_or(!got)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(ab * BN);
-        for (int kb = 0; kb < KB; ++kb) {
-          if ((kPacked && !tc_wait(&bar->full_unp[u], uph, limit_ns, abort_flag)) ||
-              !tc_wait(&bar->full_tma[s], ph, limit_ns, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          const uint64_t a_desc = a_desc0 + static_cast<uint64_t>(s * (A_BYTES >> 4));
-          const uint64_t b_desc =
-              b_desc0 + static_cast<uint64_t>((kPacked ? u : s) * (BT_BYTES >> 4));
+        const uint64_t a_desc = a_desc0 + static_cast<uint64_t>(s * (A_BYTES >> 4));
+        const uint64_t b_desc =
+            b_desc0 + static_cast<uint64_t>((kPacked ? u : s) * (BT_BYTES >> 4));
 #pragma unroll
-          for (int kk = 0; kk < BKE / MMA_K; ++kk)  // 32 bytes of bf16 per MMA
-            mma_bf16(d_tmem, a_desc + static_cast<uint64_t>(kk * 2),
-                     b_desc + static_cast<uint64_t>(kk * 2), IDESC, (kb | kk) != 0 ? 1u : 0u);
-          issued_any = true;
-          mma_commit(&bar->empty_tma[s]);
-          if (kPacked) mma_commit(&bar->empty_unp[u]);
-          if (++s == STAGES) { s = 0; ph ^= 1u; }
-          if (kPacked && ++u == USTAGES) { u = 0; uph ^= 1u; }
-        }
-        if (!ok) break;
-        mma_commit(&bar->tmem_full[ab]);
-        if (++ab == 2) { ab = 0; aph ^= 1u; }
+        for (int kk = 0; kk < BKE / MMA_K; ++kk)  // 32 bytes of bf16 per MMA
+          mma_bf16_elect(d_tmem, a_desc + static_cast<uint64_t>(kk * 2),
+                         b_desc + static_cast<uint64_t>(kk * 2), IDESC, (kb | kk) != 0 ? 1u : 0u);
+        issued_any = true;
+        mma_commit_elect(&bar->empty_tma[s]);
+        if (kPacked) mma_commit_elect(&bar->empty_unp[u]);
+        if (++s == STAGES) s = 0;
+        if (kPacked && ++u == USTAGES) u = 0;
       }
-      if (!ok && issued_any) {
-        mma_commit(&bar->drain);
-        mbar_wait(&bar->drain, 0u, 100000000ull);
+      if (!ok) break;
+      mma_commit_elect(&bar->tmem_full[ab]);
+      if (++ab == 2) { ab = 0; aph ^= 1u; }
+    }
+    if (!ok && issued_any) {
+      mma_commit_elect(&bar->drain);
+      if (lane == 0) mbar_wait(&bar->drain, 0u, 100000000ull);
+      __syncwarp();
+    }
+  } else if (warp == MMA_SENTINEL) {
+    // ------------------------------------------------------------------ MMA sentinel
+    // lane 0: stage g's TMA data landed; lane 1 (packed B): its B tile unpacked
+    long long g = 0;
+    bool stop = false;
+    for (int tile = blockIdx.x; tile < num_tiles && !stop; tile += gridDim.x) {
+      for (int kb = 0; kb < KB; ++kb, ++g) {
+        bool got = true;
+        if (lane == 0)
+          got = tc_wait(&bar->full_tma[g % STAGES], static_cast<uint32_t>((g / STAGES) & 1),
+                        limit_ns, abort_flag);
+        else if (kPacked && lane == 1)
+          got = tc_wait(&bar->full_unp[g % USTAGES], static_cast<uint32_t>((g / USTAGES) & 1),
+                        limit_ns, abort_flag);
+        if (bf_mma_bar_or(!__all_sync(0xffffffffu, got))) { stop = true; break; }
+      }
+    }
+  } else if (warp == UNPACK_SENTINEL) {
+    // ------------------------------------------------------------------ unpack sentinel
+    // lane 0: stage g's TMA data landed; lane 1: its unpacked slot is free
+    if (kPacked) {
+      long long g = 0;
+      bool stop = false;
+      for (int tile = blockIdx.x; tile < num_tiles && !stop; tile += gridDim.x) {
+        for (int kb = 0; kb < KB; ++kb, ++g) {
+          bool got = true;
+          if (lane == 0)
+            got = tc_wait(&bar->full_tma[g % STAGES], static_cast<uint32_t>((g / STAGES) & 1),
+                          limit_ns, abort_flag);
+          else if (lane == 1)
+            got = tc_wait(&bar->empty_unp[g % USTAGES],
+                          static_cast<uint32_t>(((g / USTAGES) & 1) ^ 1), limit_ns, abort_flag);
+          if (bf_unp_bar_or(!__all_sync(0xffffffffu, got))) { stop = true; break; }
+        }
       }
     }
   } else if (warp >= 4 && warp < 8) {
@@ -257,13 +309,11 @@ __global__ void __launch_bounds__(bf::THREADS, 1) gemm_bf16_kernel(
     const int uw = (warp < 4) ? (warp - 2) : (warp - 6);
     const int ut = uw * 32 + lane;
     int s = 0, u = 0;
-    uint32_t ph = 0, uph = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
       for (int kb = 0; kb < KB; ++kb) {
-        const bool got = tc_wait(&bar->full_tma[s], ph, limit_ns, abort_flag) &&
-                         tc_wait(&bar->empty_unp[u], uph ^ 1u, limit_ns, abort_flag);
-        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+        // the sentinel has seen the stage land and the unpacked slot freed
+        if (bf_unp_bar_or(false)) { ok = false; break; }
         const uint32_t* src = reinterpret_cast<const uint32_t*>(sBp + s * BP_BYTES);
         unsigned char* dst = sB + u * BT_BYTES;
 #pragma unroll 2
@@ -289,8 +339,8 @@ __global__ void __launch_bounds__(bf::THREADS, 1) gemm_bf16_kernel(
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar->full_unp[u]);
-        if (++s == STAGES) { s = 0; ph ^= 1u; }
-        if (++u == USTAGES) { u = 0; uph ^= 1u; }
+        if (++s == STAGES) s = 0;
+        if (++u == USTAGES) u = 0;
       }
     }
   }
