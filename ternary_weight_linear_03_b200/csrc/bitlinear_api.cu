@@ -879,10 +879,10 @@ bl_status bitlinear_backward(const void* x, int x_dtype, const void* grad_y,
     if (ws_bytes < w.bytes) return BL_ERR_WORKSPACE;
     bl_status st = launch_act_quant(x, x_dtype, M, K, w.f.xq, w.f.scale, nullptr, s);
     if (st != BL_OK) return st;
-    const int tiles_g = ((w.Mp + 31) / 32) * ((N + 31) / 32);
+    const int tiles_g = ((w.Mp + 63) / 64) * (N / 64);
     bl::transpose_bf16_kernel<0><<<grid_for(tiles_g, 1), 256, 0, s>>>(grad_y, nullptr, w.gT, M,
                                                                        N, w.Mp);
-    const int tiles_x = ((w.Mp + 31) / 32) * ((K + 31) / 32);
+    const int tiles_x = ((w.Mp + 63) / 64) * (K / 64);
     bl::transpose_bf16_kernel<1><<<grid_for(tiles_x, 1), 256, 0, s>>>(w.f.xq, w.f.scale, w.xT,
                                                                        M, K, w.Mp);
     if (launch_status() != BL_OK) return BL_ERR_CUDA;

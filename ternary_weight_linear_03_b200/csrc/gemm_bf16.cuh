@@ -357,39 +357,70 @@ __global__ void __launch_bounds__(bf::THREADS, 1) gemm_bf16_kernel(
 }
 
 // Tile transpose into bf16, for the grad_w operands: out[c][r] for r < R (columns R..Rp-1
-// of out are written as zero; Rp = the padded row length of out). MODE 0: in is bf16 [R][C]
-// (G -> G^T). MODE 1: in is int8 codes q [R][C] with per-row scale s (X~ = bf16(q s),
-// round half to even, transposed). 32 x 32 tiles through shared memory.
+// of out are written as zero; Rp = the padded row length of out, a multiple of 8). MODE 0:
+// in is bf16 [R][C] (G -> G^T). MODE 1: in is int8 codes q [R][C] with per-row scale s
+// (X~ = bf16(q s), round half to even, transposed). C % 64 == 0. 64 x 64 tiles through
+// shared memory, every global access 8 elements wide (16 bytes of bf16, 8 of int8); the
+// shared rows are 66 elements apart, so that both the row writes and the column gathers
+// meet at most two threads per bank.
 template <int MODE>
 __global__ void __launch_bounds__(256) transpose_bf16_kernel(
     const void* __restrict__ in, const float* __restrict__ scale,
     __nv_bfloat16* __restrict__ out, int R, int C, int Rp) {
-  __shared__ uint16_t tile[32][33];
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8
-  const int tiles_r = (Rp + 31) / 32, tiles_c = (C + 31) / 32;
+  constexpr int TS = 66;  // shared row stride in elements
+  __shared__ __align__(16) uint16_t tile[64 * TS];
+  const int tiles_r = (Rp + 63) / 64, tiles_c = C / 64;
   for (long long tl = blockIdx.x; tl < static_cast<long long>(tiles_r) * tiles_c; tl += gridDim.x) {
-    const int r0 = static_cast<int>(tl % tiles_r) * 32, c0 = static_cast<int>(tl / tiles_r) * 32;
-    for (int i = ty; i < 32; i += 8) {
-      const int r = r0 + i, c = c0 + tx;
-      uint16_t v = 0;
-      if (r < R && c < C) {
+    const int r0 = static_cast<int>(tl % tiles_r) * 64, c0 = static_cast<int>(tl / tiles_r) * 64;
+    // rows r0 .. r0 + 63 in: piece p = 8 elements of row p / 8
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int p = threadIdx.x + 256 * h;
+      const int rr = p >> 3, c8 = p & 7;
+      const int r = r0 + rr, c = c0 + 8 * c8;
+      uint32_t w[4] = {0u, 0u, 0u, 0u};
+      if (r < R) {
         if (MODE == 0) {
-          v = static_cast<const uint16_t*>(in)[static_cast<long long>(r) * C + c];
+          const uint4 v = *reinterpret_cast<const uint4*>(
+              static_cast<const uint16_t*>(in) + static_cast<long long>(r) * C + c);
+          w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
         } else {
-          const float f = __fmul_rn(
-              static_cast<float>(static_cast<const int8_t*>(in)[static_cast<long long>(r) * C + c]),
-              scale[r]);
-          const __nv_bfloat16 h = __float2bfloat16_rn(f);
-          v = *reinterpret_cast<const uint16_t*>(&h);
+          const uint2 q = *reinterpret_cast<const uint2*>(
+              static_cast<const int8_t*>(in) + static_cast<long long>(r) * C + c);
+          const float sr = scale[r];
+          const uint32_t qq[2] = {q.x, q.y};
+#pragma unroll
+          for (int e = 0; e < 8; e += 2) {
+            const int b0 = static_cast<int8_t>((qq[e >> 2] >> (8 * (e & 3))) & 0xffu);
+            const int b1 = static_cast<int8_t>((qq[e >> 2] >> (8 * ((e + 1) & 3))) & 0xffu);
+            const __nv_bfloat16 h0 = __float2bfloat16_rn(__fmul_rn(static_cast<float>(b0), sr));
+            const __nv_bfloat16 h1 = __float2bfloat16_rn(__fmul_rn(static_cast<float>(b1), sr));
+            w[e >> 1] = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) |
+                        (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
+          }
         }
       }
-      tile[i][tx] = v;
+      uint32_t* dst = reinterpret_cast<uint32_t*>(tile + rr * TS + 8 * c8);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) dst[k] = w[k];
     }
     __syncthreads();
-    for (int i = ty; i < 32; i += 8) {
-      const int c = c0 + i, r = r0 + tx;
-      if (c < C && r < Rp)
-        reinterpret_cast<uint16_t*>(out)[static_cast<long long>(c) * Rp + r] = tile[tx][i];
+    // columns c0 .. c0 + 63 out: piece p = 8 rows of output row p / 8
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int p = threadIdx.x + 256 * h;
+      const int cc = p >> 3, r8 = p & 7;
+      const int r = r0 + 8 * r8;
+      if (r < Rp) {  // Rp % 8 == 0: a piece is all in or all out
+        uint32_t w[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          w[k] = static_cast<uint32_t>(tile[(8 * r8 + 2 * k) * TS + cc]) |
+                 (static_cast<uint32_t>(tile[(8 * r8 + 2 * k + 1) * TS + cc]) << 16);
+        *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(out) +
+                                  static_cast<long long>(c0 + cc) * Rp + r) =
+            make_uint4(w[0], w[1], w[2], w[3]);
+      }
     }
     __syncthreads();
   }
