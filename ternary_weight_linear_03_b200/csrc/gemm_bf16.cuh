@@ -38,8 +38,9 @@ constexpr int BN = 192;                // B rows per tile (MMA N); 192 rather th
                                        // SMs (measured 117 against 133 us for grad_x)
 constexpr int BKE = 64;                // contraction elements per stage (128 bytes of bf16)
 constexpr int MMA_K = 16;              // K per tcgen05.mma kind::f16
-constexpr int STAGES = 4;
-constexpr int USTAGES = 2;
+constexpr int STAGES = 5;               // TMA ring (A and B, or A and packed B)
+constexpr int USTAGES = 3;              // unpacked B ring (5 / 3 against 4 / 2:
+                                        // 105 against 117 us for grad_x)
 constexpr int A_BYTES = BM * 128;      // 16 KB
 constexpr int BT_BYTES = BN * 128;     // 24 KB bf16 B tile
 constexpr int BP_BYTES = BN * BKE / 4; // 3 KB packed B tile
