@@ -70,18 +70,40 @@ __global__ void __launch_bounds__(kGemv3Threads) gemv3_kernel(
   bool bad = false;
 #pragma unroll
   for (int t = 0; t < MT; ++t) amax[t] = 0.0f;
-  for (int kb = tid; kb < KB; kb += kGemv3Threads) {
-#pragma unroll
-    for (int t = 0; t < MT; ++t) {
+  // the float pass (fp32 x, or a bf16 thread that saw a non-finite value: NaN is skipped by
+  // fmaxf and flagged)
+  auto amax_pass = [&](int t) {
+    float a = 0.0f;
+    for (int kb = tid; kb < KB; kb += kGemv3Threads) {
       float v[16];
       load16<XM>(x, static_cast<long long>(t) * K + 16 * kb, v);
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const float m = abs_bits(v[i]);
         bad |= !(m <= 3.4028234663852886e38f);
-        amax[t] = fmaxf(amax[t], m);
+        a = fmaxf(a, m);
       }
     }
+    return a;
+  };
+  if (XM == kXbf16) {  // one max.u16x2 per two values on the sign-cleared bit patterns
+    uint32_t m2[MT];
+#pragma unroll
+    for (int t = 0; t < MT; ++t) m2[t] = 0u;
+    for (int kb = tid; kb < KB; kb += kGemv3Threads) {
+#pragma unroll
+      for (int t = 0; t < MT; ++t)
+        m2[t] = absmax16_bf16(static_cast<const uint16_t*>(x) + static_cast<long long>(t) * K + 16 * kb,
+                              m2[t]);
+    }
+#pragma unroll
+    for (int t = 0; t < MT; ++t) {
+      const uint32_t m = max(m2[t] & 0xffffu, m2[t] >> 16);
+      amax[t] = (m < 0x7f80u) ? __uint_as_float(m << 16) : amax_pass(t);
+    }
+  } else {
+#pragma unroll
+    for (int t = 0; t < MT; ++t) amax[t] = amax_pass(t);
   }
   if (bad) record_status(kStatusNonfinite);
 #pragma unroll
@@ -106,18 +128,25 @@ __global__ void __launch_bounds__(kGemv3Threads) gemv3_kernel(
   for (int kb = tid; kb < KP / 16; kb += kGemv3Threads) {
 #pragma unroll
     for (int t = 0; t < MT; ++t) {
-      uint32_t w4[4] = {0u, 0u, 0u, 0u};
+      uint4 q4 = make_uint4(0u, 0u, 0u, 0u);
       if (kb < KB) {
-        float v[16];
-        load16<XM>(x, static_cast<long long>(t) * K + 16 * kb, v);
+        if (XM == kXbf16 && r[t] <= 3.4028234663852886e38f) {  // finite r (0 when amax is 0)
+          q4 = quant16_bf16(static_cast<const uint16_t*>(x) + static_cast<long long>(t) * K + 16 * kb,
+                            r[t], &sum[t]);
+        } else {
+          float v[16];
+          load16<XM>(x, static_cast<long long>(t) * K + 16 * kb, v);
+          uint32_t w4[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int q = (amax[t] > 0.0f) ? quant_i8(v[i], r[t]) : 0;
-          sum[t] += q;
-          w4[i >> 2] |= (static_cast<uint32_t>(q) & 0xffu) << (8 * (i & 3));
+          for (int i = 0; i < 16; ++i) {
+            const int q = (amax[t] > 0.0f) ? quant_i8(v[i], r[t]) : 0;
+            sum[t] += q;
+            w4[i >> 2] |= (static_cast<uint32_t>(q) & 0xffu) << (8 * (i & 3));
+          }
+          q4 = make_uint4(w4[0], w4[1], w4[2], w4[3]);
         }
       }
-      reinterpret_cast<uint4*>(xs3 + t * KP)[kb] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+      reinterpret_cast<uint4*>(xs3 + t * KP)[kb] = q4;
     }
   }
 #pragma unroll
