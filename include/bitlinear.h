@@ -303,9 +303,10 @@ bl_status bitlinear_debug_timeout_probe(uint64_t timeout_ns, void* stream);
  * nothing queued). For an M x N x K forward on a GPU with `sms` multiprocessors:
  *   *path      0 = CUDA-core GEMV (M <= 2, or M <= 4 with at most 2 MB of packed weights),
  *              1 = skinny tcgen05 kernel (other M <= 256), 2 = prefill tcgen05 GEMM.
- *   *k_splits  CTAs sharing each 128-row weight tile along K on path 1 (at least 8 K blocks
- *              of 128 per split, and the int32 sums they exchange, M*N*4 bytes per split,
- *              within a quarter of the packed weight bytes); 1 otherwise.
+ *   *k_splits  CTAs sharing each 128-row weight tile along K on path 1: as many as the CTA
+ *              slots (two per SM up to 64 tokens, one above) hold in one wave, with at least
+ *              8 K blocks of 128 per split and the int32 sums they exchange, M*N*4 bytes per
+ *              split, within a quarter of the packed weight bytes; 1 otherwise.
  * BL_ERR_INVALID_ARG for null pointers or sms < 1; BL_ERR_UNSUPPORTED_SHAPE as above. */
 bl_status bitlinear_debug_plan(int M, int N, int K, int sms, int* path, int* k_splits);
 
