@@ -575,37 +575,58 @@ def main():
     tokens = M * args.steps * world
     value = tokens / (elapsed_ms * 1e-3)
 
-    # end to end through the public API with host buffers (pinned): the batch goes up, the
-    # forward runs on the resident packed weights, the output comes back, every step
+    # end to end through the public API with host buffers (pinned): every step, the batch
+    # goes up, the forward runs on the resident packed weights and the output comes back.
+    # Three streams and two buffers of each kind: the upload of step i + 1 and the download
+    # of step i - 1 run while the forward of step i computes (PCIe is full duplex, with a
+    # copy engine per direction), as a serving loop would overlap them.
     e2e = None
     if not args.no_e2e:
         x_h = xs[0].cpu().pin_memory()
-        y_h = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
-        x_d = torch.empty_like(xs[0])
+        y_hs = [torch.empty((M, N), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+        x_ds = [torch.empty_like(xs[0]) for _ in range(2)]
+        y_ds = [y, torch.empty_like(y)]
         packed, gamma = ws_copies[0]
         e2e_steps = max(3, min(args.steps, 20))
+        s_in = torch.cuda.Stream(device)
+        s_out = torch.cuda.Stream(device)
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_comp = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
 
-        def e2e_step():
-            x_d.copy_(x_h, non_blocking=True)
-            bl.forward(x_d, packed, gamma, y=y, ws=work)
-            y_h.copy_(y, non_blocking=True)
+        def e2e_step(i):
+            b = i % 2
+            s_in.wait_event(ev_comp[b])  # the forward two steps back has read x_ds[b]
+            with torch.cuda.stream(s_in):
+                x_ds[b].copy_(x_h, non_blocking=True)
+            ev_in[b].record(s_in)
+            stream.wait_event(ev_in[b])
+            stream.wait_event(ev_out[b])  # y_ds[b] of two steps back is home
+            bl.forward(x_ds[b], packed, gamma, y=y_ds[b], ws=work, stream=stream)
+            ev_comp[b].record(stream)
+            s_out.wait_event(ev_comp[b])
+            with torch.cuda.stream(s_out):
+                y_hs[b].copy_(y_ds[b], non_blocking=True)
+            ev_out[b].record(s_out)
 
-        for _ in range(2):
-            e2e_step()
+        for i in range(2):
+            e2e_step(i)
         torch.cuda.synchronize()
         if dist is not None:
             dist.barrier()
         s2 = torch.cuda.Event(enable_timing=True)
         e2 = torch.cuda.Event(enable_timing=True)
-        s2.record(stream)
-        for _ in range(e2e_steps):
-            e2e_step()
-        e2.record(stream)
+        s2.record(s_in)
+        for i in range(e2e_steps):
+            e2e_step(i)
+        s_in.wait_stream(s_out)  # the last download is part of the step
+        e2.record(s_in)
         torch.cuda.synchronize()
         e_ms = bldist.max_over_ranks(s2.elapsed_time(e2), dist, device)
         e2e = {"value": M * e2e_steps * world / (e_ms * 1e-3), "unit": "tokens/s",
                "h2d_bytes_per_step": x_h.numel() * x_h.element_size(),
-               "d2h_bytes_per_step": y_h.numel() * y_h.element_size(), "steps": e2e_steps}
+               "d2h_bytes_per_step": y_hs[0].numel() * y_hs[0].element_size(),
+               "steps": e2e_steps, "overlap": "upload, forward and download on three streams"}
 
     if dist is not None:
         dist.barrier()
