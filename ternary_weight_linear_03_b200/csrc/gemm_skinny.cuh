@@ -91,6 +91,7 @@ struct Barriers {
   int last;
   int rowsum[MAX_M];  // per token, staged once for the epilogue
   float f[MAX_M];     // per token s_t * gamma
+  unsigned tmax[MAX_M];  // per token, this CTA's largest |y| (bits), for a chain's next layer
 };
 
 // The mbarriers above, w_full through drain, are consecutive 8-byte words.
@@ -214,6 +215,13 @@ __device__ __forceinline__ void red_max_u32(float* p, unsigned bits) {
   asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" ::"l"(p), "r"(bits) : "memory");
 }
 
+// The warp's largest |y| for token t (all 32 lanes call it with their own value) merged into
+// the CTA's tmax[t] (shared memory) by lane 0; the CTA adds tmax into the global absmax
+// once per token at the end, so the global atomics do not pile up on the M addresses.
+__device__ __forceinline__ void warp_amax_smem(unsigned* tmax, int t, unsigned bits) {
+  const unsigned m = __reduce_max_sync(0xffffffffu, bits);
+  if ((threadIdx.x & 31) == 0 && m != 0u) atomicMax(tmax + t, m);
+}
 // The warp's largest |y| for token t (all 32 lanes call it with their own value) added
 // into amax_out[t] by lane 0.
 __device__ __forceinline__ void warp_amax_out(float* amax_out, int t, unsigned bits) {
@@ -228,7 +236,7 @@ __device__ __forceinline__ void warp_amax_out(float* amax_out, int t, unsigned b
 template <int OM>
 __device__ __forceinline__ void epi_store_chunk(const int (&a)[16], const float (&fs)[16], int c0,
                                                 int M, int N, int n0, bool nvalid, bool vec,
-                                                unsigned char* stage, void* y, float* amax_out) {
+                                                unsigned char* stage, void* y, unsigned* tmax) {
   constexpr int ES = (OM == 1) ? 2 : 4;  // bytes per element of y
   const int nl = threadIdx.x;            // row within the tile
   const int n = n0 + nl;
@@ -261,12 +269,12 @@ __device__ __forceinline__ void epi_store_chunk(const int (&a)[16], const float 
       }
     }
   }
-  if (OM != 2 && amax_out != nullptr) {
+  if (OM != 2 && tmax != nullptr) {
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
       if (c0 + j < M) {  // the same for the whole warp
         const uint32_t mag = (OM == 0) ? (bits[j] & 0x7fffffffu) : ((bits[j] << 16) & 0x7fffffffu);
-        warp_amax_out(amax_out, c0 + j, nvalid ? mag : 0u);
+        warp_amax_smem(tmax, c0 + j, nvalid ? mag : 0u);
       }
     }
   }
@@ -538,9 +546,11 @@ __global__ void __launch_bounds__(sk::THREADS, 2) gemm_skinny_kernel(
         for (int t = threadIdx.x; t < M; t += 128) {
           bar->rowsum[t] = rowsum[t];
           bar->f[t] = (OM == 2) ? 0.0f : __fmul_rn(scale[t], gamma);
+          bar->tmax[t] = 0u;
         }
       }
       epi_bar_sync();
+      unsigned* tmax = (OM != 2 && amax_out != nullptr) ? bar->tmax : nullptr;
       tc_fence_after();
       const int n = n0 + warp * 32 + lane;  // this thread's TMEM lane = weight row
       const bool nvalid = n < N;
@@ -564,7 +574,7 @@ __global__ void __launch_bounds__(sk::THREADS, 2) gemm_skinny_kernel(
           int a[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) a[j] = static_cast<int>(v[j]) - rs[j];
-          epi_store_chunk<OM>(a, fs, c0, M, N, n0, nvalid, vec, stage, y, amax_out);
+          epi_store_chunk<OM>(a, fs, c0, M, N, n0, nvalid, vec, stage, y, tmax);
         }
       } else {
         // exact int32 partial of this split, added into acc32[t][n] (zeroed by the host)
@@ -607,10 +617,15 @@ __global__ void __launch_bounds__(sk::THREADS, 2) gemm_skinny_kernel(
             }
 #pragma unroll
             for (int j = 0; j < 16; ++j) a[j] -= rs[j];
-            epi_store_chunk<OM>(a, fs, t0, M, N, n0, nvalid, vec, stage, y, amax_out);
+            epi_store_chunk<OM>(a, fs, t0, M, N, n0, nvalid, vec, stage, y, tmax);
           }
           if (threadIdx.x == 0) counters[tile] = 0u;  // every split has arrived
         }
+      }
+      if (tmax != nullptr) {  // this CTA's per-token maxima into the chain's absmax
+        epi_bar_sync();
+        for (int t = threadIdx.x; t < M; t += 128)
+          if (tmax[t] != 0u) red_max_u32(amax_out + t, tmax[t]);
       }
     }
   }
