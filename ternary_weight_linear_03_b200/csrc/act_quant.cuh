@@ -75,19 +75,20 @@ __device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
 // patterns: with the sign cleared, bf16 patterns order like their values, and the NaN
 // patterns lie above infinity (0x7f80), so a maximum at or above 0x7f80 flags a
 // non-finite value.
-__device__ __forceinline__ uint32_t absmax16_bf16(const void* p, uint32_t m2) {
-  const uint4 a = reinterpret_cast<const uint4*>(p)[0], b = reinterpret_cast<const uint4*>(p)[1];
+__device__ __forceinline__ uint32_t absmax16_bf16(const uint4 a, const uint4 b, uint32_t m2) {
   const uint32_t h[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
   for (int q = 0; q < 8; ++q) m2 = max_u16x2(m2, h[q] & 0x7fff7fffu);
   return m2;
 }
+__device__ __forceinline__ uint32_t absmax16_bf16(const void* p, uint32_t m2) {
+  return absmax16_bf16(reinterpret_cast<const uint4*>(p)[0], reinterpret_cast<const uint4*>(p)[1], m2);
+}
 
 // Quantizes 16 bf16 values with a finite r (the same rounding and clamping as quant_i8;
 // its zero test only matters for an infinite r) into four words of int8, byte i & 3 of
 // word i >> 2 holding element i, and adds their sum into *sum.
-__device__ __forceinline__ uint4 quant16_bf16(const void* p, float r, int* sum) {
-  const uint4 a = reinterpret_cast<const uint4*>(p)[0], b = reinterpret_cast<const uint4*>(p)[1];
+__device__ __forceinline__ uint4 quant16_bf16(const uint4 a, const uint4 b, float r, int* sum) {
   const uint32_t h[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
   uint32_t w[4];
 #pragma unroll
@@ -103,6 +104,9 @@ __device__ __forceinline__ uint4 quant16_bf16(const void* p, float r, int* sum) 
     *sum = __dp4a(static_cast<int>(w[j]), 0x01010101, *sum);
   }
   return make_uint4(w[0], w[1], w[2], w[3]);
+}
+__device__ __forceinline__ uint4 quant16_bf16(const void* p, float r, int* sum) {
+  return quant16_bf16(reinterpret_cast<const uint4*>(p)[0], reinterpret_cast<const uint4*>(p)[1], r, sum);
 }
 
 // Zeroes n16 16-byte words at z with the whole grid (the split-K sums and counters of the

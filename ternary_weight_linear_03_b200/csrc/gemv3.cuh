@@ -20,7 +20,8 @@
 // Structure as the 2-bit GEMV: the M (<= 4) tokens are quantized in the prologue into
 // shared memory in natural order (zero beyond K up to the chunk boundary); LPR lanes share
 // a weight row, each streaming its 16-byte chunks with no-allocate loads, and the lanes of
-// a row reduce with shuffles.
+// a row reduce with shuffles. Warps take rows in turns, numbered across the grid as the
+// 2-bit GEMV numbers them (warp w of block b is w * grid + b).
 #pragma once
 
 #include "act_quant.cuh"
@@ -173,7 +174,7 @@ __global__ void __launch_bounds__(kGemv3Threads) gemv3_kernel(
   const int rsel = lane >> lpr_log2;
   const long long warps_total = static_cast<long long>(gridDim.x) * kGemv3Warps;
   const long long row_bytes = 16ll * CH;
-  for (long long rg = static_cast<long long>(blockIdx.x) * kGemv3Warps + warp; rg * RPW < N;
+  for (long long rg = static_cast<long long>(warp) * gridDim.x + blockIdx.x; rg * RPW < N;
        rg += warps_total) {
     const long long n = rg * RPW + rsel;
     const bool valid = n < N;
