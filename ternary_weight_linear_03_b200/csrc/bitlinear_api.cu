@@ -288,7 +288,15 @@ bl_status launch_gemv_t(const void* x, const uint8_t* packed, const float* gamma
   const int lpr_log2 = gemv_lpr_log2(K / 64, N, MT);
   const long long rows_per_block = static_cast<long long>(bl::kGemvWarps) * (32 >> lpr_log2) * R;
   const long long need = (N + rows_per_block - 1) / rows_per_block;
-  const int grid = static_cast<int>(std::min<long long>(need, 1ll * blocks_per_sm * num_sms()));
+  const long long slots = 1ll * blocks_per_sm * num_sms();
+  const long long rpw = 32 >> lpr_log2;  // rows of one warp turn
+  // The register path hands rows out block by block: just enough blocks. The shared-memory
+  // path numbers warps across the grid, so it takes the same number of blocks on every SM
+  // (every resident slot, or one per SM when fewer blocks would do) and the rows spread
+  // evenly over them.
+  const int grid = static_cast<int>(
+      XR ? std::min(need, slots)
+         : (need > num_sms() ? slots : std::min<long long>(num_sms(), (N + rpw - 1) / rpw)));
   const int chain = o.pdl ? 1 : 0;
   return launch_ex(kern, dim3(grid), dim3(bl::kGemvThreads), smem, s, o.pdl, x, packed, gamma,
                    y, N, K, lpr_log2, o.amax_in, o.amax_out, chain);
@@ -362,7 +370,11 @@ bl_status launch_gemv3_t(const void* x, const uint8_t* packed3, const float* gam
   const int lpr_log2 = choose_lpr_log2(CH);
   const long long rows_per_block = static_cast<long long>(bl::kGemv3Warps) * (32 >> lpr_log2);
   const long long need = (N + rows_per_block - 1) / rows_per_block;
-  const int grid = static_cast<int>(std::min<long long>(need, 1ll * blocks_per_sm * num_sms()));
+  // warps numbered across the grid: the same number of blocks on every SM (as the 2-bit
+  // GEMV's shared-memory path)
+  const int grid = static_cast<int>(
+      need > num_sms() ? 1ll * blocks_per_sm * num_sms()
+                       : std::min<long long>(num_sms(), (N + (32 >> lpr_log2) - 1) / (32 >> lpr_log2)));
   kern<<<grid, bl::kGemv3Threads, smem, s>>>(x, packed3, gamma, y, N, K, lpr_log2);
   return launch_status();
 }
