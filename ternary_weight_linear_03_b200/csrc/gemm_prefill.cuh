@@ -389,14 +389,9 @@ __global__ void __launch_bounds__(pf::THREADS, 1) gemm_prefill_kernel(
             }
           }
           if (OM != 2 && amax_out != nullptr) {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const int t = t0 + c0 + hh + j;
-              if (t < M) {  // the same for the whole warp
-                const uint32_t mag = (OM == 0) ? (bits[j] & 0x7fffffffu) : ((bits[j] << 16) & 0x7fffffffu);
-                warp_amax_out(amax_out, t, nvalid ? mag : 0u);
-              }
-            }
+            const unsigned m = warp_amax16<OM>(bits, nvalid);
+            const int t = t0 + c0 + hh + lane;
+            if (lane < 16 && t < M && m != 0u) red_max_u32(amax_out + t, m);
           }
         }
       }

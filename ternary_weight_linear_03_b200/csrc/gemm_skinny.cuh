@@ -215,18 +215,23 @@ __device__ __forceinline__ void red_max_u32(float* p, unsigned bits) {
   asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" ::"l"(p), "r"(bits) : "memory");
 }
 
-// The warp's largest |y| for token t (all 32 lanes call it with their own value) merged into
-// the CTA's tmax[t] (shared memory) by lane 0; the CTA adds tmax into the global absmax
-// once per token at the end, so the global atomics do not pile up on the M addresses.
-__device__ __forceinline__ void warp_amax_smem(unsigned* tmax, int t, unsigned bits) {
-  const unsigned m = __reduce_max_sync(0xffffffffu, bits);
-  if ((threadIdx.x & 31) == 0 && m != 0u) atomicMax(tmax + t, m);
-}
-// The warp's largest |y| for token t (all 32 lanes call it with their own value) added
-// into amax_out[t] by lane 0.
-__device__ __forceinline__ void warp_amax_out(float* amax_out, int t, unsigned bits) {
-  const unsigned m = __reduce_max_sync(0xffffffffu, bits);
-  if ((threadIdx.x & 31) == 0 && m != 0u) red_max_u32(amax_out + t, m);
+// The warp's largest |y| of each of 16 tokens, for a layer chain's next quantization.
+// bits[j] is this lane's stored value of token j (fp32 or bf16 bits), valid whether the
+// lane's row exists. Sixteen reductions with no branch between them (a branch holding an
+// atomic inside this loop made every reduction wait for the atomic before it, about 3.5 us
+// per 3B-sized layer at 64 tokens); lane j < 16 returns the maximum of token j as float
+// bits, the other lanes 0. The caller adds it with one atomic per lane.
+template <int OM>
+__device__ __forceinline__ unsigned warp_amax16(const uint32_t (&bits)[16], bool valid) {
+  const int lane = threadIdx.x & 31;
+  unsigned mine = 0u;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const uint32_t mag = (OM == 0) ? (bits[j] & 0x7fffffffu) : ((bits[j] << 16) & 0x7fffffffu);
+    const unsigned r = __reduce_max_sync(0xffffffffu, valid ? mag : 0u);
+    mine = (lane == j) ? r : mine;
+  }
+  return mine;
 }
 
 // Rescales and writes the 16 values of tokens c0 .. c0 + 15 of this thread's weight row
@@ -269,14 +274,10 @@ __device__ __forceinline__ void epi_store_chunk(const int (&a)[16], const float 
       }
     }
   }
-  if (OM != 2 && tmax != nullptr) {
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      if (c0 + j < M) {  // the same for the whole warp
-        const uint32_t mag = (OM == 0) ? (bits[j] & 0x7fffffffu) : ((bits[j] << 16) & 0x7fffffffu);
-        warp_amax_smem(tmax, c0 + j, nvalid ? mag : 0u);
-      }
-    }
+  if (OM != 2 && tmax != nullptr) {  // into the CTA's per-token maxima in shared memory
+    const unsigned m = warp_amax16<OM>(bits, nvalid);
+    const int lane = threadIdx.x & 31;
+    if (lane < 16 && c0 + lane < M && m != 0u) atomicMax(tmax + c0 + lane, m);
   }
   if (vec) {
     epi_bar_sync();
