@@ -166,9 +166,21 @@ __global__ void __launch_bounds__(NT) act_quant_kernel(
       return m;
     };
     if (kBf16) {  // K % 16 == 0: one max.u16x2 per two values
+      // two groups' loads in flight per thread before either is reduced
       uint32_t m2 = 0u;
-      for (int c = threadIdx.x; c < K / 16; c += blockDim.x)
-        m2 = absmax16_bf16(row + 32 * static_cast<size_t>(c), m2);
+      const int ng = K / 16;
+      for (int c0 = threadIdx.x; c0 < ng; c0 += 2 * blockDim.x) {
+        uint4 v[2][2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int c = c0 + u * blockDim.x;
+          const uint4* p = reinterpret_cast<const uint4*>(row + 32 * static_cast<size_t>(c));
+          v[u][0] = (c < ng) ? p[0] : make_uint4(0u, 0u, 0u, 0u);
+          v[u][1] = (c < ng) ? p[1] : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) m2 = absmax16_bf16(v[u][0], v[u][1], m2);
+      }
       const uint32_t m = max(m2 & 0xffffu, m2 >> 16);
       a = (m < 0x7f80u) ? __uint_as_float(m << 16) : float_pass();
     } else {
