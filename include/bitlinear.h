@@ -190,8 +190,10 @@ size_t bitlinear_chain_workspace_size(int M, const bl_layer* layers, int L);
  * is a single pass (or part of the GEMV's prologue); every kernel is launched with
  * programmatic dependent launch, so it sets up, and prefetches its packed weights (TMA
  * into shared memory, or into L2), while the kernel before it still runs. Capture the call
- * in a CUDA graph to take the host out of the loop. Results equal layer-by-layer
- * bitlinear_forward calls with bf16 intermediates, bit for bit.
+ * in a CUDA graph to take the host out of the loop. The skinny kernel's K splits may
+ * exchange int32 sums up to the packed weight bytes here (a quarter in bitlinear_forward):
+ * the chain clears its sums once per call and every kernel leaves them cleared. Results
+ * equal layer-by-layer bitlinear_forward calls with bf16 intermediates, bit for bit.
  *   x       device [M][K of the layers with src = -1], fp32 or bf16.
  *   layers  host array of L layers; K of a layer with src = j equals N of layer j.
  *   y       device [M][N of the last layer], BL_F32 or BL_BF16.

@@ -110,7 +110,11 @@ struct SkinnyPlan {
   int splits;  // K ranges per tile
   int kbps;    // 128-wide K blocks per split
 };
-SkinnyPlan skinny_plan_for(int M, int N, int K, int sms) {
+// sums_share: the int32 sums of one split may reach 1/sums_share of the packed weight bytes
+// (4 for a single forward, whose quantization kernel clears the sums on every call; 1
+// inside a layer chain, which clears them once per call and whose kernels leave them
+// cleared).
+SkinnyPlan skinny_plan_for(int M, int N, int K, int sms, int sums_share = 4) {
   SkinnyPlan p{};
   p.bnt = (M + 15) / 16 * 16;
   p.tiles = (N + bl::sk::BW - 1) / bl::sk::BW;
@@ -120,13 +124,16 @@ SkinnyPlan skinny_plan_for(int M, int N, int K, int sms) {
   // runs at the pace of its handoffs, so a second wave would double the time. Keep at
   // least kMinKbPerSplit K blocks per split so that each CTA streams long enough to cover
   // its fixed costs, and keep the int32 sums the splits exchange (M x N x 4 bytes each)
-  // within a quarter of the packed weight bytes (measured on B200: beyond that the
-  // reduction costs more than the extra SMs bring).
+  // within 1/sums_share of the packed weight bytes (measured on B200, single forwards:
+  // beyond a quarter, clearing and reducing the sums costs more than the extra SMs bring;
+  // in a chain, which clears them only once, up to the weight bytes paid: 3B sweep at 64
+  // tokens 1.35 -> 1.32 ms).
   const long long slots = static_cast<long long>(p.bnt <= 64 ? 2 : 1) * sms;
   long long splits = 1;
   if (p.tiles < slots) splits = std::max<long long>(1, slots / p.tiles);
   const long long by_traffic = static_cast<long long>(
-      (static_cast<double>(N) * K / 4.0) / (4.0 * 4.0 * static_cast<double>(M) * N));
+      (static_cast<double>(N) * K / 4.0) /
+      (static_cast<double>(sums_share) * 4.0 * static_cast<double>(M) * N));
   splits = std::max<long long>(
       1, std::min<long long>({splits, std::max(1, KB / kMinKbPerSplit), by_traffic}));
   p.kbps = static_cast<int>((KB + splits - 1) / splits);
@@ -135,6 +142,9 @@ SkinnyPlan skinny_plan_for(int M, int N, int K, int sms) {
   return p;
 }
 SkinnyPlan skinny_plan(int M, int N, int K) { return skinny_plan_for(M, N, K, num_sms()); }
+SkinnyPlan skinny_plan_chain(int M, int N, int K) {
+  return skinny_plan_for(M, N, K, num_sms(), 1);
+}
 
 // Workspace of the skinny path: the FwdWs part, then (only when splits > 1) the int32
 // sums [M][N] and one arrival counter per weight tile, contiguous so one memset clears
@@ -959,7 +969,7 @@ bl_status chain_plan(int M, const bl_layer* layers, int L, ChainPlan* plan) {
   for (int l = 0; l < L; ++l) {
     const bl_layer& ly = layers[l];
     if (!use_gemv(M, ly.N, ly.K) && M <= kSkinnyMaxM) {
-      const SkinnyPlan sp = skinny_plan(M, ly.N, ly.K);
+      const SkinnyPlan sp = skinny_plan_chain(M, ly.N, ly.K);
       if (sp.splits > 1) part = std::max(part, static_cast<size_t>(M) * ly.N * 4);
       tiles = std::max(tiles, static_cast<size_t>(sp.tiles));
     }
@@ -1042,7 +1052,7 @@ bl_status bitlinear_chain_forward(const void* x, int x_dtype, int M, const bl_la
       quantized[j] = 1;
     }
     if (M <= kSkinnyMaxM) {
-      const SkinnyPlan sp = skinny_plan(M, ly.N, ly.K);
+      const SkinnyPlan sp = skinny_plan_chain(M, ly.N, ly.K);
       SkinnyWs sw{};
       sw.partial = reinterpret_cast<int*>(base + p.partial_off);
       sw.counters = reinterpret_cast<unsigned int*>(base + p.counters_off);

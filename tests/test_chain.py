@@ -116,12 +116,14 @@ def test_ffn_chain_matches_oracle_layer_by_layer(M, x_dtype, out):
 
 
 @pytest.mark.gpu
-def test_chain_equals_separate_forwards_and_repeats():
+@pytest.mark.parametrize("M", [16, 64])
+def test_chain_equals_separate_forwards_and_repeats(M):
     """The chain gives the bits of separate bitlinear_forward calls; a second call on the
-    same workspace (whose absmax and split-K sums start from what the first left) agrees."""
+    same workspace (whose absmax and split-K sums start from what the first left) agrees.
+    At 64 tokens the chain splits K where a single forward does not."""
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
-    M, d, h = 16, 3200, 8640  # the 3B feed-forward shapes; K is split on these
+    d, h = 3200, 8640  # the 3B feed-forward shapes
     gate_out = [torch.empty((M, h), dtype=torch.bfloat16, device="cuda")]
     layers = _ffn_chain(1, d, h, 0.02, "cuda", gate_out)
     x = syn.activations(M, d, seed=5).cuda()
