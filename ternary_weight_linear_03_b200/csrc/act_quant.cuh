@@ -4,7 +4,7 @@
 //   q[t,k] = clip(rne(fl(x[t,k] * r_t)), -127, 127)   (0 when a_t == 0 or x == 0).
 // One block per token row; the row is read once from HBM (the second pass hits L1/L2).
 // Optionally also writes rowsum_t = sum_k q[t,k], which the tensor-core GEMM subtracts
-// from its accumulators (the packed weights are stored as c + 1, see gemm_tc.cuh).
+// from its accumulators (trit c is stored as u = c + 1, so sum_k u q = acc + sum_k q).
 #pragma once
 
 #include "common.cuh"

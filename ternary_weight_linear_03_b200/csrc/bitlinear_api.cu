@@ -18,7 +18,6 @@
 #include "gemm_bf16.cuh"
 #include "gemm_prefill.cuh"
 #include "gemm_skinny.cuh"
-#include "gemm_tc.cuh"
 #include "gemv.cuh"
 #include "gemv3.cuh"
 #include "per_device.h"

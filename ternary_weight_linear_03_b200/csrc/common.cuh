@@ -232,4 +232,22 @@ __device__ __forceinline__ int quant_i8(float v, float r) {
   return max(-127, min(127, c));
 }
 
+// Bounded wait that also gives up when another role has already aborted.
+__device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
+                                        volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if (global_ns() - t0 > limit_ns) {
+      record_status(kStatusTimeout);
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
 }  // namespace bl

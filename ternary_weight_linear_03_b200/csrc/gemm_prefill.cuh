@@ -47,7 +47,6 @@
 
 #include "common.cuh"
 #include "gemm_skinny.cuh"
-#include "gemm_tc.cuh"
 
 namespace bl {
 

@@ -52,7 +52,6 @@
 #include <cstddef>
 
 #include "common.cuh"
-#include "gemm_tc.cuh"
 
 namespace bl {
 
